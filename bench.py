@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark of the KDN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {kdn,reference}]
+
+A step is one Isotropic KDN layer forward (kdn_iso_forward) over the whole
+1.3B-layer-shaped workload: B=8, T=4096, H=16, d_k=d_v=128, bf16 q/k/v, fp32
+decay / noise / state / output, inputs resident in HBM.  It covers the whole
+hot path: per-token variance recursion, gains, chunkwise delta-rule engine,
+outputs and final state.  Inputs (403 MB of q/k/v) are larger than the 126 MB
+L2, so no flush is needed between steps.  Prints ONE JSON line (rank 0).
+
+Also measured on the same run and reported under "secondary": the Diagonal
+KDN forward at the same shape, the standalone variance scan (4096 x 65536),
+the long-context diagonal forward (B1 T65536) and the decode step (batch 256).
+
+--impl reference times the fp64 CPU oracle (the correctness reference) on a
+bounded sample of the same workload on the host cores.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of
+the workload; (b, h) heads are independent, so there is no collective on the
+data path ("weak" scaling).  Time is the max over ranks of each rank's
+CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = 'KDN layer fwd tokens/s (B8 T4096 H16 d128)'
+WORKLOAD = 'iso_1p3b'
+
+
+def peaks():
+    path = os.path.join(ROOT, 'MEASURED_PEAKS.json')
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p['hbm_gbs']), float(p['bf16_tflops']), 'measured'
+    return 6650.0, 1590.0, 'fallback'
+
+
+def layer_bytes(variant, B, T, H, dk, dv, in_bytes=2):
+    """Algorithmic HBM bytes of one layer forward: read q, k, v, a, w, r;
+    write o (fp32), S_T, p_T (S0 = 0 and p0 = 1 are not read)."""
+    qkv = B * T * H * (2 * dk + dv) * in_bytes
+    ar = 2 * B * T * H * 4
+    w = B * T * H * (dk if variant == 'diag' else 1) * 4
+    o = B * T * H * dv * 4
+    st = B * H * dv * dk * 4 + B * H * (dk if variant == 'diag' else 1) * 4
+    return qkv + ar + w + o + st
+
+
+def decode_bytes(B, H, dk, dv):
+    """Per decode step (diagonal): S read+write, p read+write, q/k/v bf16,
+    a/r, per-dimension w, o fp32."""
+    return (2 * B * H * dv * dk * 4 + 2 * B * H * dk * 4 + B * H * (2 * dk + dv) * 2 +
+            2 * B * H * 4 + B * H * dk * 4 + B * H * dv * 4)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    FIELDS = ('clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,'
+              'clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,'
+              'clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap')
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def _once(self):
+        try:
+            out = subprocess.run(['nvidia-smi', '-i', str(self.gpu), '--query-gpu=' + self.FIELDS,
+                                  '--format=csv,noheader,nounits'], capture_output=True,
+                                 text=True, timeout=10)
+            return out.stdout.strip().splitlines()
+        except Exception:
+            return []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ['nvidia-smi', '-i', str(self.gpu), '--query-gpu=' + self.FIELDS,
+                 '--format=csv,noheader,nounits', '-lms', '100'],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=10)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        if not self.lines:
+            self.lines = self._once()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ['hw_slowdown', 'hw_thermal_slowdown', 'sw_thermal_slowdown', 'sw_power_cap']
+        for line in self.lines:
+            f = [x.strip() for x in line.split(',')]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == 'active':
+                    reasons.add(n)
+        if not sm:
+            return {'sm_mhz': None, 'sm_max_mhz': None, 'reasons': ['unavailable'], 'samples': 0}
+        return {'sm_mhz': statistics.median(sm), 'sm_max_mhz': smax, 'reasons': sorted(reasons),
+                'samples': len(sm)}
+
+
+def time_launches(fn, steps, warmup, stream):
+    """CUDA-event time (ms) of `steps` back-to-back calls of fn on `stream`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+# ---------------------------------------------------------------- reference
+def run_reference(args, rank):
+    """The fp64 CPU oracle on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    from kalman_filter_linear_b200 import synth
+    from oracle import kdn_ref
+    cfg = synth.WORKLOADS[WORKLOAD]
+    B, T, H, d = cfg['B'], cfg['T'], cfg['H'], cfg['dk']
+    x = synth.layer_inputs(B, T, H, d, d, 'iso', cfg['seed'], cfg['dtype'])
+    tok = 16  # tokens of all B*H heads per step: a bounded sample of the workload
+    xs = {k: x[k][:, :tok].double().numpy() for k in 'qkvawr'}
+    for _ in range(args.warmup):
+        kdn_ref.iso_forward(*(xs[n] for n in 'qkvawr'))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        kdn_ref.iso_forward(*(xs[n] for n in 'qkvawr'))
+    el = time.perf_counter() - t0
+    value = B * tok * args.steps / el
+    print(json.dumps({
+        'impl': 'reference', 'metric': METRIC, 'value': value, 'unit': 'tokens/s',
+        'n_gpus': args.gpus, 'steps': args.steps, 'warmup': args.warmup,
+        'ms_per_step': 1000 * el / args.steps, 'higher_is_better': True, 'scaling': 'weak',
+        'vs_baseline': None, 'dtype': 'f64', 'data': 'synthetic',
+        'config': {'workload': WORKLOAD, 'B': B, 'T': T, 'H': H, 'dk': d, 'dv': d,
+                   'sample': f'first {tok} tokens of all {B}x{H} heads per step'},
+        'cpu_baseline': {'value': value, 'unit': 'tokens/s', 'cores': 1, 'kind': 'oracle',
+                         'sample': f'{tok} tokens x {B * H} heads per step, fp64 NumPy, '
+                                   'single-threaded elementwise/einsum'},
+        'e2e': {'value': value, 'unit': 'tokens/s', 'h2d_bytes_per_step': 0,
+                'd2h_bytes_per_step': 0}}))
+
+
+def cpu_baseline(seconds=12.0):
+    """Time the oracle as it stands on a bounded sample of the workload."""
+    import torch
+    from kalman_filter_linear_b200 import synth
+    from oracle import kdn_ref
+    cfg = synth.WORKLOADS[WORKLOAD]
+    B, T, H, d = cfg['B'], cfg['T'], cfg['H'], cfg['dk']
+    x = synth.layer_inputs(B, 64, H, d, d, 'iso', cfg['seed'], cfg['dtype'])
+    xs = {k: x[k].double().numpy() for k in 'qkvawr'}
+    tok = 0
+    t0 = time.perf_counter()
+    S = p = None
+    while time.perf_counter() - t0 < seconds:
+        sl = slice(tok % 64, tok % 64 + 8)
+        _, S, p = kdn_ref.iso_forward(*(xs[n][:, sl] for n in 'qkvawr'), S0=S, p0=p)
+        tok += 8
+    el = time.perf_counter() - t0
+    return {'value': B * tok / el, 'unit': 'tokens/s', 'cores': 1, 'kind': 'oracle',
+            'sample': f'{tok} tokens of all {B}x{H} heads (B8 H16 d128), fp64 NumPy '
+                      f'token loop, single-threaded, {el:.1f} s'}
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument('--gpus', type=int, default=1)
+    ap.add_argument('--steps', type=int, default=50)
+    ap.add_argument('--warmup', type=int, default=5)
+    ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
+    ap.add_argument('--no-secondary', action='store_true')
+    ap.add_argument('--no-cpu-baseline', action='store_true')
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get('RANK', '0'))
+    world = int(os.environ.get('WORLD_SIZE', '1'))
+    local = int(os.environ.get('LOCAL_RANK', '0'))
+    if args.impl == 'reference':
+        run_reference(args, rank)
+        return
+
+    import torch
+    from kalman_filter_linear_b200 import kdn, synth
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group('nccl', timeout=datetime.timedelta(seconds=120))
+    dev = torch.device('cuda', local)
+    stream = torch.cuda.current_stream()
+    hbm_peak, tf_peak, peak_kind = peaks()
+
+    cfg = synth.WORKLOADS[WORKLOAD]
+    B, T, H, d = cfg['B'], cfg['T'], cfg['H'], cfg['dk']
+    host = synth.layer_inputs(B, T, H, d, d, 'iso', cfg['seed'] + 1000 * rank, cfg['dtype'])
+    x = {k: v.to(dev) for k, v in host.items()}
+    ws = torch.empty(max(kdn.kdn_forward_workspace_size(kdn.KDN_ISO, B, T, H, d, d), 256),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, d), dtype=torch.float32, device=dev)
+    S_out = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    p_out = torch.empty((B, H), dtype=torch.float32, device=dev)
+
+    def step():
+        kdn.kdn_iso_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], o=o, S_out=S_out,
+                            p_out=p_out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        ms = time_launches(step, args.steps, 0, stream)
+    if dist:
+        dist.barrier()
+    t = torch.tensor([ms], device=dev)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    ms_step = ms_max / args.steps
+    value = world * B * T / (ms_step / 1000.0)
+    alg = layer_bytes('iso', B, T, H, d, d)
+    achieved = alg / (ms / args.steps / 1000.0) / 1e9
+
+    # ---- end to end through the public API: pinned host in, result out
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    o_host = torch.empty((B, T, H, d), dtype=torch.float32).pin_memory()
+    S_host = torch.empty((B, H, d, d), dtype=torch.float32).pin_memory()
+    p_host = torch.empty((B, H), dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = o_host.numel() * 4 + S_host.numel() * 4 + p_host.numel() * 4
+
+    def e2e_step():
+        for k in x:
+            x[k].copy_(pinned[k], non_blocking=True)
+        step()
+        o_host.copy_(o, non_blocking=True)
+        S_host.copy_(S_out, non_blocking=True)
+        p_host.copy_(p_out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    ms_e2e = time_launches(e2e_step, e2e_steps, 2, stream) / e2e_steps
+    te = torch.tensor([ms_e2e], device=dev)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * B * T / (float(te.item()) / 1000.0)
+
+    secondary = {}
+    if not args.no_secondary and rank == 0:
+        secondary = measure_secondary(kdn, synth, dev, stream, hbm_peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        'metric': METRIC, 'value': value, 'unit': 'tokens/s', 'n_gpus': world,
+        'steps': args.steps, 'warmup': args.warmup, 'ms_per_step': ms_step,
+        'higher_is_better': True, 'scaling': 'weak', 'vs_baseline': None, 'dtype': 'bf16',
+        'data': 'synthetic',
+        'config': {'workload': WORKLOAD, 'B': B, 'T': T, 'H': H, 'dk': d, 'dv': d,
+                   'chunk': 64, 'inputs': 'q/k/v bf16, a/w/r fp32, S0=0, p0=1',
+                   'outputs': 'o fp32 [B,T,H,dv], S_T fp32, p_T fp32',
+                   'arithmetic': 'bf16 hi/lo tensor-core operands, fp32 accumulate, '
+                                 'state and variance',
+                   'l2': 'inputs (403 MB q/k/v) larger than the 126 MB L2; no flush',
+                   'parallelism': f'dp{world} (independent replicas, no collective)'},
+        'roofline': {'bound': 'hbm', 'achieved': achieved, 'peak': hbm_peak, 'unit': 'GB/s',
+                     'frac': achieved / hbm_peak, 'traffic': None,
+                     'algorithmic_bytes': alg, 'peak_source': peak_kind},
+        'e2e': {'value': e2e_value, 'unit': 'tokens/s', 'h2d_bytes_per_step': h2d,
+                'd2h_bytes_per_step': d2h},
+        'gpu_launches': args.steps,
+        'clocks': clk.summary(),
+        'cpu_baseline': cpu,
+        'secondary': secondary,
+    }
+    print(json.dumps(line))
+
+
+def measure_secondary(kdn, synth, dev, stream, hbm_peak):
+    import torch
+    out = {}
+    # diagonal forward, same shape
+    c = synth.WORKLOADS['diag_1p3b']
+    B, T, H, d = c['B'], c['T'], c['H'], c['dk']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'diag', c['seed'],
+                                                     c['dtype']).items()}
+    ws = torch.empty(max(kdn.kdn_forward_workspace_size(kdn.KDN_DIAG, B, T, H, d, d), 256),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((B, T, H, d), dtype=torch.float32, device=dev)
+    S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    p = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    f = lambda: kdn.kdn_diag_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], o=o,
+                                     S_out=S, p_out=p, workspace=ws)
+    n = 10
+    ms = time_launches(f, n, 3, stream) / n
+    alg = layer_bytes('diag', B, T, H, d, d)
+    out['diag_1p3b'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms,
+                        'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                        'algorithmic_bytes': alg}
+    del x, o, S, p
+    # standalone variance scan
+    c = synth.WORKLOADS['scan']
+    N, Tn = c['N'], c['T']
+    xs = {k: v.to(dev) for k, v in synth.scan_inputs(N, Tn, c['seed']).items()}
+    lam = torch.empty_like(xs['a'])
+    wss = torch.empty(kdn.kdn_mobius_scan_workspace_size(N, Tn), dtype=torch.uint8, device=dev)
+    f = lambda: kdn.kdn_mobius_scan(xs['a'], xs['w'], xs['r'], xs['n'], None, c['info_scale'],
+                                    lambda_out=lam, workspace=wss)
+    ms = time_launches(f, n, 3, stream) / n
+    alg = N * Tn * 20
+    out['scan'] = {'steps_per_s': N * Tn / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
+                   'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg}
+    del xs, lam, wss
+    # decode step, batch 256, diagonal
+    c = synth.WORKLOADS['diag_long']
+    Bd, H, d = c['decode_batch'], c['H'], c['dk']
+    st = synth.decode_state(Bd, H, d, d, 'diag', seed=c['seed'])
+    Sd, pd = st['S'].to(dev), st['p'].to(dev)
+    xd = {k: v.to(dev) for k, v in synth.decode_inputs(Bd, H, d, d, 'diag', c['seed']).items()}
+    od = torch.empty((Bd, H, d), dtype=torch.float32, device=dev)
+    f = lambda: kdn.kdn_decode_step('diag', xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'],
+                                    Sd, pd, o=od)
+    n = 50
+    ms = time_launches(f, n, 5, stream) / n
+    alg = decode_bytes(Bd, H, d, d)
+    out['decode'] = {'tokens_per_s': Bd / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
+                     'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg}
+    return out
+
+
+if __name__ == '__main__':
+    main()

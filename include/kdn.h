@@ -1,0 +1,198 @@
+/*
+ * kdn.h -- C ABI of libkdn, the B200 (sm_100a) Kalman Delta Network layer.
+ *
+ * The model (from "Kalman Delta Networks: Uncertainty-aware Associative
+ * Memory", abstract, and "Kalman Delta Networks: 不确定性感知的联想记忆",
+ * 方法): per batch element b and head h the memory S (d_v x d_k) is the
+ * latent state of a linear-Gaussian model, S_t = a_t S_{t-1} + noise(w_t)
+ * and v_t = S_t k_t + noise(r_t).  Each token predicts, then writes the
+ * residual v_t - a_t S_{t-1} k_t with the Kalman gain g_t, then reads
+ * o_t = S_t q_t.  The uncertainty is one variance per head (Isotropic KDN)
+ * or per key dimension (Diagonal KDN); both follow the Mobius map
+ *     p_t = (r a^2 p_{t-1} + r w) / (c a^2 p_{t-1} + r + c w)
+ * with c = info_scale * ||k_t||^2 (iso) or c = k_{t,i}^2 (diag).
+ *
+ * Conventions for every call:
+ *   - Pointers are caller-owned.  Device pointers unless stated otherwise
+ *     (CUDA device memory of the current device, e.g. PyTorch tensors).  The
+ *     library never allocates device memory; calls that need scratch take a
+ *     caller-provided workspace whose size the matching *_workspace_size()
+ *     returns.
+ *   - All arrays are dense, row-major, with the last index fastest.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call only enqueues work on it and never synchronises the host,
+ *     except kdn_read_workspace_status().
+ *   - Arguments are checked before anything is enqueued.  A call that returns
+ *     anything but KDN_OK has enqueued nothing.  No C++ exception crosses
+ *     this interface.
+ *   - Floating-point state (a, w, r, S, p, o) is always fp32.  q, k, v are
+ *     fp32 or bf16 (in_dtype).  The output o is fp32: the bf16 rounding of an
+ *     exact output alone exceeds the layer's error bound (max-abs / RMS
+ *     <= 2e-2) for outputs whose max is ~10x their RMS.
+ */
+#ifndef KDN_H_
+#define KDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kdn_status {
+  KDN_OK = 0,
+  KDN_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or enum  */
+  KDN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (shape, path)      */
+  KDN_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required   */
+  KDN_ERR_TIMEOUT = 4,      /* a bounded on-device wait gave up             */
+  KDN_ERR_CUDA = 5          /* the CUDA runtime reported an error           */
+} kdn_status;
+
+typedef enum kdn_dtype { KDN_F32 = 0, KDN_BF16 = 1 } kdn_dtype;
+typedef enum kdn_variant { KDN_ISO = 0, KDN_DIAG = 1 } kdn_variant;
+
+/* Forward-path selector (the `chunk` argument of the forward calls). */
+enum {
+  KDN_CHUNK_AUTO = 0,       /* chunked engine when supported, else recurrent */
+  KDN_CHUNK_RECURRENT = 1,  /* token-by-token kernel, any supported shape    */
+  KDN_CHUNK_64 = 64         /* chunkwise tensor-core engine, 64-token chunks */
+};
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* kdn_status_string(kdn_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int kdn_version(void);
+
+/* ------------------------------------------------------------------------
+ * kdn_mobius_scan -- the uncertainty recursion alone, over N independent
+ * lanes of length T ("Kalman Delta Networks: Uncertainty-aware Associative
+ * Memory", abstract: the variance recursions are Mobius maps composed by an
+ * associative scan; "Kalman Linear Attention ...", 方法论 §2 prints the
+ * fractional-linear form).  For every lane i and step t:
+ *     c          = info_scale * n[i,t]
+ *     prior[i,t] = a^2 lambda[i,t-1] + w
+ *     lambda[i,t]= (r a^2 lambda[i,t-1] + r w) / (c a^2 lambda[i,t-1] + r + c w)
+ *     gain[i,t]  = prior / (prior * n + r)     (the isotropic write strength)
+ * with lambda[i,-1] = lambda0[i] (or 1 when lambda0 is NULL).
+ *
+ * a, w, r, n     [N, T] fp32 device; n is the squared key norm (or k_i^2)
+ * lambda0        [N] fp32 device, or NULL for all ones
+ * info_scale     c = info_scale * n; must be finite and >= 0
+ * lambda_out     [N, T] fp32 device, posterior variances (required)
+ * prior_out      [N, T] fp32 device or NULL
+ * gain_out       [N, T] fp32 device or NULL
+ * workspace      device scratch of >= kdn_mobius_scan_workspace_size(N, T)
+ *                bytes, 256-byte aligned; its contents are overwritten
+ *                (the call clears what it needs on the stream first)
+ * Requires a, w, r, n, lambda_out (and prior_out / gain_out when given) to be
+ * 16-byte aligned; any T >= 1 and N >= 1 with N*T < 2^40.
+ * Errors: KDN_ERR_INVALID_ARG, KDN_ERR_WORKSPACE, KDN_ERR_CUDA.  A look-back
+ * wait that gives up (it cannot in correct use) is recorded in the workspace
+ * and reported by kdn_read_workspace_status().
+ * ---------------------------------------------------------------------- */
+size_t kdn_mobius_scan_workspace_size(int64_t N, int64_t T);
+kdn_status kdn_mobius_scan(const float* a, const float* w, const float* r,
+                           const float* n, const float* lambda0,
+                           float info_scale, float* lambda_out,
+                           float* prior_out, float* gain_out, int64_t N,
+                           int64_t T, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* ------------------------------------------------------------------------
+ * kdn_iso_forward -- Isotropic KDN layer forward ("Kalman Delta Networks:
+ * Uncertainty-aware Associative Memory", abstract: one uncertainty scalar
+ * per head; "Kalman Delta Networks: 不确定性感知的联想记忆", 方法 — 关键模块
+ * steps 1-3 and 输出与差异点).  Per (b, h) and token t:
+ *     n = ||k_t||^2;  p- = a^2 p + w;  beta = p- / (p- n + r)
+ *     p = 1 / (1/p- + info_scale * n / r)
+ *     S = a S + (v_t - a S k_t) (beta k_t)';   o_t = S q_t
+ *
+ * q, k     [B, T, H, dk] in_dtype device
+ * v        [B, T, H, dv] in_dtype device
+ * a, w, r  [B, T, H] fp32 device (decay in (0,1], process-noise variance
+ *          >= 0, observation-noise variance > 0)
+ * S0       [B, H, dv, dk] fp32 device initial memory, or NULL for zeros
+ * p0       [B, H] fp32 device initial variance, or NULL for ones
+ * o        [B, T, H, dv] fp32 device output
+ * S_out    [B, H, dv, dk] fp32 device final memory (may alias S0)
+ * p_out    [B, H] fp32 device final variance (may alias p0)
+ * info_scale  kappa; <= 0 selects 1/dk
+ * chunk    KDN_CHUNK_AUTO, KDN_CHUNK_RECURRENT or KDN_CHUNK_64
+ * workspace   device scratch of >= kdn_forward_workspace_size(...) bytes,
+ *             256-byte aligned (NULL allowed when that size is 0).  The
+ *             chunked path keeps its device error word and a copy of p0
+ *             there; kdn_read_workspace_status() reads the error word.
+ * Supported: T >= 1; dk in {32, 64, 128}; 1 <= dv <= 128.  KDN_CHUNK_64
+ * additionally needs in_dtype == KDN_BF16, dk == 128 and dv in {64, 128}.
+ * All pointers 16-byte aligned.  o must not alias the inputs.
+ * Errors: KDN_ERR_INVALID_ARG, KDN_ERR_UNSUPPORTED, KDN_ERR_WORKSPACE,
+ * KDN_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+size_t kdn_forward_workspace_size(kdn_variant variant, int B, int T, int H,
+                                  int dk, int dv, int chunk);
+kdn_status kdn_iso_forward(const void* q, const void* k, const void* v,
+                           kdn_dtype in_dtype, const float* a, const float* w,
+                           const float* r, const float* S0, const float* p0,
+                           float* o, float* S_out, float* p_out, int B, int T,
+                           int H, int dk, int dv, float info_scale, int chunk,
+                           void* workspace, size_t workspace_bytes,
+                           void* stream);
+
+/* ------------------------------------------------------------------------
+ * kdn_diag_forward -- Diagonal KDN layer forward ("Kalman Delta Networks:
+ * Uncertainty-aware Associative Memory", abstract: online mean-field
+ * variational projection onto diagonal Gaussians).  Per (b, h), token t and
+ * key dimension i:
+ *     p-_i = a^2 p_i + w_i;   s = sum_i p-_i k_i^2 + r;   g = p- * k / s
+ *     p_i  = 1 / (1/p-_i + k_i^2 / r)
+ *     S = a S + (v_t - a S k_t) g';   o_t = S q_t
+ * Arguments as kdn_iso_forward except:
+ * w        [B, T, H, dk] fp32 device (per-dimension process noise)
+ * p0, p_out  [B, H, dk] fp32 device (NULL p0 = ones)
+ * (no info_scale: the diagonal projection has none)
+ * ---------------------------------------------------------------------- */
+kdn_status kdn_diag_forward(const void* q, const void* k, const void* v,
+                            kdn_dtype in_dtype, const float* a, const float* w,
+                            const float* r, const float* S0, const float* p0,
+                            float* o, float* S_out, float* p_out, int B, int T,
+                            int H, int dk, int dv, int chunk, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * kdn_decode_step -- one recurrent decoding step for B x H heads, updating
+ * the state in place (the constant-memory decoding of "Kalman Delta
+ * Networks: Uncertainty-aware Associative Memory", abstract).  The same
+ * update as one token of kdn_iso_forward / kdn_diag_forward.
+ *
+ * variant  KDN_ISO or KDN_DIAG
+ * q, k     [B, H, dk] in_dtype device;  v [B, H, dv] in_dtype device
+ * a, r     [B, H] fp32 device
+ * w        [B, H] (iso) or [B, H, dk] (diag) fp32 device
+ * S        [B, H, dv, dk] fp32 device, read and overwritten
+ * p        [B, H] (iso) or [B, H, dk] (diag) fp32 device, read and overwritten
+ * o        [B, H, dv] fp32 device output
+ * info_scale  iso only; <= 0 selects 1/dk
+ * Supported: dk in {32, 64, 128}; 1 <= dv <= 128; pointers 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k,
+                           const void* v, kdn_dtype in_dtype, const float* a,
+                           const float* w, const float* r, float* S, float* p,
+                           float* o, int B, int H, int dk, int dv,
+                           float info_scale, void* stream);
+
+/* ------------------------------------------------------------------------
+ * kdn_read_workspace_status -- synchronise `stream`, then report the device
+ * error word a previous call left in `workspace`: KDN_OK, or KDN_ERR_TIMEOUT
+ * if a bounded on-device wait gave up.  Also returns KDN_ERR_CUDA if the
+ * stream reports an error.  This is the only call that blocks the host.
+ * ---------------------------------------------------------------------- */
+kdn_status kdn_read_workspace_status(const void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDN_H_ */

@@ -1,0 +1,37 @@
+/*
+ * kdn_testing.h -- test-only entry points of libkdn.  They exist so the
+ * failure paths of the library can be exercised without faulting a GPU.
+ * They have no counterpart on the pages and are not part of the layer API.
+ */
+#ifndef KDN_TESTING_H_
+#define KDN_TESTING_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kdn.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* kdn_mobius_scan (lambda only), except that the tile with hand-out index
+ * `silent_tile` never publishes its aggregate or prefix.  Tiles are handed
+ * out tile-index-major: tile id = j * N + lane, where j is the 2048-step tile
+ * within the lane.  The successor tile's bounded look-back therefore runs
+ * out (after about one second), records KDN_ERR_TIMEOUT in the workspace
+ * error word and finishes.  The call returns normally;
+ * kdn_read_workspace_status() then reports KDN_ERR_TIMEOUT.  Outputs after
+ * the silent tile are not meaningful.  Arguments as kdn_mobius_scan;
+ * silent_tile >= 0. */
+kdn_status kdn_testing_mobius_scan_unpublished_tile(
+    const float* a, const float* w, const float* r, const float* n,
+    const float* lambda0, float info_scale, float* lambda_out, int64_t N,
+    int64_t T, void* workspace, size_t workspace_bytes, int64_t silent_tile,
+    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDN_TESTING_H_ */

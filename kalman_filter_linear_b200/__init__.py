@@ -6,11 +6,3 @@ over it that passes PyTorch tensors' device pointers and the current CUDA
 stream.  PyTorch is used only for device memory and streams.  The library is
 loaded on first use; if it is missing the call raises instead of falling back.
 """
-from .synth import WORKLOADS  # noqa: F401  (input generator, no filter arithmetic)
-
-
-def __getattr__(name):
-    if name == 'kdn':
-        from . import kdn
-        return kdn
-    raise AttributeError(name)

@@ -1,0 +1,323 @@
+// kdn_mobius_scan: the KDN uncertainty recursion over N independent lanes.
+//
+// Each step of a lane is the Mobius map of the variance,
+//   p_t = (r a^2 p + r w) / (c a^2 p + r + c w),   c = info_scale * n,
+// i.e. the 2x2 matrix M_t = [[r a^2, r w], [c a^2, r + c w]] acting
+// projectively ("Kalman Delta Networks: Uncertainty-aware Associative
+// Memory", abstract: the recursion is a Mobius map and composes by an
+// associative scan; "Kalman Linear Attention ...", 方法论 §2: O(T) work,
+// O(log T) depth).  Prefix compositions P_t = M_t ... M_1 (later maps on the
+// left) give p_t = P_t(p_0).
+//
+// Kernel layout (one CTA per 2048-token tile of one lane):
+//   1. 256 threads load 8 consecutive steps each (two 16-byte loads per
+//      array), build their maps and compose them serially in registers;
+//   2. warp-shuffle inclusive scan of the thread products, then a block scan
+//      of the 8 warp totals in shared memory;
+//   3. decoupled look-back across the tiles of the lane: a tile publishes its
+//      aggregate, then its inclusive prefix; a successor combines the
+//      published values of its predecessors.  Tiles are handed out by an
+//      atomic counter in tile-index-major order (all lanes' tile 0 first),
+//      so a predecessor has almost always finished already.  Every wait is
+//      bounded in wall-clock time; a wait that gives up records
+//      DEV_TIMEOUT in the workspace error word and the tile goes on with
+//      what it has.
+//   4. each thread applies its exclusive prefix to p_0 and runs the scalar
+//      recursion over its 8 steps, writing p (and optionally p^- and the
+//      isotropic write strength).
+// All products have non-negative entries (no cancellation).  They are
+// renormalised by powers of two, which is exact, so renormalisation adds no
+// rounding.
+#include "kdn_common.cuh"
+
+namespace kdn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kPerThread = 8;
+constexpr int kTile = kThreads * kPerThread;  // 2048 steps
+
+struct Mat2 {
+  float a, b, c, d;  // [[a, b], [c, d]]
+};
+
+__device__ __forceinline__ Mat2 identity() { return {1.f, 0.f, 0.f, 1.f}; }
+
+// x * y (x is the later map).
+__device__ __forceinline__ Mat2 mul(const Mat2& x, const Mat2& y) {
+  Mat2 z;
+  z.a = fmaf(x.a, y.a, x.b * y.c);
+  z.b = fmaf(x.a, y.b, x.b * y.d);
+  z.c = fmaf(x.c, y.a, x.d * y.c);
+  z.d = fmaf(x.c, y.b, x.d * y.d);
+  return z;
+}
+
+// Scale by 2^-e where 2^e is the binade of the largest entry.  Exact.
+__device__ __forceinline__ Mat2 renorm(const Mat2& x) {
+  const float m = fmaxf(fmaxf(x.a, x.b), fmaxf(x.c, x.d));
+  const int e = (int)((__float_as_uint(m) >> 23) & 0xffu) - 127;
+  if (e > -100 && e < 100 && e != 0) {
+    const float s = __uint_as_float((uint32_t)(127 - e) << 23);
+    return {x.a * s, x.b * s, x.c * s, x.d * s};
+  }
+  return x;
+}
+
+__device__ __forceinline__ float apply(const Mat2& m, float lam) {
+  return __fdividef(fmaf(m.a, lam, m.b), fmaf(m.c, lam, m.d));
+}
+
+__device__ __forceinline__ Mat2 shfl_up(const Mat2& x, int delta) {
+  return {__shfl_up_sync(0xffffffffu, x.a, delta), __shfl_up_sync(0xffffffffu, x.b, delta),
+          __shfl_up_sync(0xffffffffu, x.c, delta), __shfl_up_sync(0xffffffffu, x.d, delta)};
+}
+
+struct ScanWs {
+  uint32_t* error;    // device error word
+  uint32_t* counter;  // next tile to hand out
+  uint32_t* flag;     // per tile: 0 none, 1 aggregate, 2 inclusive prefix
+  float4* agg;        // per tile aggregate
+  float4* incl;       // per tile inclusive prefix
+};
+
+__device__ __forceinline__ float4 as_f4(const Mat2& m) { return make_float4(m.a, m.b, m.c, m.d); }
+__device__ __forceinline__ Mat2 as_mat(const float4& f) { return {f.x, f.y, f.z, f.w}; }
+
+__global__ void __launch_bounds__(kThreads)
+mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
+                   const float* __restrict__ R, const float* __restrict__ Nsq,
+                   const float* __restrict__ lambda0, float info_scale,
+                   float* __restrict__ lam_out, float* __restrict__ prior_out,
+                   float* __restrict__ gain_out, int64_t N, int64_t T, int64_t tiles_per_lane,
+                   ScanWs ws, int vec_ok, int64_t debug_skip_tile) {
+  __shared__ Mat2 s_warp[kThreads / 32];
+  __shared__ Mat2 s_tile_prefix;
+  __shared__ uint32_t s_tile;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+
+  if (tid == 0) s_tile = atomicAdd(ws.counter, 1u);
+  __syncthreads();
+  const int64_t tile = s_tile;
+  const int64_t j = tile / N;    // tile index within the lane
+  const int64_t seq = tile % N;  // lane
+  const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
+  const int64_t base = seq * T;
+
+  // ---- 1. load and compose this thread's maps
+  float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
+  if (vec_ok && t0 + kPerThread <= T) {
+    const float4* a4 = reinterpret_cast<const float4*>(A + base + t0);
+    const float4* w4 = reinterpret_cast<const float4*>(W + base + t0);
+    const float4* r4 = reinterpret_cast<const float4*>(R + base + t0);
+    const float4* n4 = reinterpret_cast<const float4*>(Nsq + base + t0);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float4 x = __ldg(a4 + h), y = __ldg(w4 + h), z = __ldg(r4 + h), u = __ldg(n4 + h);
+      a[4 * h] = x.x; a[4 * h + 1] = x.y; a[4 * h + 2] = x.z; a[4 * h + 3] = x.w;
+      w[4 * h] = y.x; w[4 * h + 1] = y.y; w[4 * h + 2] = y.z; w[4 * h + 3] = y.w;
+      r[4 * h] = z.x; r[4 * h + 1] = z.y; r[4 * h + 2] = z.z; r[4 * h + 3] = z.w;
+      n[4 * h] = u.x; n[4 * h + 1] = u.y; n[4 * h + 2] = u.z; n[4 * h + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const bool in = t0 + i < T;
+      a[i] = in ? __ldg(A + base + t0 + i) : 1.f;
+      w[i] = in ? __ldg(W + base + t0 + i) : 0.f;
+      r[i] = in ? __ldg(R + base + t0 + i) : 1.f;
+      n[i] = in ? __ldg(Nsq + base + t0 + i) : 0.f;
+    }
+  }
+
+  Mat2 P = identity();
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    if (t0 + i < T) {
+      const float c = info_scale * n[i];
+      const float a2 = a[i] * a[i];
+      const Mat2 M = {r[i] * a2, r[i] * w[i], c * a2, fmaf(c, w[i], r[i])};
+      P = mul(M, P);
+      if (i & 1) P = renorm(P);
+    }
+  }
+  P = renorm(P);
+
+  // ---- 2. warp inclusive scan, then block scan of warp totals
+  Mat2 incl = P;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const Mat2 prev = shfl_up(incl, d);
+    if (lane >= d) incl = renorm(mul(incl, prev));
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    Mat2 x = lane < kThreads / 32 ? s_warp[lane] : identity();
+#pragma unroll
+    for (int d = 1; d < kThreads / 32; d <<= 1) {
+      const Mat2 prev = shfl_up(x, d);
+      if (lane >= d) x = renorm(mul(x, prev));
+    }
+    if (lane < kThreads / 32) s_warp[lane] = x;  // inclusive over warps
+  }
+  __syncthreads();
+
+  // ---- 3. decoupled look-back (thread 0)
+  if (tid == 0) {
+    const Mat2 agg = s_warp[kThreads / 32 - 1];
+    Mat2 excl = identity();
+    const bool skip_publish = (tile == debug_skip_tile);  // fault-injection hook
+    if (j == 0) {
+      if (!skip_publish) {
+        ws.incl[tile] = as_f4(agg);
+        __threadfence();
+        st_release_u32(ws.flag + tile, 2u);
+      }
+    } else {
+      if (!skip_publish) {
+        ws.agg[tile] = as_f4(agg);
+        __threadfence();
+        st_release_u32(ws.flag + tile, 1u);
+      }
+      const uint64_t start = globaltimer_ns();
+      bool timed_out = false;
+      for (int64_t p = j - 1; p >= 0 && !timed_out;) {
+        const int64_t pt = p * N + seq;
+        uint32_t f = ld_acquire_u32(ws.flag + pt);
+        while (f == 0u) {
+          if (globaltimer_ns() - start > kWaitLimitNs) {
+            timed_out = true;
+            break;
+          }
+          __nanosleep(64);
+          f = ld_acquire_u32(ws.flag + pt);
+        }
+        if (timed_out) break;
+        if (f == 2u) {
+          excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
+          break;
+        }
+        excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
+        --p;
+      }
+      if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
+      if (!skip_publish) {
+        ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
+        __threadfence();
+        st_release_u32(ws.flag + tile, 2u);
+      }
+    }
+    s_tile_prefix = excl;
+  }
+  __syncthreads();
+
+  // ---- 4. apply the exclusive prefix and run the recursion
+  Mat2 thread_excl = shfl_up(incl, 1);
+  if (lane == 0) thread_excl = identity();
+  if (warp > 0) thread_excl = mul(thread_excl, s_warp[warp - 1]);
+  thread_excl = renorm(mul(renorm(thread_excl), s_tile_prefix));
+  const float lam0 = lambda0 ? __ldg(lambda0 + seq) : 1.f;
+  float lam = apply(thread_excl, lam0);
+
+  float out_l[kPerThread], out_p[kPerThread], out_g[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const float prior = fmaf(a[i] * a[i], lam, w[i]);
+    const float c = info_scale * n[i];
+    lam = __fdividef(r[i] * prior, fmaf(c, prior, r[i]));
+    out_l[i] = lam;
+    out_p[i] = prior;
+    out_g[i] = __fdividef(prior, fmaf(prior, n[i], r[i]));
+  }
+  if (vec_ok && t0 + kPerThread <= T) {
+    float4* l4 = reinterpret_cast<float4*>(lam_out + base + t0);
+    l4[0] = make_float4(out_l[0], out_l[1], out_l[2], out_l[3]);
+    l4[1] = make_float4(out_l[4], out_l[5], out_l[6], out_l[7]);
+    if (prior_out) {
+      float4* p4 = reinterpret_cast<float4*>(prior_out + base + t0);
+      p4[0] = make_float4(out_p[0], out_p[1], out_p[2], out_p[3]);
+      p4[1] = make_float4(out_p[4], out_p[5], out_p[6], out_p[7]);
+    }
+    if (gain_out) {
+      float4* g4 = reinterpret_cast<float4*>(gain_out + base + t0);
+      g4[0] = make_float4(out_g[0], out_g[1], out_g[2], out_g[3]);
+      g4[1] = make_float4(out_g[4], out_g[5], out_g[6], out_g[7]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      if (t0 + i < T) {
+        lam_out[base + t0 + i] = out_l[i];
+        if (prior_out) prior_out[base + t0 + i] = out_p[i];
+        if (gain_out) gain_out[base + t0 + i] = out_g[i];
+      }
+    }
+  }
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct ScanLayout {
+  int64_t tiles_per_lane, ntiles;
+  size_t off_flag, off_agg, off_incl, total, clear_bytes;
+};
+
+inline ScanLayout scan_layout(int64_t N, int64_t T) {
+  ScanLayout L;
+  L.tiles_per_lane = (T + kTile - 1) / kTile;
+  L.ntiles = L.tiles_per_lane * N;
+  L.off_flag = 256;
+  L.off_agg = align_up(L.off_flag + (size_t)L.ntiles * 4, 256);
+  L.off_incl = align_up(L.off_agg + (size_t)L.ntiles * 16, 256);
+  L.total = align_up(L.off_incl + (size_t)L.ntiles * 16, 256);
+  L.clear_bytes = L.off_flag + (size_t)L.ntiles * 4;
+  return L;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+size_t mobius_scan_workspace_size(int64_t N, int64_t T) {
+  if (N <= 0 || T <= 0) return 0;
+  return scan_layout(N, T).total;
+}
+
+kdn_status mobius_scan_launch(const float* a, const float* w, const float* r, const float* n,
+                              const float* lambda0, float info_scale, float* lambda_out,
+                              float* prior_out, float* gain_out, int64_t N, int64_t T,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                              int64_t debug_skip_tile) {
+  if (!a || !w || !r || !n || !lambda_out) return KDN_ERR_INVALID_ARG;
+  if (N <= 0 || T <= 0 || N * T >= (int64_t(1) << 40)) return KDN_ERR_INVALID_ARG;
+  if (!(info_scale >= 0.f) || !(info_scale < 3.0e38f)) return KDN_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(r) || !aligned16(n) ||
+      !aligned16(lambda_out) || (prior_out && !aligned16(prior_out)) ||
+      (gain_out && !aligned16(gain_out)))
+    return KDN_ERR_INVALID_ARG;
+  const ScanLayout L = scan_layout(N, T);
+  if (!workspace || workspace_bytes < L.total) return KDN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDN_ERR_INVALID_ARG;
+  if (L.ntiles > (int64_t)0x7fffffff) return KDN_ERR_UNSUPPORTED;
+
+  char* base = static_cast<char*>(workspace);
+  ScanWs ws;
+  ws.error = reinterpret_cast<uint32_t*>(base);
+  ws.counter = reinterpret_cast<uint32_t*>(base + 4);
+  ws.flag = reinterpret_cast<uint32_t*>(base + L.off_flag);
+  ws.agg = reinterpret_cast<float4*>(base + L.off_agg);
+  ws.incl = reinterpret_cast<float4*>(base + L.off_incl);
+
+  if (cudaMemsetAsync(workspace, 0, L.clear_bytes, stream) != cudaSuccess) return KDN_ERR_CUDA;
+  const int vec_ok = (T % 4 == 0) ? 1 : 0;
+  mobius_scan_kernel<<<(unsigned)L.ntiles, kThreads, 0, stream>>>(
+      a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out, N, T, L.tiles_per_lane,
+      ws, vec_ok, debug_skip_tile);
+  return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
+}
+
+}  // namespace kdn

@@ -1,0 +1,117 @@
+"""The C-ABI library loads and exports what include/*.h declares (CPU only).
+
+Only calls that must fail argument validation are made here: those return
+before touching the CUDA runtime, so no GPU is needed.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from kalman_filter_linear_b200 import kdn, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope='module')
+def L():
+    if build.is_stale():
+        build.build()
+    return kdn.lib()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, 'include', '*.h')):
+        src = open(h).read()
+        src = re.sub(r'/\*.*?\*/', '', src, flags=re.S)
+        for m in re.finditer(r'\b(kdn_[a-z0-9_]+)\s*\(', src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert 'kdn_iso_forward' in names and 'kdn_mobius_scan' in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    for s in range(6):
+        assert L.kdn_status_string(s).startswith(b'KDN_')
+    assert L.kdn_status_string(99) == b'unknown kdn_status'
+    assert L.kdn_version() >= 100
+
+
+def test_workspace_sizes_are_host_computable(L):
+    assert kdn.kdn_mobius_scan_workspace_size(0, 10) == 0
+    s1 = kdn.kdn_mobius_scan_workspace_size(4096, 65536)
+    s2 = kdn.kdn_mobius_scan_workspace_size(4096, 65537)
+    assert s1 > 0 and s2 > s1 and s1 % 256 == 0
+    assert kdn.kdn_forward_workspace_size(kdn.KDN_ISO, 1, 1, 1, 64, 64,
+                                          kdn.KDN_CHUNK_RECURRENT) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced
+MIS = ctypes.c_void_p(0x10004)   # misaligned
+
+
+def test_scan_rejects_bad_arguments(L):
+    ws = ctypes.c_void_p(0x20000)
+    big = ctypes.c_size_t(1 << 40)
+    call = lambda *a: L.kdn_mobius_scan(*a)
+    assert call(None, FAKE, FAKE, FAKE, None, 1.0, FAKE, None, None, 4, 8, ws, big, None) == \
+        kdn.KDN_ERR_INVALID_ARG
+    assert call(FAKE, FAKE, FAKE, FAKE, None, 1.0, FAKE, None, None, 0, 8, ws, big, None) == \
+        kdn.KDN_ERR_INVALID_ARG
+    assert call(FAKE, FAKE, FAKE, FAKE, None, -1.0, FAKE, None, None, 4, 8, ws, big, None) == \
+        kdn.KDN_ERR_INVALID_ARG
+    assert call(MIS, FAKE, FAKE, FAKE, None, 1.0, FAKE, None, None, 4, 8, ws, big, None) == \
+        kdn.KDN_ERR_INVALID_ARG
+    assert call(FAKE, FAKE, FAKE, FAKE, None, 1.0, FAKE, None, None, 4, 8, ws, 16, None) == \
+        kdn.KDN_ERR_WORKSPACE
+    assert call(FAKE, FAKE, FAKE, FAKE, None, 1.0, FAKE, None, None, 4, 8, None, big, None) == \
+        kdn.KDN_ERR_WORKSPACE
+
+
+def _fwd(L, **kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_BF16, a=FAKE, w=FAKE, r=FAKE, S0=None,
+                p0=None, o=FAKE, S=FAKE, p=FAKE, B=1, T=8, H=1, dk=128, dv=128, kappa=0.0,
+                chunk=kdn.KDN_CHUNK_RECURRENT, ws=None, wsb=0, stream=None)
+    args.update(kw)
+    return L.kdn_iso_forward(*args.values())
+
+
+def test_forward_rejects_bad_arguments(L):
+    assert _fwd(L, q=None) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, o=None) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, dt=7) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, B=0) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, T=-3) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, k=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, S0=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, kappa=float('nan')) == kdn.KDN_ERR_INVALID_ARG
+    assert _fwd(L, dk=96) == kdn.KDN_ERR_UNSUPPORTED
+    assert _fwd(L, dv=200) == kdn.KDN_ERR_UNSUPPORTED
+    assert _fwd(L, chunk=5) == kdn.KDN_ERR_INVALID_ARG
+    # the chunked engine takes bf16 inputs only
+    assert _fwd(L, dt=kdn.KDN_F32, chunk=kdn.KDN_CHUNK_64) == kdn.KDN_ERR_UNSUPPORTED
+    assert L.kdn_diag_forward(FAKE, FAKE, FAKE, kdn.KDN_BF16, FAKE, FAKE, FAKE, None, None, FAKE,
+                              FAKE, FAKE, 1, 8, 1, 128, 128, 3, None, 0, None) == \
+        kdn.KDN_ERR_INVALID_ARG
+
+
+def test_decode_rejects_bad_arguments(L):
+    d = lambda **kw: L.kdn_decode_step(*dict(dict(var=kdn.KDN_DIAG, q=FAKE, k=FAKE, v=FAKE,
+                                                  dt=kdn.KDN_BF16, a=FAKE, w=FAKE, r=FAKE, S=FAKE,
+                                                  p=FAKE, o=FAKE, B=2, H=2, dk=128, dv=128,
+                                                  kappa=0.0, stream=None), **kw).values())
+    assert d(var=5) == kdn.KDN_ERR_INVALID_ARG
+    assert d(S=None) == kdn.KDN_ERR_INVALID_ARG
+    assert d(p=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert d(H=0) == kdn.KDN_ERR_INVALID_ARG
+    assert d(dk=48) == kdn.KDN_ERR_UNSUPPORTED
+    assert L.kdn_read_workspace_status(None, 0, None) == kdn.KDN_ERR_INVALID_ARG

@@ -101,6 +101,36 @@ kdn_status kdn_mobius_scan(const float* a, const float* w, const float* r,
                            void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_mobius_scan_noalloc -- kdn_mobius_scan without a workspace argument,
+ * for callers that cannot allocate device memory where they call the scan
+ * (for example a host program that gives all device memory to its own pool
+ * at start-up and permits no cudaMalloc afterwards, or a plug-in that such a
+ * host hands only its input and output buffers).  The pages have no
+ * counterpart of this entry point; it only changes where scratch lives.
+ *
+ * The scratch is a fixed array of about 7.9 MiB inside the library's device
+ * code.  Every GPU that loads the library holds it until the process exits.
+ * Limit: N * ceil(T / 2048) <= KDN_SCAN_NOALLOC_MAX_TILES (e.g. 4096 lanes
+ * up to T = 114688); larger calls return KDN_ERR_WORKSPACE without enqueuing
+ * anything.  The call allocates nothing: the first call on a device looks up
+ * the array's device address with that device current (documented set-up;
+ * make this first call before any stream capture), and every call clears the
+ * part of the array that must start at zero on `stream` before its kernel.
+ * All calls share the one array: calls whose work overlaps on the GPU (for
+ * example on two streams without ordering between them) race and give wrong
+ * results, so order them.  A look-back wait that gives up is recorded only in
+ * that internal array and is not reported by this entry point.  Otherwise the
+ * arguments, results and errors are those of kdn_mobius_scan.
+ * ---------------------------------------------------------------------- */
+#define KDN_SCAN_NOALLOC_MAX_TILES 229376
+kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w,
+                                   const float* r, const float* n,
+                                   const float* lambda0, float info_scale,
+                                   float* lambda_out, float* prior_out,
+                                   float* gain_out, int64_t N, int64_t T,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_iso_forward -- Isotropic KDN layer forward ("Kalman Delta Networks:
  * Uncertainty-aware Associative Memory", abstract: one uncertainty scalar
  * per head; "Kalman Delta Networks: 不确定性感知的联想记忆", 方法 — 关键模块

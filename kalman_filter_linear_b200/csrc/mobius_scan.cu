@@ -28,6 +28,9 @@
 // All products have non-negative entries (no cancellation).  They are
 // renormalised by powers of two, which is exact, so renormalisation adds no
 // rounding.
+#include <atomic>
+#include <mutex>
+
 #include "kdn_common.cuh"
 
 namespace kdn {
@@ -321,3 +324,66 @@ kdn_status mobius_scan_launch(const float* a, const float* w, const float* r, co
 }
 
 }  // namespace kdn
+
+// ----------------------------------------------------------------------------
+// Allocation-free variant (kdn_mobius_scan_noalloc).
+//
+// Some callers cannot allocate device memory where they call the scan, for
+// example a host program that hands all device memory to its own pool at
+// start-up and allows no cudaMalloc afterwards, or a plug-in that such a host
+// gives only its input and output buffers.  For them the look-back scratch
+// (tile flags, aggregates, prefixes, tile counter, error word) lives in the
+// fixed-size array below, which every GPU that loads this library holds until
+// the process exits.
+// ----------------------------------------------------------------------------
+namespace kdn {
+namespace {
+
+constexpr int64_t kNoAllocMaxTiles = KDN_SCAN_NOALLOC_MAX_TILES;
+constexpr size_t align_up_c(size_t x, size_t a) { return (x + a - 1) / a * a; }
+// Same layout as a caller workspace for kNoAllocMaxTiles tiles.
+constexpr size_t kNoAllocBytes =
+    align_up_c(align_up_c(align_up_c(256 + (size_t)kNoAllocMaxTiles * 4, 256) +
+                              (size_t)kNoAllocMaxTiles * 16, 256) +
+                   (size_t)kNoAllocMaxTiles * 16, 256);
+
+static __device__ __align__(256) uint8_t g_noalloc_scan_scratch[kNoAllocBytes];
+
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device with that device current.  In host code the array's name is a
+// host-side stand-in, not a device address, so it is never passed to a kernel.
+void* noalloc_scratch_on_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scan_scratch) != cudaSuccess || !addr) return nullptr;
+  g_noalloc_addr[dev].store(addr, std::memory_order_release);
+  return addr;
+}
+
+}  // namespace
+}  // namespace kdn
+
+extern "C" kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w, const float* r,
+                                              const float* n, const float* lambda0,
+                                              float info_scale, float* lambda_out,
+                                              float* prior_out, float* gain_out, int64_t N,
+                                              int64_t T, void* stream) {
+  if (N <= 0 || T <= 0 || N * T >= (int64_t(1) << 40)) return KDN_ERR_INVALID_ARG;
+  const int64_t tiles = N * ((T + kdn::kTile - 1) / kdn::kTile);
+  if (tiles > kdn::kNoAllocMaxTiles) return KDN_ERR_WORKSPACE;
+  void* scratch = kdn::noalloc_scratch_on_current_device();
+  if (!scratch) return KDN_ERR_CUDA;
+  return kdn::mobius_scan_launch(a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out,
+                                 N, T, scratch, kdn::kNoAllocBytes,
+                                 static_cast<cudaStream_t>(stream), -1);
+}

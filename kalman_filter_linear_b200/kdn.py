@@ -50,6 +50,8 @@ def lib():
     L.kdn_mobius_scan_workspace_size.argtypes = [_i64, _i64]
     L.kdn_mobius_scan.restype = _i32
     L.kdn_mobius_scan.argtypes = [_vp] * 5 + [_f32] + [_vp] * 3 + [_i64, _i64, _vp, _sz, _vp]
+    L.kdn_mobius_scan_noalloc.restype = _i32
+    L.kdn_mobius_scan_noalloc.argtypes = [_vp] * 5 + [_f32] + [_vp] * 3 + [_i64, _i64, _vp]
     L.kdn_forward_workspace_size.restype = _sz
     L.kdn_forward_workspace_size.argtypes = [_i32] * 7
     L.kdn_iso_forward.restype = _i32
@@ -144,6 +146,34 @@ def kdn_mobius_scan(a, w, r, n, lambda0=None, info_scale=1.0, lambda_out=None, p
                                workspace.numel() if workspace is not None else 0, _stream())
     _check(st, 'kdn_mobius_scan')
     return lambda_out, prior_out, gain_out, workspace
+
+
+KDN_SCAN_NOALLOC_MAX_TILES = 229376
+
+
+def kdn_mobius_scan_noalloc(a, w, r, n, lambda0=None, info_scale=1.0, lambda_out=None,
+                            prior_out=None, gain_out=None, want_prior=False, want_gain=False):
+    """kdn_mobius_scan with the library's internal scratch (no workspace):
+    for callers that cannot allocate device memory at the call.  Returns
+    (lambda, prior, gain); calls that overlap on the GPU race."""
+    N, T = a.shape
+    f = torch.float32
+    for name, t in (('a', a), ('w', w), ('r', r), ('n', n)):
+        _req(t, name, f, (N, T))
+    _opt(lambda0, 'lambda0', f, (N,))
+    lambda_out = _opt(lambda_out, 'lambda_out', f, (N, T)) if lambda_out is not None else \
+        torch.empty_like(a)
+    if prior_out is None and want_prior:
+        prior_out = torch.empty_like(a)
+    if gain_out is None and want_gain:
+        gain_out = torch.empty_like(a)
+    _opt(prior_out, 'prior_out', f, (N, T))
+    _opt(gain_out, 'gain_out', f, (N, T))
+    st = lib().kdn_mobius_scan_noalloc(_ptr(a), _ptr(w), _ptr(r), _ptr(n), _ptr(lambda0),
+                                       float(info_scale), _ptr(lambda_out), _ptr(prior_out),
+                                       _ptr(gain_out), N, T, _stream())
+    _check(st, 'kdn_mobius_scan_noalloc')
+    return lambda_out, prior_out, gain_out
 
 
 def kdn_forward_workspace_size(variant, B, T, H, dk, dv, chunk=KDN_CHUNK_AUTO):

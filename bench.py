@@ -211,7 +211,14 @@ def main():
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
+    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode'],
+                    help='run only this kernel (for profiler captures) and print its timing')
+    ap.add_argument('--B', type=int, default=None, help='batch override for --only')
+    ap.add_argument('--T', type=int, default=None, help='length override for --only')
     args = ap.parse_args()
+    if args.only:
+        run_only(args)
+        return
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get('RANK', '0'))
@@ -328,6 +335,53 @@ def main():
     print(json.dumps(line))
 
 
+def run_only(args):
+    """One kernel on its own, for profiler captures: `steps` timed launches
+    after `warmup` untimed ones."""
+    import torch
+    from kalman_filter_linear_b200 import kdn, synth
+    dev = torch.device('cuda', 0)
+    stream = torch.cuda.current_stream()
+    if args.only in ('iso', 'diag'):
+        c = synth.WORKLOADS['iso_1p3b' if args.only == 'iso' else 'diag_1p3b']
+        B = args.B or c['B']
+        T = args.T or c['T']
+        H, d = c['H'], c['dk']
+        x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, args.only, c['seed'],
+                                                         c['dtype']).items()}
+        var = kdn.KDN_ISO if args.only == 'iso' else kdn.KDN_DIAG
+        ws = torch.empty(max(kdn.kdn_forward_workspace_size(var, B, T, H, d, d), 256),
+                         dtype=torch.uint8, device=dev)
+        fwd = kdn.kdn_iso_forward if args.only == 'iso' else kdn.kdn_diag_forward
+        f = lambda: fwd(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], workspace=ws)
+        units, alg = B * T, layer_bytes(args.only, B, T, H, d, d)
+    elif args.only == 'scan':
+        c = synth.WORKLOADS['scan']
+        N = args.B or c['N']
+        T = args.T or c['T']
+        xs = {k: v.to(dev) for k, v in synth.scan_inputs(N, T, c['seed']).items()}
+        lam = torch.empty_like(xs['a'])
+        wss = torch.empty(kdn.kdn_mobius_scan_workspace_size(N, T), dtype=torch.uint8,
+                          device=dev)
+        f = lambda: kdn.kdn_mobius_scan(xs['a'], xs['w'], xs['r'], xs['n'], None,
+                                        c['info_scale'], lambda_out=lam, workspace=wss)
+        units, alg = N * T, N * T * 20
+    else:
+        c = synth.WORKLOADS['diag_long']
+        B = args.B or c['decode_batch']
+        H, d = c['H'], c['dk']
+        st = synth.decode_state(B, H, d, d, 'diag', seed=c['seed'])
+        Sd, pd = st['S'].to(dev), st['p'].to(dev)
+        xd = {k: v.to(dev) for k, v in synth.decode_inputs(B, H, d, d, 'diag', c['seed']).items()}
+        od = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+        f = lambda: kdn.kdn_decode_step('diag', xd['q'], xd['k'], xd['v'], xd['a'], xd['w'],
+                                        xd['r'], Sd, pd, o=od)
+        units, alg = B, decode_bytes(B, H, d, d)
+    ms = time_launches(f, args.steps, args.warmup, stream) / max(args.steps, 1)
+    print(json.dumps({'only': args.only, 'ms': ms, 'units_per_s': units / ms * 1e3,
+                      'achieved_gbs': alg / ms / 1e6, 'algorithmic_bytes': alg}))
+
+
 def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     import torch
     out = {}
@@ -350,6 +404,21 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
                         'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                         'algorithmic_bytes': alg}
     del x, o, S, p
+    # long-context diagonal forward, B1 T65536 H16
+    c = synth.WORKLOADS['diag_long']
+    B, T, H, d = c['B'], c['T'], c['H'], c['dk']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'diag', c['seed'],
+                                                     c['dtype']).items()}
+    ws = torch.empty(max(kdn.kdn_forward_workspace_size(kdn.KDN_DIAG, B, T, H, d, d), 256),
+                     dtype=torch.uint8, device=dev)
+    f = lambda: kdn.kdn_diag_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'],
+                                     workspace=ws)
+    ms = time_launches(f, 3, 2, stream) / 3
+    alg = layer_bytes('diag', B, T, H, d, d)
+    out['diag_long'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms,
+                        'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                        'algorithmic_bytes': alg}
+    del x, ws
     # standalone variance scan
     c = synth.WORKLOADS['scan']
     N, Tn = c['N'], c['T']

@@ -12,16 +12,18 @@
 //     O    = diag(gamma) Q S0' + ((Q G') o D) U,   D_tj = gamma_t/gamma_j (j <= t)
 //     S    = gamma_C S0 + U' diag(gamma_C/gamma) G
 // (derived from the token recursion S_t = a_t S_{t-1} + (v_t - a_t S_{t-1}
-// k_t) g_t'; the pages only say a hardware-efficient chunkwise form exists).
-// The variance recursion (a Mobius map per token) runs inside the chunk as a
-// warp scan of 2x2 maps (iso) or a per-dimension recursion (diag), with the
-// carried value passed from chunk to chunk.
+// k_t) g_t'; the pages only say that a hardware-efficient chunkwise form
+// exists).  The variance recursion (a Mobius map per token and lane) crosses
+// chunks through one carried value per lane.
 //
 // One CTA owns one (batch, head, block of NV value columns) for the whole
-// sequence; 256 threads.  Per chunk:
+// sequence: 16 warps.  The K/Q tiles are double-buffered and the V tile is
+// single-buffered; the copies of chunk c+1 (and its per-token scalars) are
+// issued during chunk c's diagonal-block solve, when 14 of the 16 warps are
+// idle and both buffers are free.  Per chunk:
 //   MMA1  D1 = [K;Q] G~'          (iso: G~ = K; diag: G~ = p- * k, hi/lo)
 //   MMA2  D2 = [K;Q] S'           (S as bf16 hi + lo)
-//   SIMT  A, T = (I+A)^-1 (blocked 16x16 forward substitution), Z
+//   SIMT  A, T = (I+A)^-1 (16x16 blocks, in place), Z = V - gamma K S'
 //   MMA3  D3 = [T_hi;T_lo] [Z_hi Z_lo]  -> U = top + bottom
 //   MMA4  D4 = [P_hi;P_lo] [U_hi U_lo]  -> O = D4 top + bottom + gamma Q S'
 //   MMA5  D5 = G~' [B_hi B_lo]          (B = diag(coef) U) -> S update
@@ -36,6 +38,10 @@
 // same warp, so the two halves combine with one shuffle.  K's rows are the
 // even groups, so the same tile is K (B operand of MMA1, stride 2048 B) and K'
 // (MN-major A operand of MMA5).
+//
+// Every wait is bounded.  A wait that gives up records DEV_TIMEOUT in the
+// workspace error word and raises an abort flag; the CTA then waits (bounded)
+// for its MMAs and copies in flight, frees TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -44,62 +50,93 @@
 namespace kdn {
 namespace {
 
-constexpr int kC = 64;     // tokens per chunk
-constexpr int kDK = 128;   // key dimension of the engine
-constexpr int kThreads = 256;
-constexpr int kScrLd = 68; // fp32 row stride of the 64x64 solve buffers
+constexpr int kC = 64;                   // tokens per chunk
+constexpr int kDK = 128;                 // key dimension of the engine
+constexpr int kCompute = 512;            // 16 warps
+constexpr int kThreads = kCompute;
+constexpr int kIssueWarp = 15;           // its lane 0 issues the TMA copies
+constexpr int kScalarWarp = 14;          // fetches the per-token scalars
+constexpr int kLd = 68;                  // fp32 row stride of the 64x64 solve buffer
 
 template <bool DIAG, int NV>
 struct Plan {
-  static constexpr int NVB = NV / 64;
-  static constexpr uint32_t KQ_BYTES = 2u * 128u * 128u;       // [kb 2][128 rows][64] bf16
-  static constexpr uint32_t V_BYTES = (uint32_t)NV * 64u * 2u; // [vb][64 t][64] bf16
-  static constexpr uint32_t SREG_BYTES = (uint32_t)NV * 512u;  // S hi+lo [vb][128 k][64]
-  static constexpr uint32_t ZU_BYTES = (uint32_t)NV * 128u;    // one of Z/U/B (hi or lo)
+  static constexpr int HC = NV / 4;  // result columns per warp
+  static constexpr int QC = HC / 2;  // result columns per lane (interleaved results)
+  static constexpr uint32_t KQ_BYTES = 2u * 128u * 128u;  // [kb 2][128 rows][64] bf16
+  static constexpr uint32_t V_BYTES = NV * 128u;          // [vb][64 t][64] bf16
+  static constexpr uint32_t S_BYTES = NV * 512u;          // S' hi+lo [vb][128 k][64]
+  static constexpr uint32_t ZU_BYTES = NV * 128u;         // one of Z/U/B (hi or lo)
   static constexpr uint32_t OFF_KQ = 0;
   static constexpr uint32_t OFF_V = OFF_KQ + 2 * KQ_BYTES;
-  static constexpr uint32_t OFF_S = OFF_V + 2 * V_BYTES;
-  static constexpr uint32_t OFF_TP = OFF_S + SREG_BYTES;       // [128][64] bf16 (T or P)
-  static constexpr uint32_t OFF_G = OFF_TP + 16384;            // diag: G~ hi, lo [kb][64][64]
-  static constexpr uint32_t OFF_SA = OFF_G + (DIAG ? 32768u : 0u);  // fp32 A [64][68]
-  static constexpr uint32_t OFF_ST = OFF_SA + 64u * kScrLd * 4u;    // fp32 T [64][68]
-  static constexpr uint32_t OFF_X = OFF_ST + 64u * kScrLd * 4u;     // fp32 [3][16][17]
-  static constexpr uint32_t OFF_SC = OFF_X + 3u * 16u * 17u * 4u + 64u;
-  static constexpr uint32_t OFF_BAR = OFF_SC + 8u * 64u * 4u;
-  static constexpr uint32_t TOTAL = OFF_BAR + 64u;
+  static constexpr uint32_t OFF_S = OFF_V + V_BYTES;
+  static constexpr uint32_t OFF_TP = OFF_S + S_BYTES;     // [128][64] bf16 (T, then P)
+  static constexpr uint32_t OFF_G = OFF_TP + 16384u;      // diag: G~ hi, lo [kb][64][64]
+  static constexpr uint32_t OFF_AT = OFF_G + (DIAG ? 32768u : 0u);  // fp32 [64][68]
+  static constexpr uint32_t OFF_X = OFF_AT + 64u * kLd * 4u;          // fp32 [4][16][18]
+  static constexpr uint32_t OFF_SC = OFF_X + 4608u;                   // 1152 floats
+  static constexpr uint32_t OFF_BAR = OFF_SC + 4608u;
+  static constexpr uint32_t TOTAL = OFF_BAR + 128u;
   static constexpr uint32_t ALLOC = TOTAL + 1024u;
-  // TMEM columns
   static constexpr uint32_t COL_D1 = 0, COL_D2 = 64, COL_D3 = 64 + NV, COL_D4 = 64 + 2 * NV;
   static constexpr uint32_t COL_D5 = COL_D3;
   static constexpr uint32_t TMEM_COLS = (64 + 3 * NV) <= 256 ? 256u : 512u;
   static_assert(TOTAL <= 227u * 1024u, "shared memory plan too large");
+  static_assert(NV == 64 || NV == 128, "value block");
 };
 
-// Token of 128-row interleaved operand row m, and whether it is the second half.
 __device__ __forceinline__ int il_token(int m) { return 8 * (m >> 4) + (m & 7); }
 __device__ __forceinline__ int il_second(int m) { return (m >> 3) & 1; }
-__device__ __forceinline__ int il_row(int t, int second) { return 16 * (t >> 3) + (t & 7) + 8 * second; }
-
-__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
-  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+__device__ __forceinline__ int il_row(int t, int second) {
+  return 16 * (t >> 3) + (t & 7) + 8 * second;
 }
 
-// Write 8 consecutive columns [col8*8, col8*8+8) of swizzled row `row` as hi
-// and lo bf16 halves of x[0..7].
-__device__ __forceinline__ void st_split8(uint8_t* hi_tile, uint8_t* lo_tile, uint32_t row,
-                                          uint32_t col8, const float* x) {
-  __nv_bfloat16 h[8], l[8];
+// Byte offset of 16-byte chunk col8 of swizzled 128-byte row `row`.
+__device__ __forceinline__ uint32_t chunk_off(uint32_t row, uint32_t col8) {
+  return row * 128u + (((col8 ^ row) & 7u) << 4);
+}
+
+// (hi, lo) bf16 splits of 8 floats, packed as two uint4.
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  uint32_t hw[4], lw[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) split_bf16(x[i], h[i], l[i]);
-  const uint32_t off = sw128_offset(row, col8 * 8);
-  *reinterpret_cast<uint4*>(hi_tile + off) =
-      make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
-  *reinterpret_cast<uint4*>(lo_tile + off) =
-      make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    const uint32_t hu = *reinterpret_cast<const uint32_t*>(&hb);
+    const float h0 = __uint_as_float(hu << 16);
+    const float h1 = __uint_as_float(hu & 0xffff0000u);
+    const __nv_bfloat162 lb = __floats2bfloat162_rn(x[2 * i] - h0, x[2 * i + 1] - h1);
+    hw[i] = hu;
+    lw[i] = *reinterpret_cast<const uint32_t*>(&lb);
+  }
+  hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+// hi half of x[0..7] into (hi_tile, hi_row), lo half into (lo_tile, lo_row),
+// both at 16-byte chunk col8.
+__device__ __forceinline__ void st_split8(uint8_t* hi_tile, uint32_t hi_row, uint8_t* lo_tile,
+                                          uint32_t lo_row, uint32_t col8, const float* x) {
+  uint4 hv, lv;
+  split8(x, hv, lv);
+  *reinterpret_cast<uint4*>(hi_tile + chunk_off(hi_row, col8)) = hv;
+  *reinterpret_cast<uint4*>(lo_tile + chunk_off(lo_row, col8)) = lv;
+}
+
+// 8 bf16 of chunk col8 of swizzled row `row`, as floats.
+__device__ __forceinline__ void ld_bf16x8(const uint8_t* tile, uint32_t row, uint32_t col8,
+                                          float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(tile + chunk_off(row, col8));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
 }
 
 __device__ __forceinline__ float ld_bf16(const uint8_t* tile, uint32_t row, uint32_t col) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col)));
+  return __bfloat162float(
+      *reinterpret_cast<const __nv_bfloat16*>(tile + sw128_offset(row, col)));
 }
 
 struct Mat2 { float a, b, c, d; };
@@ -107,6 +144,7 @@ __device__ __forceinline__ Mat2 mmul(const Mat2& x, const Mat2& y) {
   return {fmaf(x.a, y.a, x.b * y.c), fmaf(x.a, y.b, x.b * y.d), fmaf(x.c, y.a, x.d * y.c),
           fmaf(x.c, y.b, x.d * y.d)};
 }
+// Exact power-of-two renormalisation by the largest entry's binade.
 __device__ __forceinline__ Mat2 mnorm(const Mat2& x) {
   const float m = fmaxf(fmaxf(x.a, x.b), fmaxf(x.c, x.d));
   const int e = (int)((__float_as_uint(m) >> 23) & 0xffu) - 127;
@@ -117,42 +155,90 @@ __device__ __forceinline__ Mat2 mnorm(const Mat2& x) {
   return x;
 }
 
-// Issue K-steps of one MMA group: `steps` consecutive K=16 slices.
-// a0/b0: descriptors of the first slice; a_step/b_step: byte advance per slice
-// (applied to the 14-bit start-address field, >> 4).
+__device__ __forceinline__ void bar_compute() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory");
+}
+
+// `steps` consecutive K=16 MMAs; descriptor start addresses advance by
+// a_step / b_step bytes per step.
 __device__ __forceinline__ void mma_steps(uint32_t tmem_d, uint64_t a0, uint64_t b0,
                                           uint32_t a_step, uint32_t b_step, int steps,
                                           uint32_t idesc, bool accumulate_first) {
-  for (int s = 0; s < steps; ++s) {
-    const uint64_t a = a0 + (uint64_t)((s * a_step) >> 4);
-    const uint64_t b = b0 + (uint64_t)((s * b_step) >> 4);
-    umma_bf16(tmem_d, a, b, idesc, (accumulate_first || s > 0) ? 1u : 0u);
-  }
+  for (int s = 0; s < steps; ++s)
+    umma_bf16(tmem_d, a0 + (uint64_t)((s * a_step) >> 4), b0 + (uint64_t)((s * b_step) >> 4),
+              idesc, (accumulate_first || s > 0) ? 1u : 0u);
 }
 
-// K-major SW128 operand whose K extent spans two 64-column blocks `kb_stride`
-// apart: K-step s covers columns [16s, 16s+16).
-__device__ __forceinline__ void mma_kmajor_2blocks(uint32_t tmem_d, uint32_t a_base,
-                                                   uint32_t a_kb_stride, uint32_t a_sbo,
-                                                   uint32_t b_base, uint32_t b_kb_stride,
-                                                   uint32_t b_sbo, uint32_t b_lbo, uint32_t idesc,
-                                                   bool accumulate_first, bool b_mn,
-                                                   uint32_t b_mn_kstep) {
-  for (int kb = 0; kb < 2; ++kb) {
-    const uint64_t a0 = umma_desc_sw128(a_base + kb * a_kb_stride, 16, a_sbo);
-    uint64_t b0;
-    if (b_mn) {
-      b0 = umma_desc_sw128(b_base + kb * 4 * b_mn_kstep, b_lbo, b_sbo);
+// The off-diagonal 16x16 blocks of T = (I + A)^-1 at level D (block row i =
+// block column b + D): T_ib = -T_ii sum_{l=b}^{i-1} A_il T_lb, stored
+// transposed in the upper triangle, T_ib[r][c] at AT[16 b + c][16 i + r].
+// Each term A_il T_lb is a task of 64 threads (2x2 outputs each); every loop
+// bound is a compile-time constant.
+template <int D>
+__device__ __forceinline__ void t_level(float* AT, float* X, int tid) {
+  constexpr int NP = 4 - D;
+  const int task = tid >> 6, e = tid & 63;
+  const int r0 = 2 * (e >> 3), c0 = 2 * (e & 7);
+  if (task < NP * D) {
+    const int pr = task / D, bb = pr, ii = pr + D, l = bb + task % D;
+    float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+    const float* a_r0 = AT + (16 * ii + r0) * kLd + 16 * l;
+    if (l == bb) {
+      const float* tb = AT + (16 * bb) * kLd + 16 * bb + c0;
+#pragma unroll
+      for (int mm = 0; mm < 16; ++mm) {
+        const float2 tt = *reinterpret_cast<const float2*>(tb + mm * kLd);
+        const float a0v = a_r0[mm], a1v = a_r0[kLd + mm];
+        x00 = fmaf(a0v, tt.x, x00);
+        x01 = fmaf(a0v, tt.y, x01);
+        x10 = fmaf(a1v, tt.x, x10);
+        x11 = fmaf(a1v, tt.y, x11);
+      }
     } else {
-      b0 = umma_desc_sw128(b_base + kb * b_kb_stride, 16, b_sbo);
+      const float* tb = AT + (16 * bb + c0) * kLd + 16 * l;
+#pragma unroll
+      for (int mm = 0; mm < 16; ++mm) {
+        const float t0v = tb[mm], t1v = tb[kLd + mm];
+        const float a0v = a_r0[mm], a1v = a_r0[kLd + mm];
+        x00 = fmaf(a0v, t0v, x00);
+        x01 = fmaf(a0v, t1v, x01);
+        x10 = fmaf(a1v, t0v, x10);
+        x11 = fmaf(a1v, t1v, x11);
+      }
     }
-    mma_steps(tmem_d, a0, b0, 32, b_mn ? b_mn_kstep : 32, 4, idesc, accumulate_first || kb > 0);
+    float* xs = X + task * 288;  // [16][18]
+    *reinterpret_cast<float2*>(xs + r0 * 18 + c0) = make_float2(x00, x01);
+    *reinterpret_cast<float2*>(xs + (r0 + 1) * 18 + c0) = make_float2(x10, x11);
   }
+  bar_compute();
+  if (task < NP) {
+    const int pr = task, bb = pr, ii = pr + D;
+    const float* t_r0 = AT + (16 * ii + r0) * kLd + 16 * ii;
+    const float* xs = X + pr * D * 288 + c0;
+    float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < 16; ++mm) {
+      float2 xv = *reinterpret_cast<const float2*>(xs + mm * 18);
+#pragma unroll
+      for (int q = 1; q < D; ++q) {
+        const float2 v = *reinterpret_cast<const float2*>(xs + q * 288 + mm * 18);
+        xv.x += v.x;
+        xv.y += v.y;
+      }
+      const float ta = t_r0[mm], tb = t_r0[kLd + mm];
+      y00 = fmaf(ta, xv.x, y00);
+      y01 = fmaf(ta, xv.y, y01);
+      y10 = fmaf(tb, xv.x, y10);
+      y11 = fmaf(tb, xv.y, y11);
+    }
+    float* out = AT + (16 * bb + c0) * kLd + 16 * ii + r0;
+    out[0] = -y00;
+    out[1] = -y10;
+    out[kLd] = -y01;
+    out[kLd + 1] = -y11;
+  }
+  bar_compute();
 }
-
-struct Maps {
-  CUtensorMap q, k, v;
-};
 
 template <bool DIAG, int NV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -164,49 +250,57 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
                     float* __restrict__ P_out, int T, int H, int dv, float kappa,
                     uint32_t* __restrict__ err) {
   using P = Plan<DIAG, NV>;
-  constexpr int NVB = P::NVB;
-  constexpr int HC = NV / 2;  // value columns per warp in the epilogues
+  constexpr int HC = P::HC, QC = P::QC, NVB = NV / 64;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nvblk = dv / NV;
   const int bh = blockIdx.x / nvblk, vblk = blockIdx.x % nvblk;
   const int b = bh / H, h = bh % H;
   const int v0 = vblk * NV;
   const int nchunks = (T + kC - 1) / kC;
-  const int sub = warp & 3;      // TMEM lane quarter of this warp
-  const int colhalf = warp >> 2; // which half of the columns this warp handles
-
-  float* sA = reinterpret_cast<float*>(smem + P::OFF_SA);
-  float* sT = reinterpret_cast<float*>(smem + P::OFF_ST);
-  float* sX = reinterpret_cast<float*>(smem + P::OFF_X);
-  float* s_a = reinterpret_cast<float*>(smem + P::OFF_SC);
-  float* s_w = s_a + 64;
-  float* s_r = s_a + 128;
-  float* s_n = s_a + 192;
-  float* s_beta = s_a + 256;  // iso: beta_t; diag: 1 / s_t
-  float* s_lg = s_a + 320;
-  float* s_coef = s_a + 384;
-  float* s_misc = s_a + 448;  // [0]: p carry (iso), [1]: abort flag
-  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
-  uint64_t* bar_mma = bar_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 3);
   const uint32_t sbase = smem_u32(smem);
+
+  // scalar area (floats); [2][64] arrays are indexed by chunk parity
+  float* scf = reinterpret_cast<float*>(smem + P::OFF_SC);
+  float* sc_a = scf;           // decay a_t
+  float* sc_w = scf + 128;     // iso process noise w_t
+  float* sc_r = scf + 256;     // observation noise r_t
+  float* sc_n = scf + 384;     // iso ||k_t||^2
+  float* sc_beta = scf + 512;  // iso beta_t; diag 1 / s_t
+  float* sc_lg = scf + 640;    // log2 of the in-chunk cumulative decay
+  float* sc_coef = scf + 768;  // state-update coefficient
+  float* sc_pcar = scf + 896;  // [128] carried variance (iso: [0])
+  float* sc_misc = scf + 1024; // [0] abort flag
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
+  uint64_t* full_kq = bars;       // [2] K/Q tiles of a stage landed
+  uint64_t* full_v = bars + 2;    // V tile landed
+  uint64_t* mma1_bar = bars + 3;  // MMA1 (D1) finished
+  uint64_t* mma2_bar = bars + 4;  // MMA2 (D2) finished
+  uint64_t* mma_bar = bars + 5;   // MMA3, then MMA4 + MMA5, finished
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8);
+  float* AT = reinterpret_cast<float*>(smem + P::OFF_AT);
+  float* X = reinterpret_cast<float*>(smem + P::OFF_X);
   uint8_t* sS = smem + P::OFF_S;
   uint8_t* sTP = smem + P::OFF_TP;
   uint8_t* sG = smem + P::OFF_G;
+  uint8_t* sV = smem + P::OFF_V;
 
   if (tid == 0) {
-    mbar_init(&bar_full[0], 1);
-    mbar_init(&bar_full[1], 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(&full_kq[0], 1);
+    mbar_init(&full_kq[1], 1);
+    mbar_init(full_v, 1);
+    mbar_init(mma1_bar, 1);
+    mbar_init(mma2_bar, 1);
+    mbar_init(mma_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    s_misc[1] = 0.f;
+    sc_misc[0] = 0.f;
+  }
+  if (DIAG) {
+    if (tid < kDK) sc_pcar[tid] = P0 ? P0[(size_t)bh * kDK + tid] : 1.f;
+  } else if (tid == 0) {
+    sc_pcar[0] = P0 ? P0[bh] : 1.f;
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, P::TMEM_COLS);
@@ -215,594 +309,614 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_lane = (uint32_t)(32 * sub) << 16;
 
-  // ---- initial state: this thread holds S'[k][v] for k = 32*sub + lane and
-  //      v in [colhalf*HC, colhalf*HC + HC) of the CTA's value block.
-  const int my_k = 32 * sub + lane;
+  // ------------------------------------------------------- copy issue helpers
+  // per-token scalars of chunk c (warp kScalarWarp): loaded early into
+  // registers, stored into the chunk-parity slot later
+  float ps_a[2], ps_r[2], ps_w[2];
+  auto fetch_scalars = [&](int c) {
+    const int t0 = c * kC, valid = min(kC, T - t0);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int t = lane + 32 * i;
+      const bool in = t < valid;
+      const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+      ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
+      ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
+      ps_w[i] = (!DIAG && in) ? __ldg(Wg + tok) : 0.f;
+    }
+  };
+  auto store_scalars = [&](int c) {
+    const int st = c & 1;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int t = lane + 32 * i;
+      sc_a[64 * st + t] = ps_a[i];
+      sc_r[64 * st + t] = ps_r[i];
+      sc_w[64 * st + t] = ps_w[i];
+    }
+  };
+  // TMA copies (one thread): chunk c's K/Q tiles into stage c & 1, its V tile
+  int pend_kq[2] = {-1, -1}, pend_v = -1;  // parities of copies not yet seen landed
+  auto issue_kq = [&](int c) {
+    const int st = c & 1, t0 = c * kC;
+    uint8_t* kqd = smem + P::OFF_KQ + st * P::KQ_BYTES;
+    mbar_expect_tx(&full_kq[st], P::KQ_BYTES);
+    for (int kb = 0; kb < 2; ++kb)
+      for (int g = 0; g < 8; ++g) {
+        tma_load_4d(kqd + kb * 16384 + (2 * g) * 1024, &tm_k, &full_kq[st], kb * 64, h,
+                    t0 + 8 * g, b);
+        tma_load_4d(kqd + kb * 16384 + (2 * g + 1) * 1024, &tm_q, &full_kq[st], kb * 64, h,
+                    t0 + 8 * g, b);
+      }
+    pend_kq[st] = (c >> 1) & 1;
+  };
+  auto issue_v = [&](int c) {
+    mbar_expect_tx(full_v, P::V_BYTES);
+    for (int vb = 0; vb < NVB; ++vb)
+      tma_load_4d(sV + vb * 8192, &tm_v, full_v, v0 + 64 * vb, h, c * kC, b);
+    pend_v = c & 1;
+  };
+  const bool issuer = (warp == kIssueWarp && lane == 0);
+  if (issuer) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    issue_kq(0);
+    issue_v(0);
+  }
+  if (warp == kScalarWarp) {
+    fetch_scalars(0);
+    store_scalars(0);
+  }
+
+  // ----------------------------------------------------------- per-thread roles
+  const uint32_t tmem = *tmem_slot;
+  const int sub = warp & 3;  // TMEM lane quarter
+  const int cq = warp >> 2;  // column quarter
+  const uint32_t tm_lane = (uint32_t)(32 * sub) << 16;
+  const int m = 32 * sub + lane;     // row of a 128-row result held by this lane
+  const int tk = il_token(m);        // its token (interleaved results)
+  const int second = il_second(m);   // Q / lo row
+  const int my_k = m;                // state row k of this thread
+
+  // state S'[k][v], k = my_k, v in [HC cq, HC cq + HC) of this CTA's block
   float Sreg[HC];
   const size_t s_head = (size_t)bh * dv * kDK;
 #pragma unroll
-  for (int c = 0; c < HC; ++c) {
-    const int v = v0 + colhalf * HC + c;
-    Sreg[c] = S0 ? S0[s_head + (size_t)v * kDK + my_k] : 0.f;
-  }
-  // variance carry: iso in s_misc[0] (thread 0 of warp 0 owns it), diag in a
-  // register of threads 0..127 (dimension i = tid)
-  float p_dim = 1.f;
-  if (DIAG) {
-    if (tid < kDK) p_dim = P0 ? P0[(size_t)bh * kDK + tid] : 1.f;
-  } else if (tid == 0) {
-    s_misc[0] = P0 ? P0[bh] : 1.f;
-  }
+  for (int c = 0; c < HC; ++c)
+    Sreg[c] = S0 ? S0[s_head + (size_t)(v0 + HC * cq + c) * kDK + my_k] : 0.f;
 
   auto write_state_operand = [&]() {
-    // S' (K = k, N = v) as an MN-major operand: [vb][k 128][64 v], hi then lo
-    uint8_t* hi = sS;
-    uint8_t* lo = sS + P::SREG_BYTES / 2;
+    // S' as the MN-major B operand of MMA2: [vb][k 128][64 v]; hi, then lo
+    const int vcol = HC * cq;
+    uint8_t* base_hi = sS + (vcol >> 6) * 16384;
+    uint8_t* base_lo = base_hi + P::S_BYTES / 2;
 #pragma unroll
-    for (int c8 = 0; c8 < HC / 8; ++c8) {
-      const int v = colhalf * HC + c8 * 8;
-      const int vb = v >> 6;
-      st_split8(hi + vb * 16384, lo + vb * 16384, my_k, (v & 63) >> 3, &Sreg[c8 * 8]);
-    }
+    for (int i = 0; i < HC / 8; ++i)
+      st_split8(base_hi, (uint32_t)my_k, base_lo, (uint32_t)my_k,
+                (uint32_t)(((vcol & 63) >> 3) + i), &Sreg[8 * i]);
   };
   write_state_operand();
   fence_async_smem();
+  bar_compute();  // chunk 0's scalars are in place
 
-  auto issue_loads = [&](int c, int s) {
-    uint8_t* kq = smem + P::OFF_KQ + s * P::KQ_BYTES;
-    uint8_t* vv = smem + P::OFF_V + s * P::V_BYTES;
-    mbar_expect_tx(&bar_full[s], P::KQ_BYTES + P::V_BYTES);
-    const int t0 = c * kC;
-#pragma unroll 1
-    for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll 1
-      for (int g = 0; g < 8; ++g) {
-        tma_load_4d(kq + kb * 16384 + (2 * g) * 1024, &tm_k, &bar_full[s], kb * 64, h,
-                    t0 + 8 * g, b);
-        tma_load_4d(kq + kb * 16384 + (2 * g + 1) * 1024, &tm_q, &bar_full[s], kb * 64, h,
-                    t0 + 8 * g, b);
-      }
-    }
-#pragma unroll 1
-    for (int vb = 0; vb < NVB; ++vb)
-      tma_load_4d(vv + vb * 8192, &tm_v, &bar_full[s], v0 + vb * 64, h, t0, b);
-  };
-
-  // MMA issue helpers (thread 0 only)
   constexpr uint32_t ID_D1 = umma_idesc_bf16(128, 64, 0, 0);
   constexpr uint32_t ID_D2 = umma_idesc_bf16(128, NV, 0, 1);
   constexpr uint32_t ID_D34 = umma_idesc_bf16(128, NV, 0, 1);
   constexpr uint32_t ID_D5 = umma_idesc_bf16(128, NV, 1, 1);
 
-  // parity of a TMA stage load / MMA commit not yet seen complete (-1: none);
-  // only thread 0 issues, so only its copies matter for the drain
-  int pend_load[2] = {-1, -1};
-  int pend_mma = -1;
-  uint32_t mma_phase = 0;
-  if (tid == 0) {
-    issue_loads(0, 0);
-    pend_load[0] = 0;
-    if (nchunks > 1) {
-      issue_loads(1, 1);
-      pend_load[1] = 0;
-    }
-  }
-  __syncthreads();
-
-  // Bounded wait by every thread; on a timeout, record it and raise the abort
-  // flag that all threads check after the next barrier.
-  auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
-    if (!mbar_wait(bar, parity)) {
+  auto wait_or_abort = [&](uint64_t* bar_, uint32_t parity) -> bool {
+    if (!mbar_wait(bar_, parity)) {
       atomicOr(err, DEV_TIMEOUT);
-      s_misc[1] = 1.f;
+      sc_misc[0] = 1.f;
       return false;
     }
     return true;
   };
 
+  // iso: ||k_t||^2 (all threads), then warp 0's log2-decay prefix and Mobius
+  // scan of chunk c; the K tile and scalars of chunk c must be in place.
+  // Ends with a barrier.
+  auto iso_variance = [&](int c) {
+    const int cb = c & 1;
+    const uint8_t* kq = smem + P::OFF_KQ + cb * P::KQ_BYTES;
+    {
+      const int t = tid >> 3, part = tid & 7;  // 8 threads per token
+      float x[16];
+      const uint8_t* kt = kq + (part >> 2) * 16384;
+      ld_bf16x8(kt, (uint32_t)il_row(t, 0), (uint32_t)((part & 3) * 2), x);
+      ld_bf16x8(kt, (uint32_t)il_row(t, 0), (uint32_t)((part & 3) * 2 + 1), x + 8);
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc = fmaf(x[i], x[i], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (part == 0) sc_n[64 * cb + t] = acc;
+    }
+    bar_compute();
+    if (warp == 0) {
+      const float* a_s = sc_a + 64 * cb;
+      const float* w_s = sc_w + 64 * cb;
+      const float* r_s = sc_r + 64 * cb;
+      const int ta = 2 * lane, tb = ta + 1;
+      const float a0 = a_s[ta], a1 = a_s[tb];
+      const float l0 = __log2f(a0), l1 = __log2f(a1);
+      float incl = l0 + l1;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+      }
+      const float lg0 = incl - l1, lg1 = incl;
+      sc_lg[64 * cb + ta] = lg0;
+      sc_lg[64 * cb + tb] = lg1;
+      const float lg_last = __shfl_sync(0xffffffffu, lg1, 31);
+      const float n0 = sc_n[64 * cb + ta], n1 = sc_n[64 * cb + tb];
+      const float w0 = w_s[ta], w1 = w_s[tb], r0 = r_s[ta], r1 = r_s[tb];
+      const float c0 = kappa * n0, c1 = kappa * n1;
+      const Mat2 M0 = {r0 * a0 * a0, r0 * w0, c0 * a0 * a0, fmaf(c0, w0, r0)};
+      const Mat2 M1 = {r1 * a1 * a1, r1 * w1, c1 * a1 * a1, fmaf(c1, w1, r1)};
+      Mat2 Pm = mnorm(mmul(M1, M0));
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        Mat2 o;
+        o.a = __shfl_up_sync(0xffffffffu, Pm.a, d);
+        o.b = __shfl_up_sync(0xffffffffu, Pm.b, d);
+        o.c = __shfl_up_sync(0xffffffffu, Pm.c, d);
+        o.d = __shfl_up_sync(0xffffffffu, Pm.d, d);
+        if (lane >= d) Pm = mnorm(mmul(Pm, o));
+      }
+      Mat2 ex;
+      ex.a = __shfl_up_sync(0xffffffffu, Pm.a, 1);
+      ex.b = __shfl_up_sync(0xffffffffu, Pm.b, 1);
+      ex.c = __shfl_up_sync(0xffffffffu, Pm.c, 1);
+      ex.d = __shfl_up_sync(0xffffffffu, Pm.d, 1);
+      const float carry = sc_pcar[0];
+      float p = lane == 0 ? carry
+                          : __fdividef(fmaf(ex.a, carry, ex.b), fmaf(ex.c, carry, ex.d));
+      const float pp0 = fmaf(a0 * a0, p, w0);
+      p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
+      const float pp1 = fmaf(a1 * a1, p, w1);
+      p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
+      const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
+      const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
+      sc_beta[64 * cb + ta] = b0;
+      sc_beta[64 * cb + tb] = b1;
+      sc_coef[64 * cb + ta] = b0 * exp2f(lg_last - lg0);
+      sc_coef[64 * cb + tb] = b1 * exp2f(lg_last - lg1);
+      const float pnext = __shfl_sync(0xffffffffu, p, 31);
+      __syncwarp();
+      if (lane == 0) sc_pcar[0] = pnext;
+    }
+    bar_compute();
+  };
 
+  // diag: thread (di, dq) runs dimension di over tokens [16 dq, 16 dq + 16);
+  // its w values for the next chunk are prefetched into registers.
+  const int di = tid & 127, dq = tid >> 7;
+  float wpre[DIAG ? 16 : 1];
+  auto prefetch_w = [&](int c) {
+    if constexpr (DIAG) {
+      const int t0 = c * kC;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = t0 + 16 * dq + i;
+        wpre[i] = (c < nchunks && t < T)
+                      ? __ldg(Wg + (((size_t)b * T + t) * H + h) * kDK + di)
+                      : 0.f;
+      }
+    }
+  };
+  prefetch_w(0);
+
+  uint32_t mma_phase = 0;  // phase of mma_bar (two commits per chunk)
+  // parities of MMA commits not yet seen complete (thread 0), for the drain
+  int pend_mma = -1, pend_mma1 = -1, pend_mma2 = -1;
+  // output of the previous chunk, finished while the next chunk's MMAs run:
+  // gamma_t (Q S')_t for this lane's columns and the chunk's token range
+  float qpart[QC];
+  int prev_t0 = 0, prev_valid = 0;
+
+  auto finish_output = [&]() {
+    // o_t = D4 top + D4 bottom + gamma_t (Q S')_t (D4 holds the previous chunk)
+    float d4[HC];
+#pragma unroll
+    for (int i = 0; i < HC / 16; ++i) tmem_ld16(tmem + tm_lane + P::COL_D4 + HC * cq + 16 * i,
+                                                *reinterpret_cast<float(*)[16]>(d4 + 16 * i));
+    tmem_wait_ld();
+    float ov[QC];
+#pragma unroll
+    for (int i = 0; i < QC; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, second ? d4[i] : d4[QC + i], 8);
+      ov[i] = (second ? d4[QC + i] : d4[i]) + other + qpart[i];
+    }
+    if (tk < prev_valid) {
+      float* dst = O + (((size_t)b * T + prev_t0 + tk) * H + h) * dv + v0 + HC * cq + QC * second;
+#pragma unroll
+      for (int i = 0; i < QC; i += 4)
+        *reinterpret_cast<float4*>(dst + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+    }
+  };
+
+  if (!DIAG) {
+    if (wait_or_abort(&full_kq[0], 0u) && issuer) pend_kq[0] = -1;
+    iso_variance(0);
+  }
+
+  bool aborted = false;
   for (int c = 0; c < nchunks; ++c) {
     const int s = c & 1;
     const int t0 = c * kC;
     const int valid = min(kC, T - t0);
-    uint8_t* kq = smem + P::OFF_KQ + s * P::KQ_BYTES;
-    uint8_t* vv = smem + P::OFF_V + s * P::V_BYTES;
+    const bool more = c + 1 < nchunks;
     const uint32_t kq_a = sbase + P::OFF_KQ + s * P::KQ_BYTES;
+    const uint8_t* kq = smem + P::OFF_KQ + s * P::KQ_BYTES;
+    const float* a_s = sc_a + 64 * s;
+    const float* r_s = sc_r + 64 * s;
+    float* lg_c = sc_lg + 64 * s;
+    float* beta_c = sc_beta + 64 * s;
+    float* coef_c = sc_coef + 64 * s;
+    if (warp == kScalarWarp && more) fetch_scalars(c + 1);  // lands during this chunk
 
-    if (tid < kC) {
-      const bool in = tid < valid;
-      const size_t tok = ((size_t)b * T + t0 + tid) * H + h;
-      s_a[tid] = in ? Ag[tok] : 1.f;
-      s_r[tid] = in ? Rg[tok] : 1.f;
-      if (!DIAG) s_w[tid] = in ? Wg[tok] : 0.f;
-    }
-    if (wait_bar(&bar_full[s], (uint32_t)((c >> 1) & 1)) && tid == 0) pend_load[s] = -1;
+    if (wait_or_abort(&full_kq[s], (uint32_t)((c >> 1) & 1)) && issuer) pend_kq[s] = -1;
     tc_fence_before();
-    __syncthreads();
-    if (s_misc[1] != 0.f) break;
+    bar_compute();
+    if (sc_misc[0] != 0.f) { aborted = true; break; }
 
-    // ---- MMA2 (both variants) and MMA1 (iso) need only the tiles and S
     if (tid == 0) {
       tc_fence_after();
-      // D2 = [K;Q] S' (hi, then lo)
-      mma_kmajor_2blocks(tmem + P::COL_D2, kq_a, 16384, 1024, sbase + P::OFF_S, 0, 1024, 16384,
-                         ID_D2, false, true, 2048);
-      mma_kmajor_2blocks(tmem + P::COL_D2, kq_a, 16384, 1024,
-                         sbase + P::OFF_S + P::SREG_BYTES / 2, 0, 1024, 16384, ID_D2, true, true,
-                         2048);
       if (!DIAG) {
-        // D1 = [K;Q] K'  (B = the K rows: even 8-row groups, stride 2048 B)
-        mma_kmajor_2blocks(tmem + P::COL_D1, kq_a, 16384, 1024, kq_a, 16384, 2048, 16, ID_D1,
-                           false, false, 0);
+        // D1 = [K;Q] K' (B = the K rows: even 8-row groups, 2048 B apart)
+        for (int kb = 0; kb < 2; ++kb)
+          mma_steps(tmem + P::COL_D1, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
+                    umma_desc_sw128(kq_a + kb * 16384, 16, 2048), 32, 32, 4, ID_D1, kb > 0);
+        umma_commit(mma1_bar);
+        pend_mma1 = c & 1;
       }
-      if (!DIAG) {
-        umma_commit(bar_mma);
-        pend_mma = (int)mma_phase;
-      }
+      // D2 = [K;Q] S' : A K-major (d blocks 16 KB apart), B MN-major S' (hi, lo)
+      for (int hl = 0; hl < 2; ++hl)
+        for (int kb = 0; kb < 2; ++kb)
+          mma_steps(tmem + P::COL_D2, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
+                    umma_desc_sw128(sbase + P::OFF_S + hl * (P::S_BYTES / 2) + kb * 8192,
+                                    16384, 1024),
+                    32, 2048, 4, ID_D2, hl > 0 || kb > 0);
+      umma_commit(mma2_bar);
+      pend_mma2 = c & 1;
     }
+    // the next chunk's K/Q stage and scalars (their last readers are done)
+    if (issuer && more) issue_kq(c + 1);
+    if (warp == kScalarWarp && more) store_scalars(c + 1);
+    // the previous chunk's output (D4 is not overwritten before MMA4 below)
+    if (c > 0) finish_output();
 
-    // ---- per-token quantities
-    if (!DIAG) {
-      // n_t = ||k_t||^2 from the K tile (4 threads per token)
-      {
-        const int t = tid >> 2, q4 = tid & 3;
-        const int row = il_row(t, 0);
-        const uint8_t* tile = kq + (q4 >> 1) * 16384;
-        float acc = 0.f;
+    if constexpr (DIAG) {
+      // per-dimension variance: quarter products, exchanged through AT (free now)
+      float* mob = AT;  // [4 quarters][128 dims][4]
+      const int kb = di >> 6, col = di & 63;
+      const uint8_t* ktile = kq + kb * 16384;
+      float av[16], rv[16], kv[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t chunk = (uint32_t)((q4 & 1) * 4 + i);
-          const uint4 u = *reinterpret_cast<const uint4*>(
-              tile + row * 128 + ((chunk ^ (uint32_t)(row & 7)) << 4));
-          const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float lo = __uint_as_float(wds[j] << 16);
-            const float hi = __uint_as_float(wds[j] & 0xffff0000u);
-            acc = fmaf(lo, lo, acc);
-            acc = fmaf(hi, hi, acc);
-          }
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (q4 == 0) s_n[t] = acc;
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * dq + i;
+        av[i] = a_s[t];
+        rv[i] = r_s[t];
+        kv[i] = ld_bf16(ktile, (uint32_t)il_row(t, 0), (uint32_t)col);
       }
-      __syncthreads();
-      if (warp == 0) {
-        // lane l owns tokens 2l, 2l+1: log-decay prefix and the Mobius scan
-        const int t0l = 2 * lane, t1l = 2 * lane + 1;
-        const float a0 = s_a[t0l], a1 = s_a[t1l];
-        const float l0 = __logf(a0), l1 = __logf(a1);
+      Mat2 Pq = {1.f, 0.f, 0.f, 1.f};
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float kk = kv[i] * kv[i], a2 = av[i] * av[i];
+        const Mat2 M = {rv[i] * a2, rv[i] * wpre[i], kk * a2, fmaf(kk, wpre[i], rv[i])};
+        Pq = mmul(M, Pq);
+        if ((i & 3) == 3) Pq = mnorm(Pq);
+      }
+      *reinterpret_cast<float4*>(mob + (dq * 128 + di) * 4) = make_float4(Pq.a, Pq.b, Pq.c, Pq.d);
+      if (warp == 15) {
+        // log2 decay prefix
+        const int ta = 2 * lane, tb = ta + 1;
+        const float l0 = __log2f(a_s[ta]), l1 = __log2f(a_s[tb]);
         float incl = l0 + l1;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
           const float o = __shfl_up_sync(0xffffffffu, incl, d);
           if (lane >= d) incl += o;
         }
-        const float lg0 = incl - l1, lg1 = incl;
-        s_lg[t0l] = lg0;
-        s_lg[t1l] = lg1;
-        const float lg_last = __shfl_sync(0xffffffffu, lg1, 31);
-        const float n0 = s_n[t0l], n1 = s_n[t1l];
-        const float w0 = s_w[t0l], w1 = s_w[t1l], r0 = s_r[t0l], r1 = s_r[t1l];
-        const float c0 = kappa * n0, c1 = kappa * n1;
-        const Mat2 M0 = {r0 * a0 * a0, r0 * w0, c0 * a0 * a0, fmaf(c0, w0, r0)};
-        const Mat2 M1 = {r1 * a1 * a1, r1 * w1, c1 * a1 * a1, fmaf(c1, w1, r1)};
-        Mat2 Pm = mnorm(mmul(M1, M0));
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          Mat2 o;
-          o.a = __shfl_up_sync(0xffffffffu, Pm.a, d);
-          o.b = __shfl_up_sync(0xffffffffu, Pm.b, d);
-          o.c = __shfl_up_sync(0xffffffffu, Pm.c, d);
-          o.d = __shfl_up_sync(0xffffffffu, Pm.d, d);
-          if (lane >= d) Pm = mnorm(mmul(Pm, o));
-        }
-        Mat2 ex;
-        ex.a = __shfl_up_sync(0xffffffffu, Pm.a, 1);
-        ex.b = __shfl_up_sync(0xffffffffu, Pm.b, 1);
-        ex.c = __shfl_up_sync(0xffffffffu, Pm.c, 1);
-        ex.d = __shfl_up_sync(0xffffffffu, Pm.d, 1);
-        const float carry = s_misc[0];
-        float p = lane == 0 ? carry : __fdividef(fmaf(ex.a, carry, ex.b), fmaf(ex.c, carry, ex.d));
-        const float pp0 = fmaf(a0 * a0, p, w0);
-        p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
-        const float pp1 = fmaf(a1 * a1, p, w1);
-        p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
-        const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
-        const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
-        s_beta[t0l] = b0;
-        s_beta[t1l] = b1;
-        s_coef[t0l] = b0 * __expf(lg_last - lg0);
-        s_coef[t1l] = b1 * __expf(lg_last - lg1);
-        const float pnext = __shfl_sync(0xffffffffu, p, 31);
-        __syncwarp();
-        if (lane == 0) s_misc[0] = pnext;
+        lg_c[ta] = incl - l1;
+        lg_c[tb] = incl;
       }
-    } else {
-      // diag: dimension i = tid (< 128) runs the recursion over the chunk and
-      // writes the unnormalised gain G~ = p- * k (hi/lo, [kb][t][64]);
-      // warp 4 forms the log-decay prefix.
-      if (tid < kDK) {
-        const int i = tid;
-        const int kb = i >> 6, col = i & 63;
-        const uint8_t* ktile = kq + kb * 16384;
-        uint8_t* ghi = sG + kb * 8192;
-        uint8_t* glo = sG + 16384 + kb * 8192;
-        const size_t tok0 = ((size_t)b * T + t0) * H + h;
-        float wv[kC];
-#pragma unroll
-        for (int t = 0; t < kC; ++t)
-          wv[t] = (t < valid) ? Wg[(tok0 + (size_t)t * H) * kDK + i] : 0.f;
-        float p = p_dim;
-#pragma unroll
-        for (int t = 0; t < kC; ++t) {
-          const float a = s_a[t], r = s_r[t];
-          const float k = ld_bf16(ktile, il_row(t, 0), col);
-          const float pp = fmaf(a * a, p, wv[t]);
-          p = __fdividef(r * pp, fmaf(k * k, pp, r));
-          const float g = pp * k;
-          __nv_bfloat16 gh, gl;
-          split_bf16(g, gh, gl);
-          *reinterpret_cast<__nv_bfloat16*>(ghi + sw128_offset(t, col)) = gh;
-          *reinterpret_cast<__nv_bfloat16*>(glo + sw128_offset(t, col)) = gl;
-        }
-        p_dim = p;
-      } else if (warp == 4) {
-        const int t0l = 2 * lane, t1l = 2 * lane + 1;
-        const float l0 = __logf(s_a[t0l]), l1 = __logf(s_a[t1l]);
-        float incl = l0 + l1;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          const float o = __shfl_up_sync(0xffffffffu, incl, d);
-          if (lane >= d) incl += o;
-        }
-        s_lg[t0l] = incl - l1;
-        s_lg[t1l] = incl;
+      bar_compute();
+      float p = sc_pcar[di];
+      for (int q2 = 0; q2 < dq; ++q2) {
+        const float4 e = *reinterpret_cast<const float4*>(mob + (q2 * 128 + di) * 4);
+        p = __fdividef(fmaf(e.x, p, e.y), fmaf(e.z, p, e.w));
       }
+      uint8_t* ghi = sG + kb * 8192;
+      uint8_t* glo = sG + 16384 + kb * 8192;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * dq + i;
+        const float pp = fmaf(av[i] * av[i], p, wpre[i]);
+        p = __fdividef(rv[i] * pp, fmaf(kv[i] * kv[i], pp, rv[i]));
+        const float g = pp * kv[i];
+        const __nv_bfloat16 gh = __float2bfloat16_rn(g);
+        const __nv_bfloat16 gl = __float2bfloat16_rn(g - __bfloat162float(gh));
+        const uint32_t off = sw128_offset((uint32_t)t, (uint32_t)col);
+        *reinterpret_cast<__nv_bfloat16*>(ghi + off) = gh;
+        *reinterpret_cast<__nv_bfloat16*>(glo + off) = gl;
+      }
+      bar_compute();  // every quarter has read the old carry
+      if (dq == 3) sc_pcar[di] = p;
+      prefetch_w(c + 1);
       fence_async_smem();
-      __syncthreads();
+      bar_compute();
       if (tid == 0) {
+        tc_fence_after();
         // D1 = [K;Q] G~' (hi, then lo)
-        mma_kmajor_2blocks(tmem + P::COL_D1, kq_a, 16384, 1024, sbase + P::OFF_G, 8192, 1024, 16,
-                           ID_D1, false, false, 0);
-        mma_kmajor_2blocks(tmem + P::COL_D1, kq_a, 16384, 1024, sbase + P::OFF_G + 16384, 8192,
-                           1024, 16, ID_D1, true, false, 0);
-        umma_commit(bar_mma);
-        pend_mma = (int)mma_phase;
+        for (int hl = 0; hl < 2; ++hl)
+          for (int kb2 = 0; kb2 < 2; ++kb2)
+            mma_steps(tmem + P::COL_D1, umma_desc_sw128(kq_a + kb2 * 16384, 16, 1024),
+                      umma_desc_sw128(sbase + P::OFF_G + hl * 16384 + kb2 * 8192, 16, 1024),
+                      32, 32, 4, ID_D1, hl > 0 || kb2 > 0);
+        umma_commit(mma1_bar);
+        pend_mma1 = c & 1;
       }
     }
-    __syncthreads();
 
-    // ---- wait for MMA1 + MMA2
-    if (wait_bar(bar_mma, mma_phase)) pend_mma = -1;
-    mma_phase ^= 1u;
+    // ---------------- D1 epilogue: A (first-half rows), P (second-half rows)
+    if (wait_or_abort(mma1_bar, (uint32_t)(c & 1)) && tid == 0) pend_mma1 = -1;
     tc_fence_after();
-
-    // lane roles in the interleaved 128-row results
-    const int m = 32 * sub + lane;
-    const int tk = il_token(m);        // token of this lane's row
-    const bool second = il_second(m);  // Q row (D1, D2) / lo row (D3, D4)
-
-    // ---- D1 epilogue: A (first-half rows) and P (second-half rows)
-    float d1[32];
+    const float lg_t = lg_c[tk];
+    float preg[16];
     {
-      float tmp[16];
-      tmem_ld16(tmem + tm_lane + P::COL_D1 + colhalf * 32, tmp);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) d1[i] = tmp[i];
-      tmem_ld16(tmem + tm_lane + P::COL_D1 + colhalf * 32 + 16, tmp);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) d1[16 + i] = tmp[i];
+      float d1[16];
+      tmem_ld16(tmem + tm_lane + P::COL_D1 + 16 * cq, d1);
       tmem_wait_ld();
-    }
-    if (DIAG) {
-      // innovation variance s_t = (K G~')_tt + r_t; 1/s_t into s_beta
-      if (!second && (tk >> 5) == colhalf) s_beta[tk] = 1.f / (d1[tk & 31] + s_r[tk]);
-      __syncthreads();
-      if (tid < kC) {
-        s_coef[tid] = s_beta[tid] * __expf(s_lg[kC - 1] - s_lg[tid]);
+      if (DIAG) {
+        if (!second && (tk >> 4) == cq) beta_c[tk] = 1.f / (d1[tk & 15] + r_s[tk]);
+        bar_compute();
+        if (tid < kC) coef_c[tid] = beta_c[tid] * exp2f(lg_c[kC - 1] - lg_c[tid]);
       }
-    }
-    const float lg_t = s_lg[tk];
-    float preg[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int j = colhalf * 32 + i;
-      const float wj = s_beta[j];  // iso: beta_j; diag: 1/s_j
-      const float dec = __expf(lg_t - s_lg[j]);
-      const float val = dec * wj * d1[i];
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const float4 lgj = *reinterpret_cast<const float4*>(lg_c + 16 * cq + 4 * i4);
+        const float4 wj = *reinterpret_cast<const float4*>(beta_c + 16 * cq + 4 * i4);
+        const float lj[4] = {lgj.x, lgj.y, lgj.z, lgj.w};
+        const float bj[4] = {wj.x, wj.y, wj.z, wj.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 16 * cq + 4 * i4 + e;
+          const float v = exp2f(lg_t - lj[e]) * bj[e] * d1[4 * i4 + e];
+          preg[4 * i4 + e] = (j < tk + second) ? v : 0.f;  // A: j < t; P: j <= t
+        }
+      }
       if (!second) {
-        sA[tk * kScrLd + j] = (j < tk) ? val : 0.f;
-      } else {
-        preg[i] = (j <= tk) ? val : 0.f;
+        float* row = AT + tk * kLd + 16 * cq;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4)
+          *reinterpret_cast<float4*>(row + 4 * i4) =
+              make_float4(preg[4 * i4], preg[4 * i4 + 1], preg[4 * i4 + 2], preg[4 * i4 + 3]);
       }
     }
+    bar_compute();
 
-    // ---- D2 epilogue: Z = V - gamma K S' (first-half lanes take the first
-    //      half of this warp's columns, second-half lanes the rest)
+    // ---------------- T = (I + A)^-1 in place (overlaps MMA2)
+    // diagonal 16x16 blocks: column cc of block blk per thread (right-looking)
+    if (tid < 64) {
+      const int blk = tid >> 4, cc = tid & 15;
+      const float* Ab = AT + 16 * blk * kLd + 16 * blk;
+      float x[16], acc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int l = 0; l < 16; ++l) {
+        x[l] = (l == cc) ? 1.f : (l < cc ? 0.f : -acc[l]);
+#pragma unroll
+        for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kLd + l], x[l], acc[i]);
+      }
+      asm volatile("bar.sync 2, 64;" ::: "memory");  // all A columns read
+#pragma unroll
+      for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
+    }
+    bar_compute();
+    t_level<1>(AT, X, tid);
+    t_level<2>(AT, X, tid);
+    t_level<3>(AT, X, tid);
+    // T hi/lo into the interleaved A operand of MMA3: rows il_row(t, 0 | 1)
     {
-      const float gam = __expf(lg_t);
+      const int t = tid & 63, part = tid >> 6;  // columns [8 part, 8 part + 8)
+      const int bt = t >> 4, bj = part >> 1;
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int j = 8 * part + i;
+        x[i] = (bj == bt) ? AT[t * kLd + j] : (bj < bt ? AT[j * kLd + t] : 0.f);
+      }
+      st_split8(sTP, (uint32_t)il_row(t, 0), sTP, (uint32_t)il_row(t, 1), (uint32_t)part, x);
+    }
+    fence_async_smem();
+
+    // ---------------- D2 epilogue: Z = V - gamma K S'
+    if (wait_or_abort(mma2_bar, (uint32_t)(c & 1)) && tid == 0) pend_mma2 = -1;
+    tc_fence_after();
+    {
       float d2[HC];
 #pragma unroll
-      for (int c16 = 0; c16 < HC / 16; ++c16) {
-        float tmp[16];
-        tmem_ld16(tmem + tm_lane + P::COL_D2 + colhalf * HC + 16 * c16, tmp);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) d2[16 * c16 + i] = tmp[i];
-      }
+      for (int i = 0; i < HC / 16; ++i) tmem_ld16(tmem + tm_lane + P::COL_D2 + HC * cq + 16 * i,
+                                                  *reinterpret_cast<float(*)[16]>(d2 + 16 * i));
       tmem_wait_ld();
-      constexpr int QC = HC / 2;
+      if (wait_or_abort(full_v, (uint32_t)(c & 1)) && issuer) pend_v = -1;
+      const float gam = exp2f(lg_t);
+      const int vc = HC * cq + QC * second;  // this lane's first column
       float z[QC];
 #pragma unroll
       for (int i = 0; i < QC; ++i) {
         const float other = __shfl_xor_sync(0xffffffffu, d2[QC + i], 8);
-        const float ks = second ? other : d2[i];
-        const int v = colhalf * HC + (second ? QC : 0) + i;  // column within the CTA block
-        const float vv_ = ld_bf16(vv + (v >> 6) * 8192, tk, v & 63);
-        z[i] = vv_ - gam * ks;
+        z[i] = second ? other : d2[i];
       }
-      // Z hi -> sS[0 : ZU), Z lo -> sS[ZU : 2 ZU); layout [vb][t][64]
+      const uint8_t* vt = sV + (vc >> 6) * 8192;
+      uint8_t* zhi = sS + (vc >> 6) * 8192;
+      uint8_t* zlo = zhi + P::ZU_BYTES;
 #pragma unroll
-      for (int c8 = 0; c8 < QC / 8; ++c8) {
-        const int v = colhalf * HC + (second ? QC : 0) + c8 * 8;
-        st_split8(sS + (v >> 6) * 8192, sS + P::ZU_BYTES + (v >> 6) * 8192, tk, (v & 63) >> 3,
-                  &z[c8 * 8]);
+      for (int i8 = 0; i8 < QC / 8; ++i8) {
+        float vv[8];
+        ld_bf16x8(vt, (uint32_t)tk, (uint32_t)(((vc & 63) >> 3) + i8), vv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[8 * i8 + i] = fmaf(-gam, z[8 * i8 + i], vv[i]);
+        st_split8(zhi, (uint32_t)tk, zlo, (uint32_t)tk, (uint32_t)(((vc & 63) >> 3) + i8),
+                  z + 8 * i8);
       }
-    }
-    __syncthreads();
-
-    // ---- T = (I + A)^-1, blocked 16x16 forward substitution
-    if (tid < 64) {
-      const int blk = tid >> 4, cc = tid & 15;
-      float x[16];
+      // gamma_t (Q S')_t of this lane's output columns, kept for the output
+      // (D2 is overwritten by the next chunk's MMA2 before the output runs)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float acc = 0.f;
-#pragma unroll
-        for (int l = 0; l < i; ++l) acc = fmaf(sA[(16 * blk + i) * kScrLd + 16 * blk + l], x[l], acc);
-        x[i] = (i == cc) ? 1.f : (i < cc ? 0.f : -acc);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) sT[(16 * blk + i) * kScrLd + 16 * blk + cc] = x[i];
-    }
-    // upper blocks of T are zero
-    for (int e = tid; e < 64 * 64; e += kThreads) {
-      const int r = e >> 6, cl = e & 63;
-      if ((cl >> 4) > (r >> 4)) sT[r * kScrLd + cl] = 0.f;
-    }
-    __syncthreads();
-    // levels d = 1, 2, 3 of the block recursion T_ib = -T_ii sum_l A_il T_lb
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-      const int npairs = 4 - d;
-      const int r = tid >> 4, cc = tid & 15;
-      for (int pr = 0; pr < npairs; ++pr) {
-        const int bb = pr, ii = pr + d;
-        float acc = 0.f;
-        for (int l = bb; l < ii; ++l) {
-#pragma unroll
-          for (int mm = 0; mm < 16; ++mm)
-            acc = fmaf(sA[(16 * ii + r) * kScrLd + 16 * l + mm], sT[(16 * l + mm) * kScrLd + 16 * bb + cc], acc);
-        }
-        sX[pr * 272 + r * 17 + cc] = acc;
-      }
-      __syncthreads();
-      for (int pr = 0; pr < npairs; ++pr) {
-        const int bb = pr, ii = pr + d;
-        float acc = 0.f;
-#pragma unroll
-        for (int mm = 0; mm < 16; ++mm)
-          acc = fmaf(sT[(16 * ii + r) * kScrLd + 16 * ii + mm], sX[pr * 272 + mm * 17 + cc], acc);
-        sT[(16 * ii + r) * kScrLd + 16 * bb + cc] = -acc;
-      }
-      __syncthreads();
-    }
-    // T hi/lo into the interleaved A operand [128][64] (row il_row(t, 0|1))
-    {
-      const int t = tid >> 2, q = tid & 3;
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = sT[t * kScrLd + 16 * q + i];
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        __nv_bfloat16 hv[8], lv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) split_bf16(x[8 * half + i], hv[i], lv[i]);
-        const uint32_t col8 = (uint32_t)(2 * q + half);
-        *reinterpret_cast<uint4*>(sTP + sw128_offset(il_row(t, 0), col8 * 8)) =
-            make_uint4(pack2(hv[0], hv[1]), pack2(hv[2], hv[3]), pack2(hv[4], hv[5]), pack2(hv[6], hv[7]));
-        *reinterpret_cast<uint4*>(sTP + sw128_offset(il_row(t, 1), col8 * 8)) =
-            make_uint4(pack2(lv[0], lv[1]), pack2(lv[2], lv[3]), pack2(lv[4], lv[5]), pack2(lv[6], lv[7]));
+      for (int i = 0; i < QC; ++i) {
+        const float other = __shfl_xor_sync(0xffffffffu, d2[i], 8);
+        qpart[i] = gam * (second ? d2[QC + i] : other);
       }
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    bar_compute();
 
-    // ---- MMA3: D3 = [T_hi;T_lo] Z  (Z hi then lo; B MN-major [vb][t][64])
+    // ---------------- MMA3: D3 = [T_hi;T_lo] Z (Z hi then lo; B MN-major [vb][t][64])
     if (tid == 0) {
       tc_fence_after();
       const uint64_t a0 = umma_desc_sw128(sbase + P::OFF_TP, 16, 1024);
-      const uint64_t bz_hi = umma_desc_sw128(sbase + P::OFF_S, 8192, 1024);
-      const uint64_t bz_lo = umma_desc_sw128(sbase + P::OFF_S + P::ZU_BYTES, 8192, 1024);
-      mma_steps(tmem + P::COL_D3, a0, bz_hi, 32, 2048, 4, ID_D34, false);
-      mma_steps(tmem + P::COL_D3, a0, bz_lo, 32, 2048, 4, ID_D34, true);
-      umma_commit(bar_mma);
+      mma_steps(tmem + P::COL_D3, a0, umma_desc_sw128(sbase + P::OFF_S, 8192, 1024), 32, 2048,
+                4, ID_D34, false);
+      mma_steps(tmem + P::COL_D3, a0,
+                umma_desc_sw128(sbase + P::OFF_S + P::ZU_BYTES, 8192, 1024), 32, 2048, 4,
+                ID_D34, true);
+      umma_commit(mma_bar);
       pend_mma = (int)mma_phase;
     }
-    if (wait_bar(bar_mma, mma_phase)) pend_mma = -1;
+    if (issuer && more) issue_v(c + 1);  // the V tile is consumed
+    if (wait_or_abort(mma_bar, mma_phase) && tid == 0) pend_mma = -1;
     mma_phase ^= 1u;
     tc_fence_after();
 
-    // ---- D3 epilogue: U = top + bottom; U hi/lo and B = coef U hi/lo
+    // ---------------- D3 epilogue: U = top + bottom; U hi/lo and B = coef U hi/lo
     {
-      constexpr int QC = HC / 2;
       float d3[HC];
 #pragma unroll
-      for (int c16 = 0; c16 < HC / 16; ++c16) {
-        float tmp[16];
-        tmem_ld16(tmem + tm_lane + P::COL_D3 + colhalf * HC + 16 * c16, tmp);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) d3[16 * c16 + i] = tmp[i];
-      }
+      for (int i = 0; i < HC / 16; ++i) tmem_ld16(tmem + tm_lane + P::COL_D3 + HC * cq + 16 * i,
+                                                  *reinterpret_cast<float(*)[16]>(d3 + 16 * i));
       tmem_wait_ld();
-      float u[QC];
+      const int vc = HC * cq + QC * second;
+      float u[QC], bu[QC];
+      const float coef = coef_c[tk];
 #pragma unroll
       for (int i = 0; i < QC; ++i) {
         const float other = __shfl_xor_sync(0xffffffffu, second ? d3[i] : d3[QC + i], 8);
         u[i] = (second ? d3[QC + i] : d3[i]) + other;
+        bu[i] = coef * u[i];
       }
-      const float coef = s_coef[tk];
-      float bu[QC];
+      uint8_t* uhi = sS + (vc >> 6) * 8192;
 #pragma unroll
-      for (int i = 0; i < QC; ++i) bu[i] = coef * u[i];
-      // U -> sS[0 : 2ZU) (hi, lo); B -> sS[2ZU : 4ZU)
-#pragma unroll
-      for (int c8 = 0; c8 < QC / 8; ++c8) {
-        const int v = colhalf * HC + (second ? QC : 0) + c8 * 8;
-        const uint32_t vo = (uint32_t)(v >> 6) * 8192;
-        st_split8(sS + vo, sS + P::ZU_BYTES + vo, tk, (v & 63) >> 3, &u[c8 * 8]);
-        st_split8(sS + 2 * P::ZU_BYTES + vo, sS + 3 * P::ZU_BYTES + vo, tk, (v & 63) >> 3,
-                  &bu[c8 * 8]);
+      for (int i8 = 0; i8 < QC / 8; ++i8) {
+        const uint32_t col8 = (uint32_t)(((vc & 63) >> 3) + i8);
+        st_split8(uhi, (uint32_t)tk, uhi + P::ZU_BYTES, (uint32_t)tk, col8, u + 8 * i8);
+        st_split8(uhi + 2 * P::ZU_BYTES, (uint32_t)tk, uhi + 3 * P::ZU_BYTES, (uint32_t)tk, col8,
+                  bu + 8 * i8);
       }
-      // P hi/lo (held by the second-half lanes) into the interleaved A operand
       if (second) {
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          __nv_bfloat16 hv[8], lv[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) split_bf16(preg[8 * c8 + i], hv[i], lv[i]);
-          const uint32_t col = (uint32_t)(colhalf * 32 + 8 * c8);
-          *reinterpret_cast<uint4*>(sTP + sw128_offset(il_row(tk, 0), col)) =
-              make_uint4(pack2(hv[0], hv[1]), pack2(hv[2], hv[3]), pack2(hv[4], hv[5]), pack2(hv[6], hv[7]));
-          *reinterpret_cast<uint4*>(sTP + sw128_offset(il_row(tk, 1), col)) =
-              make_uint4(pack2(lv[0], lv[1]), pack2(lv[2], lv[3]), pack2(lv[4], lv[5]), pack2(lv[6], lv[7]));
-        }
+        // P hi/lo into the interleaved A operand of MMA4 (T is consumed)
+        st_split8(sTP, (uint32_t)il_row(tk, 0), sTP, (uint32_t)il_row(tk, 1),
+                  (uint32_t)(2 * cq), preg);
+        st_split8(sTP, (uint32_t)il_row(tk, 0), sTP, (uint32_t)il_row(tk, 1),
+                  (uint32_t)(2 * cq + 1), preg + 8);
       }
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (s_misc[1] != 0.f) break;
+    bar_compute();
+    if (sc_misc[0] != 0.f) { aborted = true; break; }
 
-    // ---- MMA4 (output) and MMA5 (state)
+    // ---------------- MMA4 (output) and MMA5 (state)
     if (tid == 0) {
       tc_fence_after();
       const uint64_t a0 = umma_desc_sw128(sbase + P::OFF_TP, 16, 1024);
-      const uint64_t bu_hi = umma_desc_sw128(sbase + P::OFF_S, 8192, 1024);
-      const uint64_t bu_lo = umma_desc_sw128(sbase + P::OFF_S + P::ZU_BYTES, 8192, 1024);
-      mma_steps(tmem + P::COL_D4, a0, bu_hi, 32, 2048, 4, ID_D34, false);
-      mma_steps(tmem + P::COL_D4, a0, bu_lo, 32, 2048, 4, ID_D34, true);
-      const uint64_t bb_hi = umma_desc_sw128(sbase + P::OFF_S + 2 * P::ZU_BYTES, 8192, 1024);
-      const uint64_t bb_lo = umma_desc_sw128(sbase + P::OFF_S + 3 * P::ZU_BYTES, 8192, 1024);
+      mma_steps(tmem + P::COL_D4, a0, umma_desc_sw128(sbase + P::OFF_S, 8192, 1024), 32, 2048,
+                4, ID_D34, false);
+      mma_steps(tmem + P::COL_D4, a0,
+                umma_desc_sw128(sbase + P::OFF_S + P::ZU_BYTES, 8192, 1024), 32, 2048, 4,
+                ID_D34, true);
+      const uint64_t b_hi = umma_desc_sw128(sbase + P::OFF_S + 2 * P::ZU_BYTES, 8192, 1024);
+      const uint64_t b_lo = umma_desc_sw128(sbase + P::OFF_S + 3 * P::ZU_BYTES, 8192, 1024);
       if (!DIAG) {
-        // A = K' (MN-major view of the K rows: d-blocks 16 KB apart, token
-        // groups 2048 B apart)
+        // A = K' (MN-major view of the K rows: d blocks 16 KB apart, token groups 2048 B)
         const uint64_t ak = umma_desc_sw128(kq_a, 16384, 2048);
-        mma_steps(tmem + P::COL_D5, ak, bb_hi, 4096, 2048, 4, ID_D5, false);
-        mma_steps(tmem + P::COL_D5, ak, bb_lo, 4096, 2048, 4, ID_D5, true);
+        mma_steps(tmem + P::COL_D5, ak, b_hi, 4096, 2048, 4, ID_D5, false);
+        mma_steps(tmem + P::COL_D5, ak, b_lo, 4096, 2048, 4, ID_D5, true);
       } else {
         const uint64_t ag_hi = umma_desc_sw128(sbase + P::OFF_G, 8192, 1024);
         const uint64_t ag_lo = umma_desc_sw128(sbase + P::OFF_G + 16384, 8192, 1024);
-        mma_steps(tmem + P::COL_D5, ag_hi, bb_hi, 2048, 2048, 4, ID_D5, false);
-        mma_steps(tmem + P::COL_D5, ag_hi, bb_lo, 2048, 2048, 4, ID_D5, true);
-        mma_steps(tmem + P::COL_D5, ag_lo, bb_hi, 2048, 2048, 4, ID_D5, true);
+        mma_steps(tmem + P::COL_D5, ag_hi, b_hi, 2048, 2048, 4, ID_D5, false);
+        mma_steps(tmem + P::COL_D5, ag_hi, b_lo, 2048, 2048, 4, ID_D5, true);
+        mma_steps(tmem + P::COL_D5, ag_lo, b_hi, 2048, 2048, 4, ID_D5, true);
       }
-      umma_commit(bar_mma);
+      umma_commit(mma_bar);
       pend_mma = (int)mma_phase;
     }
-    if (wait_bar(bar_mma, mma_phase)) pend_mma = -1;
+    // iso: the next chunk's ||k||^2 and variances, in the shadow of MMA4 + MMA5
+    if (!DIAG && more) {
+      if (wait_or_abort(&full_kq[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) & 1)) && issuer)
+        pend_kq[(c + 1) & 1] = -1;
+      iso_variance(c + 1);
+    }
+    if (wait_or_abort(mma_bar, mma_phase) && tid == 0) pend_mma = -1;
     mma_phase ^= 1u;
     tc_fence_after();
-    __syncthreads();
-    if (s_misc[1] != 0.f) break;
-    if (tid == 0 && c + 2 < nchunks) {
-      issue_loads(c + 2, s);
-      pend_load[s] = ((c + 2) >> 1) & 1;
-    }
 
-    // ---- output: o_t = D4 top + D4 bottom + gamma_t (Q S')_t
+    // ---------------- state: S' = gamma_C S' + D5, then its hi/lo operand
     {
-      constexpr int QC = HC / 2;
-      const float gam = __expf(lg_t);
-      float d4[HC], q2[HC];
+      const float gC = exp2f(lg_c[kC - 1]);
+      float d5[HC];
 #pragma unroll
-      for (int c16 = 0; c16 < HC / 16; ++c16) {
-        float tmp[16], tmp2[16];
-        tmem_ld16(tmem + tm_lane + P::COL_D4 + colhalf * HC + 16 * c16, tmp);
-        tmem_ld16(tmem + tm_lane + P::COL_D2 + colhalf * HC + 16 * c16, tmp2);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          d4[16 * c16 + i] = tmp[i];
-          q2[16 * c16 + i] = tmp2[i];
-        }
-      }
+      for (int i = 0; i < HC / 16; ++i) tmem_ld16(tmem + tm_lane + P::COL_D5 + HC * cq + 16 * i,
+                                                  *reinterpret_cast<float(*)[16]>(d5 + 16 * i));
       tmem_wait_ld();
-      float ov[QC];
 #pragma unroll
-      for (int i = 0; i < QC; ++i) {
-        const float send = second ? fmaf(gam, q2[i], d4[i]) : d4[QC + i];
-        const float other = __shfl_xor_sync(0xffffffffu, send, 8);
-        ov[i] = second ? (fmaf(gam, q2[QC + i], d4[QC + i]) + other) : (d4[i] + other);
-      }
-      if (tk < valid) {
-        const int vcol = v0 + colhalf * HC + (second ? QC : 0);
-        float* dst = O + (((size_t)b * T + t0 + tk) * H + h) * dv + vcol;
-#pragma unroll
-        for (int i = 0; i < QC; i += 4)
-          *reinterpret_cast<float4*>(dst + i) = make_float4(ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-      }
+      for (int e = 0; e < HC; ++e) Sreg[e] = fmaf(gC, Sreg[e], d5[e]);
     }
-
-    // ---- state: S' = gamma_C S' + D5
-    {
-      const float gC = __expf(s_lg[kC - 1]);
-#pragma unroll
-      for (int c16 = 0; c16 < HC / 16; ++c16) {
-        float tmp[16];
-        tmem_ld16(tmem + tm_lane + P::COL_D5 + colhalf * HC + 16 * c16, tmp);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Sreg[16 * c16 + i] = fmaf(gC, Sreg[16 * c16 + i], tmp[i]);
-      }
-    }
-    __syncthreads();  // all reads of U/B in sS are long done (MMA waited); S overwrites them
     write_state_operand();
+    prev_t0 = t0;
+    prev_valid = valid;
     fence_async_smem();
     tc_fence_before();
   }
-
-  // ---- drain (only the abort path has anything left): bounded waits for
-  //      the copies and MMAs still in flight before TMEM is released
-  if (tid == 0) {
-    for (int st = 0; st < 2; ++st)
-      if (pend_load[st] >= 0) (void)mbar_wait(&bar_full[st], (uint32_t)pend_load[st]);
-    if (pend_mma >= 0) (void)mbar_wait(bar_mma, (uint32_t)pend_mma);
+  if (!aborted && sc_misc[0] == 0.f && nchunks > 0) {
+    tc_fence_after();
+    finish_output();
   }
-  __syncthreads();
-  const bool aborted = s_misc[1] != 0.f;
 
-  // ---- final state and variance
-  if (!aborted) {
+  // ---- abort path: bounded waits for MMAs and copies still in flight
+  if (tid == 0) {
+    if (pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
+    if (pend_mma2 >= 0) (void)mbar_wait(mma2_bar, (uint32_t)pend_mma2);
+    if (pend_mma >= 0) (void)mbar_wait(mma_bar, (uint32_t)pend_mma);
+  }
+  if (issuer) {
+    for (int st = 0; st < 2; ++st)
+      if (pend_kq[st] >= 0) (void)mbar_wait(&full_kq[st], (uint32_t)pend_kq[st]);
+    if (pend_v >= 0) (void)mbar_wait(full_v, (uint32_t)pend_v);
+  }
+  bar_compute();
+  if (!aborted && sc_misc[0] == 0.f) {
 #pragma unroll
-    for (int c = 0; c < HC; ++c) {
-      const int v = v0 + colhalf * HC + c;
-      S_out[s_head + (size_t)v * kDK + my_k] = Sreg[c];
-    }
+    for (int c = 0; c < HC; ++c)
+      S_out[s_head + (size_t)(v0 + HC * cq + c) * kDK + my_k] = Sreg[c];
     if (vblk == 0) {
       if (DIAG) {
-        if (tid < kDK) P_out[(size_t)bh * kDK + tid] = p_dim;
+        if (tid < kDK) P_out[(size_t)bh * kDK + tid] = sc_pcar[tid];
       } else if (tid == 0) {
-        P_out[bh] = s_misc[0];
+        P_out[bh] = sc_pcar[0];
       }
     }
   }
   tc_fence_before();
-  __syncthreads();
+  bar_compute();
   if (warp == 0) tmem_dealloc(tmem, P::TMEM_COLS);
 }
 
@@ -882,9 +996,12 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
                                int T, int H, int dv, float kappa, void* ws, cudaStream_t s) {
-  if (diag) return launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
-  if (dv == 128) return launch<false, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
-  return launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+  if (dv == 128) {
+    return diag ? launch<true, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
+                : launch<false, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+  }
+  return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
+              : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
 }
 
 }  // namespace kdn

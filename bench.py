@@ -129,6 +129,23 @@ class ClockSampler:
                 'samples': len(sm)}
 
 
+def max_over_ranks(value, dist, device):
+    """The largest of every rank's value (all-reduce MAX); the value itself
+    when there is one rank."""
+    import torch
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_max_per_step):
+    """Units per second of the whole job: every rank processes
+    `units_per_rank` per step, and a step lasts as long as the slowest rank."""
+    return world * units_per_rank / (ms_max_per_step / 1000.0)
+
+
 def time_launches(fn, steps, warmup, stream):
     """CUDA-event time (ms) of `steps` back-to-back calls of fn on `stream`."""
     import torch
@@ -265,12 +282,9 @@ def main():
         ms = time_launches(step, args.steps, 0, stream)
     if dist:
         dist.barrier()
-    t = torch.tensor([ms], device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
     ms_step = ms_max / args.steps
-    value = world * B * T / (ms_step / 1000.0)
+    value = whole_job_rate(B * T, world, ms_step)
     alg = layer_bytes('iso', B, T, H, d, d)
     achieved = alg / (ms / args.steps / 1000.0) / 1e9
 
@@ -292,10 +306,7 @@ def main():
 
     e2e_steps = max(3, min(args.steps, 10))
     ms_e2e = time_launches(e2e_step, e2e_steps, 2, stream) / e2e_steps
-    te = torch.tensor([ms_e2e], device=dev)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * B * T / (float(te.item()) / 1000.0)
+    e2e_value = whole_job_rate(B * T, world, max_over_ranks(ms_e2e, dist, dev))
 
     secondary = {}
     if not args.no_secondary and rank == 0:

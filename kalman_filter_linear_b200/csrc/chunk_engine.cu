@@ -56,6 +56,7 @@ constexpr int kCompute = 512;            // 16 warps
 constexpr int kThreads = kCompute;
 constexpr int kIssueWarp = 15;           // its lane 0 issues the TMA copies
 constexpr int kScalarWarp = 14;          // fetches the per-token scalars
+constexpr int kMma2Warp = 13;            // its lane 0 issues MMA2
 constexpr int kLd = 68;                  // fp32 row stride of the 64x64 solve buffer
 
 template <bool DIAG, int NV>
@@ -358,6 +359,7 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
     pend_v = c & 1;
   };
   const bool issuer = (warp == kIssueWarp && lane == 0);
+  const bool mma2_issuer = (warp == kMma2Warp && lane == 0);
   if (issuer) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -565,28 +567,16 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
     bar_compute();
     if (sc_misc[0] != 0.f) { aborted = true; break; }
 
-    if (tid == 0) {
+    if (!DIAG && tid == 0) {
       tc_fence_after();
-      if (!DIAG) {
-        // D1 = [K;Q] K' (B = the K rows: even 8-row groups, 2048 B apart)
-        for (int kb = 0; kb < 2; ++kb)
-          mma_steps(tmem + P::COL_D1, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
-                    umma_desc_sw128(kq_a + kb * 16384, 16, 2048), 32, 32, 4, ID_D1, kb > 0);
-        umma_commit(mma1_bar);
-        pend_mma1 = c & 1;
-      }
-      // D2 = [K;Q] S' : A K-major (d blocks 16 KB apart), B MN-major S' (hi, lo)
-      for (int hl = 0; hl < 2; ++hl)
-        for (int kb = 0; kb < 2; ++kb)
-          mma_steps(tmem + P::COL_D2, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
-                    umma_desc_sw128(sbase + P::OFF_S + hl * (P::S_BYTES / 2) + kb * 8192,
-                                    16384, 1024),
-                    32, 2048, 4, ID_D2, hl > 0 || kb > 0);
-      umma_commit(mma2_bar);
-      pend_mma2 = c & 1;
+      // D1 = [K;Q] K' (B = the K rows: even 8-row groups, 2048 B apart)
+      for (int kb = 0; kb < 2; ++kb)
+        mma_steps(tmem + P::COL_D1, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
+                  umma_desc_sw128(kq_a + kb * 16384, 16, 2048), 32, 32, 4, ID_D1, kb > 0);
+      umma_commit(mma1_bar);
+      pend_mma1 = c & 1;
     }
-    // the next chunk's K/Q stage and scalars (their last readers are done)
-    if (issuer && more) issue_kq(c + 1);
+    // the next chunk's scalars (their last readers are done)
     if (warp == kScalarWarp && more) store_scalars(c + 1);
     // the previous chunk's output (D4 is not overwritten before MMA4 below)
     if (c > 0) finish_output();
@@ -718,6 +708,20 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
       asm volatile("bar.sync 2, 64;" ::: "memory");  // all A columns read
 #pragma unroll
       for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
+    } else if (mma2_issuer) {
+      // D2 = [K;Q] S' (A K-major, d blocks 16 KB apart; B MN-major S', hi then lo).
+      // Issued here, while only two warps work, because issuing blocks.
+      tc_fence_after();
+      for (int hl = 0; hl < 2; ++hl)
+        for (int kb = 0; kb < 2; ++kb)
+          mma_steps(tmem + P::COL_D2, umma_desc_sw128(kq_a + kb * 16384, 16, 1024),
+                    umma_desc_sw128(sbase + P::OFF_S + hl * (P::S_BYTES / 2) + kb * 8192,
+                                    16384, 1024),
+                    32, 2048, 4, ID_D2, hl > 0 || kb > 0);
+      umma_commit(mma2_bar);
+      pend_mma2 = c & 1;
+    } else if (issuer && more) {
+      issue_kq(c + 1);  // stage (c+1) & 1 was released when chunk c-1's MMA5 finished
     }
     bar_compute();
     t_level<1>(AT, X, tid);
@@ -738,7 +742,7 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
     fence_async_smem();
 
     // ---------------- D2 epilogue: Z = V - gamma K S'
-    if (wait_or_abort(mma2_bar, (uint32_t)(c & 1)) && tid == 0) pend_mma2 = -1;
+    if (wait_or_abort(mma2_bar, (uint32_t)(c & 1)) && mma2_issuer) pend_mma2 = -1;
     tc_fence_after();
     {
       float d2[HC];
@@ -894,9 +898,9 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
   // ---- abort path: bounded waits for MMAs and copies still in flight
   if (tid == 0) {
     if (pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
-    if (pend_mma2 >= 0) (void)mbar_wait(mma2_bar, (uint32_t)pend_mma2);
     if (pend_mma >= 0) (void)mbar_wait(mma_bar, (uint32_t)pend_mma);
   }
+  if (mma2_issuer && pend_mma2 >= 0) (void)mbar_wait(mma2_bar, (uint32_t)pend_mma2);
   if (issuer) {
     for (int st = 0; st < 2; ++st)
       if (pend_kq[st] >= 0) (void)mbar_wait(&full_kq[st], (uint32_t)pend_kq[st]);

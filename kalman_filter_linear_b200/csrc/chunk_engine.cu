@@ -156,8 +156,11 @@ __device__ __forceinline__ Mat2 mnorm(const Mat2& x) {
   return x;
 }
 
+// Named barriers use the non-aligned form: threads of a warp may arrive
+// separately (single-lane issue blocks and bounded waits diverge a warp), and
+// each thread is counted on its own.
 __device__ __forceinline__ void bar_compute() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory");
+  asm volatile("barrier.sync 1, %0;" ::"n"(kCompute) : "memory");
 }
 
 // `steps` consecutive K=16 MMAs; descriptor start addresses advance by
@@ -175,7 +178,14 @@ __device__ __forceinline__ void mma_steps(uint32_t tmem_d, uint64_t a0, uint64_t
 // transposed in the upper triangle, T_ib[r][c] at AT[16 b + c][16 i + r].
 // Each term A_il T_lb is a task of 64 threads (2x2 outputs each); every loop
 // bound is a compile-time constant.
-template <int D>
+template <int BAR, int NT>
+__device__ __forceinline__ void named_bar() {
+  asm volatile("barrier.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
+// Every level uses at most 256 threads (tid < 256); BAR / NT name the barrier
+// of the threads that run the solve.
+template <int D, int BAR = 1, int NT = kCompute>
 __device__ __forceinline__ void t_level(float* AT, float* X, int tid) {
   constexpr int NP = 4 - D;
   const int task = tid >> 6, e = tid & 63;
@@ -211,7 +221,7 @@ __device__ __forceinline__ void t_level(float* AT, float* X, int tid) {
     *reinterpret_cast<float2*>(xs + r0 * 18 + c0) = make_float2(x00, x01);
     *reinterpret_cast<float2*>(xs + (r0 + 1) * 18 + c0) = make_float2(x10, x11);
   }
-  bar_compute();
+  named_bar<BAR, NT>();
   if (task < NP) {
     const int pr = task, bb = pr, ii = pr + D;
     const float* t_r0 = AT + (16 * ii + r0) * kLd + 16 * ii;
@@ -238,7 +248,7 @@ __device__ __forceinline__ void t_level(float* AT, float* X, int tid) {
     out[kLd] = -y01;
     out[kLd + 1] = -y11;
   }
-  bar_compute();
+  named_bar<BAR, NT>();
 }
 
 template <bool DIAG, int NV>
@@ -705,7 +715,7 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kLd + l], x[l], acc[i]);
       }
-      asm volatile("bar.sync 2, 64;" ::: "memory");  // all A columns read
+      named_bar<2, 64>();  // all A columns read
 #pragma unroll
       for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
     } else if (mma2_issuer) {
@@ -924,6 +934,787 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (warp == 0) tmem_dealloc(tmem, P::TMEM_COLS);
 }
 
+// ===========================================================================
+// Warp-specialised isotropic engine (one CTA per head, d_v = 128).
+//
+// Every product runs transposed, with the value index v on the 128 TMEM lanes,
+// so that the fp32 state S'^T [v][k] itself is the A operand (tf32, read from
+// TMEM) of the product with the chunk's keys and queries, and every operand a
+// lane needs later is its own row:
+//   D2 = V^T [I;0] + S'^T [-gamma K ; gamma Q]^T    Z^T (key half), gamma (Q S')^T
+//   D3 = Z^T T^T                                    U^T (bf16 hi/lo Z and T)
+//   D2 (query half) += U^T P^T                      o^T
+//   S'^T = gamma_C S'^T + B^T K,  B = coef U        (bf16 hi/lo B, exact K)
+// The tf32 products take operands rounded to nearest (P, -gamma K, gamma Q);
+// U and S' are read as the tensor cores truncate them.  Z and T enter the
+// state path, so their product keeps three bf16 hi/lo terms.
+//
+// Warps 0-7 (the chain) run the part that depends on the state, with three
+// small TMEM passes per chunk: Z in bf16 hi/lo plus the state decay, B = coef U
+// in bf16 hi/lo, and the output copy.  Warps 8-15 (prep) run the part that depends
+// only on the chunk's inputs, one chunk ahead: the decay prefix, the fp32
+// key/query copies, the variance scan, MMA1, A and P, and T = (I + A)^-1.
+// The groups hand buffers over through mbarriers:
+//   kq32_ready / t_ready / p_ready   prep -> chain (with the chunk's scalars)
+//   mma2 / mma3 / mma4               the chain's commits; they also hand the
+//                                    fp32 key/query copy, T and P back to prep
+// A K/Q stage is refilled (chunk c + 2) once MMA5 of chunk c has finished.
+// TMEM columns: D1 [0,64) (prep); S'^T [64,192); D2 [192,320) (key half, then
+// query half); D3 [320,384); B^T hi [384,416), lo [416,448); Z^T hi [448,480),
+// lo [480,512).
+// ===========================================================================
+struct WsPlan {
+  static constexpr uint32_t KQ_BYTES = 32768;           // bf16 [kb 2][K|Q][64 t][64]
+  static constexpr uint32_t OFF_KQ = 0;                 // two stages
+  static constexpr uint32_t OFF_KQ32 = 2 * KQ_BYTES;    // fp32 [kb 4][128 L][32]
+  static constexpr uint32_t OFF_V = OFF_KQ32 + 65536;   // bf16 [vb 2][64 t][64 v]
+  static constexpr uint32_t OFF_I = OFF_V + 16384;      // bf16 [128 L][64 u]: I over 0
+  static constexpr uint32_t OFF_T = OFF_I + 16384;      // bf16 hi, lo [64 t][64 j]
+  static constexpr uint32_t OFF_P = OFF_T + 16384;      // fp32 [jb 2][64 t][32 j]
+  static constexpr uint32_t OFF_AT = OFF_P + 16384;     // fp32 [64][68]
+  static constexpr uint32_t OFF_X = OFF_AT + 64u * kLd * 4u;
+  static constexpr uint32_t OFF_SC = OFF_X + 5120u;     // X: fp32 [4][16][20]
+  static constexpr uint32_t OFF_BAR = OFF_SC + 6144u;
+  static constexpr uint32_t TOTAL = OFF_BAR + 256u;
+  static constexpr uint32_t ALLOC = TOTAL + 1024u;
+  static constexpr uint32_t COL_D1 = 0, COL_ST = 64, COL_D2 = 192, COL_D3 = 320, COL_B = 384,
+                            COL_Z = 448;
+  static_assert(TOTAL <= 227u * 1024u, "shared memory plan too large");
+  static_assert(OFF_KQ32 % 1024 == 0 && OFF_V % 1024 == 0 && OFF_I % 1024 == 0 &&
+                    OFF_T % 1024 == 0 && OFF_P % 1024 == 0,
+                "operand alignment");
+};
+
+// (hi, lo) bf16 splits of two consecutive K elements, packed low-first as a
+// 32-bit TMEM column of a bf16 A operand.
+__device__ __forceinline__ void split_pack2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+  hi = *reinterpret_cast<const uint32_t*>(&hb);
+  const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16),
+                                                  x1 - __uint_as_float(hi & 0xffff0000u));
+  lo = *reinterpret_cast<const uint32_t*>(&lb);
+}
+
+// --------------------------------------------- 16x16 products on warp MMAs
+// The off-diagonal blocks of T come from 16x16x16 products done by single
+// warps with mma.sync (m16n8k8, tf32).  Each operand is split x = hi + lo in
+// tf32 and the product keeps hi*hi + hi*lo + lo*hi in three accumulators, which
+// leaves about fp32 accuracy.  Fragment layout of m16n8k8 (g = lane / 4,
+// q = lane % 4): A (16x8) rows g, g+8 x cols q, q+4; B (8x8) rows q, q+4 x col
+// g; C (16x8) rows g, g+8 x cols 2q, 2q+1.
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = rna_tf32(x);
+  lo = rna_tf32(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
+                                                const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// acc[term][n tile] += A (16x16, element A(r, k)) * B (16x16, element B(k, n))
+template <class FA, class FB>
+__device__ __forceinline__ void warp_mm16(float (&acc)[3][2][4], FA A, FB B, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    uint32_t ah[4], al[4];
+    split_tf32(A(g, 8 * ks + q), ah[0], al[0]);
+    split_tf32(A(g + 8, 8 * ks + q), ah[1], al[1]);
+    split_tf32(A(g, 8 * ks + q + 4), ah[2], al[2]);
+    split_tf32(A(g + 8, 8 * ks + q + 4), ah[3], al[3]);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      uint32_t bh[2], bl[2];
+      split_tf32(B(8 * ks + q, 8 * nt + g), bh[0], bl[0]);
+      split_tf32(B(8 * ks + q + 4, 8 * nt + g), bh[1], bl[1]);
+      mma_tf32_16x8x8(acc[0][nt], ah, bh);
+      mma_tf32_16x8x8(acc[1][nt], ah, bl);
+      mma_tf32_16x8x8(acc[2][nt], al, bh);
+    }
+  }
+}
+// Hand the summed 16x16 result, scaled by s, to C(r, c, v_c, v_c+1) in pairs.
+template <class FC>
+__device__ __forceinline__ void warp_put16(const float (&acc)[3][2][4], float s, FC C, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = s * (acc[2][nt][e] + acc[1][nt][e] + acc[0][nt][e]);
+    C(g, 8 * nt + 2 * q, v[0], v[1]);
+    C(g + 8, 8 * nt + 2 * q, v[2], v[3]);
+  }
+}
+
+constexpr int kChainBar = 3, kPrepBar = 4, kPhase1Bar = 5, kGroup = 256;
+
+__device__ __forceinline__ void bar_group(int id) {
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "n"(kGroup) : "memory");
+}
+
+// Barrier of one 256-thread group that also ORs a flag over the group, so an
+// abort decision taken after it is the same in every thread of the group.
+__device__ __forceinline__ bool bar_group_or(int id, bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)flag), "r"(id), "n"(kGroup)
+      : "memory");
+  return r != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ Ag,
+                       const float* __restrict__ Wg, const float* __restrict__ Rg,
+                       const float* S0, const float* __restrict__ P0, float* __restrict__ O,
+                       float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
+                       uint32_t* __restrict__ err) {
+  using P = WsPlan;
+  constexpr int DV = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  const int b = bh / H, h = bh % H;
+  const int nchunks = (T + kC - 1) / kC;
+  const uint32_t sbase = smem_u32(smem);
+
+  // scalar area (floats); [2][64] arrays are indexed by chunk parity
+  float* scf = reinterpret_cast<float*>(smem + P::OFF_SC);
+  float* sc_a = scf;            // decay a_t
+  float* sc_w = scf + 128;      // process noise w_t
+  float* sc_r = scf + 256;      // observation noise r_t
+  float* sc_n = scf + 384;      // [2 halves][64] partial ||k_t||^2
+  float* sc_beta = scf + 512;   // beta_t
+  float* sc_lg = scf + 640;     // log2 of the in-chunk cumulative decay
+  float* sc_gam = scf + 768;    // gamma_t
+  float* sc_coef = scf + 896;   // state-update coefficient
+  float* sc_gC = scf + 1024;    // [2] gamma of the whole chunk
+  float* sc_pcar = scf + 1026;  // carried variance
+  volatile float* sc_abort = scf + 1027;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
+  uint64_t* full_kq = bars;         // [2] K/Q tiles of a stage landed
+  uint64_t* full_v = bars + 2;      // V tile landed
+  uint64_t* mma1_bar = bars + 3;    // MMA1 finished (D1)
+  uint64_t* mma2_bar = bars + 4;    // MMA2 finished: fp32 K/Q copy and V free
+  uint64_t* mma3_bar = bars + 5;    // MMA3 finished: T free
+  uint64_t* mma4_bar = bars + 6;    // MMA4 finished: P free, output ready
+  uint64_t* mma5_bar = bars + 7;    // MMA5 finished: state updated, stage free
+  uint64_t* kq32_ready = bars + 8;  // fp32 K/Q copy and decay scalars written
+  uint64_t* t_ready = bars + 9;     // T and the update coefficients written
+  uint64_t* p_ready = bars + 10;    // P written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  float* AT = reinterpret_cast<float*>(smem + P::OFF_AT);
+  float* X = reinterpret_cast<float*>(smem + P::OFF_X);
+  uint8_t* sKQ32 = smem + P::OFF_KQ32;
+  uint8_t* sT = smem + P::OFF_T;
+  uint8_t* sP = smem + P::OFF_P;
+  uint8_t* sI = smem + P::OFF_I;
+  uint8_t* sV = smem + P::OFF_V;
+
+  if (tid == 0) {
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    *sc_abort = 0.f;
+    sc_pcar[0] = P0 ? P0[bh] : 1.f;
+  }
+  // [I; 0]: bf16 K-major rows L of 64 u, 1.0 at u = L for L < 64
+  for (int i = tid; i < 1024; i += kThreads) {
+    const int L = i >> 3, q = i & 7;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (L < 64 && (L >> 3) == q) w[(L & 7) >> 1] = 0x3F80u << (16 * (L & 1));
+    *reinterpret_cast<uint4*>(sI + chunk_off((uint32_t)L, (uint32_t)q)) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+    // T operand (hi, lo): blocks above the diagonal are never written again
+    *reinterpret_cast<uint4*>(sT + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_async_smem();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // Bounded wait; once any thread has recorded a timeout every later wait
+  // fails at once, so an aborting CTA ends within a few wait limits.
+  auto fail1 = [&](uint64_t* bar_, uint32_t parity) -> bool {
+    if (*sc_abort != 0.f) return true;
+    if (!mbar_wait(bar_, parity)) {
+      atomicOr(err, DEV_TIMEOUT);
+      *sc_abort = 1.f;
+      return true;
+    }
+    return false;
+  };
+  auto fail = fail1;
+
+  const int m = 32 * (warp & 3) + lane;  // TMEM lane of this thread
+  const uint32_t tm_lane = (uint32_t)(32 * (warp & 3)) << 16;
+
+  if (warp < 8) {
+    // ================================================================ chain
+    const int ch = warp >> 2;  // tokens [32 ch, 32 ch + 32), state columns [64 ch, 64 ch + 64)
+    const int v = m;           // value index of this lane
+    const bool issuer = (warp == 0 && lane == 0);
+    constexpr uint32_t ID_V = umma_idesc(128, 128, 1, 1, 0);   // bf16, A MN-major
+    constexpr uint32_t ID_2 = umma_idesc(128, 128, 2, 0, 0);   // tf32
+    constexpr uint32_t ID_3 = umma_idesc(128, 64, 1, 0, 0);    // bf16
+    constexpr uint32_t ID_4 = umma_idesc(128, 64, 2, 0, 0);    // tf32
+    constexpr uint32_t ID_5 = umma_idesc(128, 128, 1, 0, 1);   // bf16, B MN-major
+
+    int pend_kq[2] = {-1, -1}, pend_v = -1;  // copies not yet seen landed (issuer)
+    auto issue_kq = [&](int c) {
+      const int st = c & 1, t0 = c * kC;
+      uint8_t* kqd = smem + P::OFF_KQ + st * P::KQ_BYTES;
+      mbar_expect_tx(&full_kq[st], P::KQ_BYTES);
+      for (int kb = 0; kb < 2; ++kb) {
+        tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, t0, b);
+        tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, t0, b);
+      }
+      pend_kq[st] = (c >> 1) & 1;
+    };
+    auto issue_v = [&](int c) {
+      mbar_expect_tx(full_v, 16384);
+      tma_load_4d(sV, &tm_v, full_v, 0, h, c * kC, b);
+      tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
+      pend_v = c & 1;
+    };
+    if (issuer) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      issue_kq(0);
+      issue_v(0);
+      if (nchunks > 1) issue_kq(1);
+    }
+
+    // S'^T [v][k] into TMEM, k in [64 ch, 64 ch + 64)
+    const size_t s_row = ((size_t)bh * DV + v) * kDK + 64 * ch;
+#pragma unroll
+    for (int h32 = 0; h32 < 2; ++h32) {
+      uint32_t r[32];
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        const float4 x = S0 ? *reinterpret_cast<const float4*>(S0 + s_row + 32 * h32 + i)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        r[i] = __float_as_uint(x.x);
+        r[i + 1] = __float_as_uint(x.y);
+        r[i + 2] = __float_as_uint(x.z);
+        r[i + 3] = __float_as_uint(x.w);
+      }
+      tmem_st32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, r);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    bar_group(kChainBar);
+
+    int pend_mma2 = -1, pend_mma3 = -1, pend_mma4 = -1, pend_mma5 = -1;
+    bool bad = false;
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      const int t0 = c * kC;
+      const uint32_t kq_a = sbase + P::OFF_KQ + s * P::KQ_BYTES;
+      if (fail(kq32_ready, (uint32_t)(c & 1))) bad = true;
+      if (fail(full_v, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_v = -1;
+      if (issuer) {
+        if (fail1(&full_kq[s], (uint32_t)((c >> 1) & 1))) bad = true;
+        else pend_kq[s] = -1;
+      }
+      // ---- MMA2: D2 = V^T [I;0] + S'^T [-gamma K; gamma Q]^T
+      if (issuer && !bad) {
+        tc_fence_after();
+        for (int ks = 0; ks < 4; ++ks)
+          umma_bf16(tmem + P::COL_D2, umma_desc_sw128(sbase + P::OFF_V + ks * 2048, 8192, 1024),
+                    umma_desc_sw128(sbase + P::OFF_I + ks * 32, 16, 1024), ID_V,
+                    ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < 16; ++ks)
+          umma_tf32_ts(tmem + P::COL_D2, tmem + P::COL_ST + 8 * ks,
+                       umma_desc_sw128(sbase + P::OFF_KQ32 + (ks >> 2) * 16384 + (ks & 3) * 32,
+                                       16, 1024),
+                       ID_2, 1u);
+        umma_commit(mma2_bar);
+        pend_mma2 = c & 1;
+      }
+      if (fail(mma2_bar, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_mma2 = -1;
+      tc_fence_after();
+      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
+
+      // ---- Z^T as bf16 hi/lo token pairs; the state decays by gamma_C
+      {
+        float z[32];
+        uint32_t hi[16], lo[16];
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 32 * ch, z);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) split_pack2(z[2 * i], z[2 * i + 1], hi[i], lo[i]);
+        tmem_st16u(tmem + tm_lane + P::COL_Z + 16 * ch, hi);
+        tmem_st16u(tmem + tm_lane + P::COL_Z + 32 + 16 * ch, lo);
+      }
+      {
+        const float gC = sc_gC[s];
+#pragma unroll
+        for (int h32 = 0; h32 < 2; ++h32) {
+          float x[32];
+          uint32_t r[32];
+          tmem_ld32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(gC * x[i]);
+          tmem_st32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, r);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      bar_group(kChainBar);
+
+      // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
+      if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
+      if (issuer && !bad) {
+        tc_fence_after();
+        for (int term = 0; term < 3; ++term)
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16_ts(tmem + P::COL_D3, tmem + P::COL_Z + (term == 1 ? 32 : 0) + 8 * ks,
+                         umma_desc_sw128(sbase + P::OFF_T + (term == 2 ? 8192 : 0) + ks * 32, 16,
+                                         1024),
+                         ID_3, (term > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(mma3_bar);
+        pend_mma3 = c & 1;
+      }
+      if (fail(mma3_bar, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_mma3 = -1;
+      tc_fence_after();
+
+      // ---- B^T = coef U^T as bf16 hi/lo pairs (token pairs packed per column)
+      {
+        float u[32];
+        tmem_ld32(tmem + tm_lane + P::COL_D3 + 32 * ch, u);
+        tmem_wait_ld();
+        const float* cf = sc_coef + 64 * s + 32 * ch;
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 cc = *reinterpret_cast<const float2*>(cf + 2 * i);
+          split_pack2(cc.x * u[2 * i], cc.y * u[2 * i + 1], hi[i], lo[i]);
+        }
+        tmem_st16u(tmem + tm_lane + P::COL_B + 16 * ch, hi);
+        tmem_st16u(tmem + tm_lane + P::COL_B + 32 + 16 * ch, lo);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      bar_group(kChainBar);
+
+      // ---- MMA4: output += U^T P^T; MMA5: state += B^T K
+      if (fail(p_ready, (uint32_t)(c & 1))) bad = true;
+      if (issuer && !bad) {
+        tc_fence_after();
+        for (int ks = 0; ks < 8; ++ks)
+          umma_tf32_ts(tmem + P::COL_D2 + 64, tmem + P::COL_D3 + 8 * ks,
+                       umma_desc_sw128(sbase + P::OFF_P + (ks >> 2) * 8192 + (ks & 3) * 32, 16,
+                                       1024),
+                       ID_4, 1u);
+        umma_commit(mma4_bar);
+        pend_mma4 = c & 1;
+        // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
+        for (int hl = 0; hl < 2; ++hl)
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_B + 32 * hl + 8 * ks,
+                         umma_desc_sw128(kq_a + ks * 2048, 16384, 1024), ID_5, 1u);
+        umma_commit(mma5_bar);
+        pend_mma5 = c & 1;
+      }
+      if (fail(mma4_bar, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_mma4 = -1;
+      tc_fence_after();
+
+      // ---- o^T of this chunk's tokens [32 ch, 32 ch + 32)
+      {
+        float x[32];
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
+        tmem_wait_ld();
+        const int nvalid = min(32, T - t0 - 32 * ch);
+        float* dst = O + (((size_t)b * T + t0 + 32 * ch) * H + h) * DV + v;
+        const size_t tstride = (size_t)H * DV;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (i < nvalid) dst[i * tstride] = x[i];
+      }
+      if (fail(mma5_bar, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_mma5 = -1;
+      if (issuer && !bad && c + 2 < nchunks) issue_kq(c + 2);  // stage s is free
+      tc_fence_before();
+      if (bar_group_or(kChainBar, bad || *sc_abort != 0.f)) {
+        bad = true;
+        break;
+      }
+    }
+    // abort path: bounded waits for this group's MMAs and copies in flight
+    if (issuer) {
+      if (pend_mma2 >= 0) (void)mbar_wait(mma2_bar, (uint32_t)pend_mma2);
+      if (pend_mma3 >= 0) (void)mbar_wait(mma3_bar, (uint32_t)pend_mma3);
+      if (pend_mma4 >= 0) (void)mbar_wait(mma4_bar, (uint32_t)pend_mma4);
+      if (pend_mma5 >= 0) (void)mbar_wait(mma5_bar, (uint32_t)pend_mma5);
+      for (int st = 0; st < 2; ++st)
+        if (pend_kq[st] >= 0) (void)mbar_wait(&full_kq[st], (uint32_t)pend_kq[st]);
+      if (pend_v >= 0) (void)mbar_wait(full_v, (uint32_t)pend_v);
+    }
+    if (!bad) {
+      tc_fence_after();
+#pragma unroll
+      for (int h32 = 0; h32 < 2; ++h32) {
+        float x[32];
+        tmem_ld32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(S_out + s_row + 32 * h32 + i) =
+              make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+      }
+    }
+  } else {
+    // ================================================================= prep
+    const int ptid = tid - kGroup;
+    const int pch = (warp - 8) >> 2;  // D1 columns [32 pch, 32 pch + 32)
+    const bool mma_issuer = (warp == 9 && lane == 0);
+    const bool qrow = m >= 64;        // D1 row: query (P) or key (A) of token tk
+    const int tk = m & 63;
+    constexpr uint32_t ID_1 = umma_idesc(128, 64, 1, 0, 0);
+    int pend_mma1 = -1;
+    bool pbad = false;
+    // per-token scalars (warp 14): loaded one chunk ahead into registers
+    float ps_a[2], ps_r[2], ps_w[2];
+    auto fetch_scalars = [&](int c) {
+      const int t0 = c * kC, valid = min(kC, T - t0);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int t = lane + 32 * i;
+        const bool in = t < valid;
+        const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+        ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
+        ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
+        ps_w[i] = in ? __ldg(Wg + tok) : 0.f;
+      }
+    };
+    auto store_scalars = [&](int c) {
+      const int st = c & 1;
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int t = lane + 32 * i;
+        sc_a[64 * st + t] = ps_a[i];
+        sc_r[64 * st + t] = ps_r[i];
+        sc_w[64 * st + t] = ps_w[i];
+      }
+    };
+    if (warp == 14) {
+      fetch_scalars(0);
+      store_scalars(0);
+    }
+    bar_group(kPrepBar);
+
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c & 1;
+      const uint32_t kq_a = sbase + P::OFF_KQ + s * P::KQ_BYTES;
+      const uint8_t* kq = smem + P::OFF_KQ + s * P::KQ_BYTES;
+      if (warp == 14 && c + 1 < nchunks) fetch_scalars(c + 1);
+      if (fail(&full_kq[s], (uint32_t)((c >> 1) & 1))) pbad = true;
+      if (mma_issuer && !pbad) {
+        // D1 = [K;Q] K^T (A: the stage's K rows then Q rows per d block)
+        tc_fence_after();
+        for (int kb = 0; kb < 2; ++kb)
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t d = umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024);
+            umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
+          }
+        umma_commit(mma1_bar);
+        pend_mma1 = c & 1;
+      }
+      if (warp == 8) {
+        // log2-decay prefix, gamma_t and gamma_C (two tokens per lane)
+        const float* a_s = sc_a + 64 * s;
+        const int ta = 2 * lane, tb = ta + 1;
+        const float l0 = __log2f(a_s[ta]), l1 = __log2f(a_s[tb]);
+        float incl = l0 + l1;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const float o = __shfl_up_sync(0xffffffffu, incl, d);
+          if (lane >= d) incl += o;
+        }
+        const float lg0 = incl - l1, lg1 = incl;
+        sc_lg[64 * s + ta] = lg0;
+        sc_lg[64 * s + tb] = lg1;
+        sc_gam[64 * s + ta] = exp2f(lg0);
+        sc_gam[64 * s + tb] = exp2f(lg1);
+        if (lane == 31) sc_gC[s] = exp2f(lg1);
+      }
+      bar_group(kPrepBar);
+
+      // ---- fp32 copies -gamma_t k_t (rows 0-63), gamma_t q_t (rows 64-127),
+      // once MMA2 of the previous chunk released the buffer; ||k_t||^2 halves
+      if (c > 0 && fail(mma2_bar, (uint32_t)((c - 1) & 1))) pbad = true;
+      {
+        const int L = ptid & 127, half = ptid >> 7;  // d in [64 half, 64 half + 64)
+        const int t = L & 63;
+        const bool isq = L >= 64;
+        const float g = sc_gam[64 * s + t];
+        const float scale = isq ? g : -g;
+        const uint8_t* src = kq + half * 16384 + (isq ? 8192 : 0);
+        uint8_t* dst0 = sKQ32 + (2 * half) * 16384;
+        float acc = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          float x[8];
+          ld_bf16x8(src, (uint32_t)t, (uint32_t)cc, x);
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            acc = fmaf(x[e], x[e], acc);
+            w[e] = rna_tf32(scale * x[e]);
+          }
+          uint8_t* dst = dst0 + (cc >> 2) * 16384;
+          const uint32_t q0 = 2u * (uint32_t)(cc & 3);
+          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)L, q0)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)L, q0 + 1)) =
+              make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        if (!isq) sc_n[64 * half + t] = acc;
+      }
+      fence_async_smem();
+      bar_group(kPrepBar);
+      if (ptid == 0) mbar_arrive(kq32_ready);
+      if (warp == 8) {
+        // Mobius scan of the variance: beta_t, the update coefficients, the carry
+        const float* w_s = sc_w + 64 * s;
+        const float* r_s = sc_r + 64 * s;
+        const float* a_s = sc_a + 64 * s;
+        const int ta = 2 * lane, tb = ta + 1;
+        const float a0 = a_s[ta], a1 = a_s[tb];
+        const float n0 = sc_n[ta] + sc_n[64 + ta], n1 = sc_n[tb] + sc_n[64 + tb];
+        const float w0 = w_s[ta], w1 = w_s[tb], r0 = r_s[ta], r1 = r_s[tb];
+        const float c0 = kappa * n0, c1 = kappa * n1;
+        const Mat2 M0 = {r0 * a0 * a0, r0 * w0, c0 * a0 * a0, fmaf(c0, w0, r0)};
+        const Mat2 M1 = {r1 * a1 * a1, r1 * w1, c1 * a1 * a1, fmaf(c1, w1, r1)};
+        Mat2 Pm = mnorm(mmul(M1, M0));
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          Mat2 o;
+          o.a = __shfl_up_sync(0xffffffffu, Pm.a, d);
+          o.b = __shfl_up_sync(0xffffffffu, Pm.b, d);
+          o.c = __shfl_up_sync(0xffffffffu, Pm.c, d);
+          o.d = __shfl_up_sync(0xffffffffu, Pm.d, d);
+          if (lane >= d) Pm = mnorm(mmul(Pm, o));
+        }
+        Mat2 ex;
+        ex.a = __shfl_up_sync(0xffffffffu, Pm.a, 1);
+        ex.b = __shfl_up_sync(0xffffffffu, Pm.b, 1);
+        ex.c = __shfl_up_sync(0xffffffffu, Pm.c, 1);
+        ex.d = __shfl_up_sync(0xffffffffu, Pm.d, 1);
+        const float carry = sc_pcar[0];
+        float p = lane == 0 ? carry
+                            : __fdividef(fmaf(ex.a, carry, ex.b), fmaf(ex.c, carry, ex.d));
+        const float pp0 = fmaf(a0 * a0, p, w0);
+        p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
+        const float pp1 = fmaf(a1 * a1, p, w1);
+        p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
+        const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
+        const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
+        const float lg0 = sc_lg[64 * s + ta], lg1 = sc_lg[64 * s + tb];
+        const float lg_last = __shfl_sync(0xffffffffu, lg1, 31);
+        sc_beta[64 * s + ta] = b0;
+        sc_beta[64 * s + tb] = b1;
+        sc_coef[64 * s + ta] = b0 * exp2f(lg_last - lg0);
+        sc_coef[64 * s + tb] = b1 * exp2f(lg_last - lg1);
+        const float pnext = __shfl_sync(0xffffffffu, p, 31);
+        __syncwarp();
+        if (lane == 0) sc_pcar[0] = pnext;
+      }
+      if (warp == 14 && c + 1 < nchunks) store_scalars(c + 1);
+      bar_group(kPrepBar);
+
+      // ---- D1 epilogue: A (key rows) into AT; P (query rows) kept
+      if (fail(mma1_bar, (uint32_t)(c & 1))) pbad = true;
+      else if (mma_issuer) pend_mma1 = -1;
+      tc_fence_after();
+      const float* lg_c = sc_lg + 64 * s;
+      const float* beta_c = sc_beta + 64 * s;
+      float preg[32];
+      {
+        float d1[32];
+        tmem_ld32(tmem + tm_lane + P::COL_D1 + 32 * pch, d1);
+        tmem_wait_ld();
+        const float lg_t = lg_c[tk];
+        const int lim = tk + (qrow ? 1 : 0);  // A: j < t; P: j <= t
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const int j0 = 32 * pch + 4 * i4;
+          const float4 lgj = *reinterpret_cast<const float4*>(lg_c + j0);
+          const float4 bj = *reinterpret_cast<const float4*>(beta_c + j0);
+          const float lj[4] = {lgj.x, lgj.y, lgj.z, lgj.w};
+          const float bv[4] = {bj.x, bj.y, bj.z, bj.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float val = exp2f(lg_t - lj[e]) * bv[e] * d1[4 * i4 + e];
+            preg[4 * i4 + e] = (j0 + e < lim) ? val : 0.f;
+          }
+        }
+      }
+      tc_fence_before();
+      if (!qrow) {
+        float* row = AT + tk * kLd + 32 * pch;
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4)
+          *reinterpret_cast<float4*>(row + 4 * i4) =
+              make_float4(preg[4 * i4], preg[4 * i4 + 1], preg[4 * i4 + 2], preg[4 * i4 + 3]);
+      }
+      bar_group(kPrepBar);
+
+      // ---- T = (I + A)^-1 into AT (for the solve) and as the bf16 hi/lo B
+      // operand [t][j] of MMA3, once MMA3 of the previous chunk released it.
+      // AT keeps A below the diagonal blocks; T's blocks below the diagonal go
+      // to the transposed places above it (T_ib[r][c] at AT[16 b + c][16 i + r]).
+      if (c > 0 && fail(mma3_bar, (uint32_t)((c - 1) & 1))) pbad = true;
+      if (ptid < 64) {
+        const int blk = ptid >> 4, cc = ptid & 15;
+        const float* Ab = AT + 16 * blk * kLd + 16 * blk;
+        float x[16], acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+          x[l] = (l == cc) ? 1.f : (l < cc ? 0.f : -acc[l]);
+#pragma unroll
+          for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kLd + l], x[l], acc[i]);
+        }
+        named_bar<kPhase1Bar, 64>();  // all A columns read
+#pragma unroll
+        for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
+      }
+      bar_group(kPrepBar);
+      {
+        const int pw = warp - 8;
+        auto Ael = [&](int i, int l, int r, int k) { return AT[(16 * i + r) * kLd + 16 * l + k]; };
+        auto Tdg = [&](int i, int r, int k) { return AT[(16 * i + r) * kLd + 16 * i + k]; };
+        auto Tlo = [&](int i, int b, int r, int k) { return AT[(16 * b + k) * kLd + 16 * i + r]; };
+        auto Tset = [&](int i, int b, int r, int k, float v0, float v1) {
+          AT[(16 * b + k) * kLd + 16 * i + r] = v0;
+          AT[(16 * b + k + 1) * kLd + 16 * i + r] = v1;
+        };
+        auto Top = [&](int i, int b, int r, int k, float v0, float v1) {
+          // T[16 i + r][16 b + k, +1] as bf16 hi/lo pairs
+          uint32_t hi, lo;
+          split_pack2(v0, v1, hi, lo);
+          const uint32_t row = (uint32_t)(16 * i + r), col = (uint32_t)(16 * b + k);
+          const uint32_t off = chunk_off(row, col >> 3) + ((col & 7u) << 1);
+          *reinterpret_cast<uint32_t*>(sT + off) = hi;
+          *reinterpret_cast<uint32_t*>(sT + 8192 + off) = lo;
+        };
+        if (pw < 2) {
+          // T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_bb inside each 32-block (b = 0, 2)
+          const int b = 2 * pw, i = b + 1;
+          float* xs = X + pw * 320;
+          float acc[3][2][4] = {};
+          warp_mm16(acc, [&](int r, int k) { return Ael(i, b, r, k); },
+                    [&](int k, int n) { return Tdg(b, k, n); }, lane);
+          warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
+            *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
+          __syncwarp();
+          float acc2[3][2][4] = {};
+          warp_mm16(acc2, [&](int r, int k) { return Tdg(i, r, k); },
+                    [&](int k, int n) { return xs[k * 20 + n]; }, lane);
+          warp_put16(acc2, -1.f, [&](int r, int k, float v0, float v1) {
+            Tset(i, b, r, k, v0, v1);
+            Top(i, b, r, k, v0, v1); }, lane);
+        } else if (pw < 6) {
+          // the diagonal blocks into the operand: lane -> row r, 8 columns
+          const int i = pw - 2, r = lane >> 1, half = lane & 1;
+          const float* src = AT + (16 * i + r) * kLd + 16 * i + 8 * half;
+          const float4 x0 = *reinterpret_cast<const float4*>(src);
+          const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
+          const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          st_split8(sT, (uint32_t)(16 * i + r), sT + 8192, (uint32_t)(16 * i + r),
+                    (uint32_t)(2 * i + half), x);
+        }
+        bar_group(kPrepBar);
+        // the 32x32 block below the diagonal: T^(10) = -T^(1) (A^(10) T^(0)),
+        // first X2 = A^(10) T^(0) by four warps, one 16x16 block each
+        const int i2 = 2 + (pw >> 1), b2 = pw & 1;
+        if (pw < 4) {
+          float acc[3][2][4] = {};
+          if (b2 == 0) {
+            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 0, r, k); },
+                      [&](int k, int n) { return Tdg(0, k, n); }, lane);
+            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                      [&](int k, int n) { return Tlo(1, 0, k, n); }, lane);
+          } else {
+            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                      [&](int k, int n) { return Tdg(1, k, n); }, lane);
+          }
+          float* xs = X + pw * 320;
+          warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
+            *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
+        }
+        bar_group(kPrepBar);
+        if (pw < 4) {
+          float acc[3][2][4] = {};
+          // X2 block (m, b2) sits in X slot 2 (m - 2) + b2
+          if (i2 == 2) {
+            warp_mm16(acc, [&](int r, int k) { return Tdg(2, r, k); },
+                      [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
+          } else {
+            warp_mm16(acc, [&](int r, int k) { return Tlo(3, 2, r, k); },
+                      [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
+            warp_mm16(acc, [&](int r, int k) { return Tdg(3, r, k); },
+                      [&](int k, int n) { return X[(2 + b2) * 320 + k * 20 + n]; }, lane);
+          }
+          warp_put16(acc, -1.f, [&](int r, int k, float v0, float v1) {
+            Top(i2, b2, r, k, v0, v1); }, lane);
+        }
+      }
+      fence_async_smem();
+      bar_group(kPrepBar);
+      if (ptid == 0) mbar_arrive(t_ready);
+
+      // ---- P as the tf32 B operand [t][j], once MMA4 of the previous chunk
+      // released the buffer
+      if (c > 0 && fail(mma4_bar, (uint32_t)((c - 1) & 1))) pbad = true;
+      if (qrow) {
+        uint8_t* dst = sP + pch * 8192;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)tk, (uint32_t)q)) =
+              make_uint4(rna_tf32(preg[4 * q]), rna_tf32(preg[4 * q + 1]),
+                         rna_tf32(preg[4 * q + 2]), rna_tf32(preg[4 * q + 3]));
+      }
+      fence_async_smem();
+      if (bar_group_or(kPrepBar, pbad || *sc_abort != 0.f)) {
+        pbad = true;
+        break;
+      }
+      if (ptid == 0) mbar_arrive(p_ready);
+    }
+    if (mma_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
+    if (ptid == 0 && !pbad) P_out[bh] = sc_pcar[0];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
 // ------------------------------------------------------------------ host
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -985,6 +1776,28 @@ kdn_status launch(const void* q, const void* k, const void* v, const float* a, c
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
+kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a,
+                     const float* w, const float* r, const float* S0, const float* p0, float* o,
+                     float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
+                     cudaStream_t s) {
+  using P = WsPlan;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, B, T, H, kDK, 64) || !make_map(&mk, k, B, T, H, kDK, 64) ||
+      !make_map(&mv, v, B, T, H, 128, 64))
+    return KDN_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(chunk_engine_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             P::ALLOC) != cudaSuccess)
+      return KDN_ERR_CUDA;
+    attr_set = true;
+  }
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
+  chunk_engine_ws_kernel<<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
+      mq, mk, mv, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa, static_cast<uint32_t*>(ws));
+  return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
+}
+
 }  // namespace
 
 bool chunk_engine_supported(kdn_dtype dt, int dk, int dv) {
@@ -1001,6 +1814,8 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                const float* p0, float* o, float* S_out, float* p_out, int B,
                                int T, int H, int dv, float kappa, void* ws, cudaStream_t s) {
   if (dv == 128) {
+    // one CTA per head reads p0 and writes p_out: no snapshot needed
+    if (!diag) return launch_ws(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s);
     return diag ? launch<true, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
                 : launch<false, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
   }

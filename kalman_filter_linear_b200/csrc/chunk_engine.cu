@@ -938,52 +938,60 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 // Warp-specialised isotropic engine (one CTA per head, d_v = 128).
 //
 // Every product runs transposed, with the value index v on the 128 TMEM lanes,
-// so that the fp32 state S'^T [v][k] itself is the A operand (tf32, read from
-// TMEM) of the product with the chunk's keys and queries, and every operand a
-// lane needs later is its own row:
-//   D2 = V^T [I;0] + S'^T [-gamma K ; gamma Q]^T    Z^T (key half), gamma (Q S')^T
-//   D3 = Z^T T^T                                    U^T (bf16 hi/lo Z and T)
-//   D2 (query half) += U^T P^T                      o^T
-//   S'^T = gamma_C S'^T + B^T K,  B = coef U        (bf16 hi/lo B, exact K)
-// The tf32 products take operands rounded to nearest (P, -gamma K, gamma Q);
-// U and S' are read as the tensor cores truncate them.  Z and T enter the
-// state path, so their product keeps three bf16 hi/lo terms.
+// so that the fp32 state S'^T [v][k] stays in TMEM, every operand a lane
+// produces is its own TMEM row (an A operand read from TMEM), and the keys and
+// queries are B operands straight from the copies' tiles:
+//   D2 = S'^T [K ; Q]^T                       (S' as bf16 hi/lo, exact K and Q)
+//   Z = V - gamma K S',  gamma (Q S')          Z as bf16 hi/lo
+//   D3 = Z^T T^T                              U^T (bf16 hi/lo Z and T, three terms)
+//   D2 (query half) += U^T P^T                o^T (tf32: U as the tensor cores
+//                                             truncate it, P rounded)
+//   S'^T = gamma_C S'^T + B^T K,  B = coef U  (bf16 hi/lo B, exact K)
 //
-// Warps 0-7 (the chain) run the part that depends on the state, with three
-// small TMEM passes per chunk: Z in bf16 hi/lo plus the state decay, B = coef U
-// in bf16 hi/lo, and the output copy.  Warps 8-15 (prep) run the part that depends
-// only on the chunk's inputs, one chunk ahead: the decay prefix, the fp32
-// key/query copies, the variance scan, MMA1, A and P, and T = (I + A)^-1.
-// The groups hand buffers over through mbarriers:
-//   kq32_ready / t_ready / p_ready   prep -> chain (with the chunk's scalars)
-//   mma2 / mma3 / mma4               the chain's commits; they also hand the
-//                                    fp32 key/query copy, T and P back to prep
-// A K/Q stage is refilled (chunk c + 2) once MMA5 of chunk c has finished.
+// Warps 0-7 (the chain) run the part that depends on the state.  Per chunk:
+// MMA2; Z (with gamma_t (Q S')_t and the state decay); MMA3; B = coef U; MMA5
+// and MMA4; the state's bf16 hi/lo operand for the next chunk and the output
+// copy.  Warps 8-15 (prep) run the
+// part that depends only on the chunk's inputs, one chunk ahead: the D1
+// epilogue (A and P) on all eight warps, then T = (I + A)^-1 on warps 8-11
+// while warps 12-15 prepare the next chunk's ||k||^2, decay prefix and
+// variance scan.  MMA1 of the next chunk is issued as soon as D1 is read.
+// The groups hand over through mbarriers:
+//   t_ready / p_ready   prep -> chain: T / P written, with the chunk's scalars
+//                       and the next chunk's decay
+//   mma3 / mma4         the chain's commits; they also hand T and P back
+// Per-token scalars live in four slots (chunk index mod 4).
 // TMEM columns: D1 [0,64) (prep); S'^T [64,192); D2 [192,320) (key half, then
-// query half); D3 [320,384); B^T hi [384,416), lo [416,448); Z^T hi [448,480),
-// lo [480,512).
+// query half); D3 [320,384); W [384,512) holds in turn S'^T hi [384,448) and lo
+// [448,512) (k pairs), Z^T hi [384,416) and lo [416,448), B^T hi and lo (same).
 // ===========================================================================
 struct WsPlan {
   static constexpr uint32_t KQ_BYTES = 32768;           // bf16 [kb 2][K|Q][64 t][64]
-  static constexpr uint32_t OFF_KQ = 0;                 // two stages
-  static constexpr uint32_t OFF_KQ32 = 2 * KQ_BYTES;    // fp32 [kb 4][128 L][32]
-  static constexpr uint32_t OFF_V = OFF_KQ32 + 65536;   // bf16 [vb 2][64 t][64 v]
-  static constexpr uint32_t OFF_I = OFF_V + 16384;      // bf16 [128 L][64 u]: I over 0
-  static constexpr uint32_t OFF_T = OFF_I + 16384;      // bf16 hi, lo [64 t][64 j]
+  static constexpr int kStages = 3;
+  static constexpr uint32_t OFF_KQ = 0;                 // kStages stages
+  static constexpr uint32_t OFF_V = kStages * KQ_BYTES; // bf16 [vb 2][64 t][64 v]
+  static constexpr uint32_t OFF_T = OFF_V + 16384;      // bf16 hi, lo [64 t][64 j]
   static constexpr uint32_t OFF_P = OFF_T + 16384;      // fp32 [jb 2][64 t][32 j]
   static constexpr uint32_t OFF_AT = OFF_P + 16384;     // fp32 [64][68]
   static constexpr uint32_t OFF_X = OFF_AT + 64u * kLd * 4u;
   static constexpr uint32_t OFF_SC = OFF_X + 5120u;     // X: fp32 [4][16][20]
-  static constexpr uint32_t OFF_BAR = OFF_SC + 6144u;
+  static constexpr uint32_t OFF_OUT = OFF_SC + 9216u;   // fp32 [64 t][128 v] output tile
+  static constexpr uint32_t OFF_BAR = OFF_OUT + 32768u;
   static constexpr uint32_t TOTAL = OFF_BAR + 256u;
   static constexpr uint32_t ALLOC = TOTAL + 1024u;
-  static constexpr uint32_t COL_D1 = 0, COL_ST = 64, COL_D2 = 192, COL_D3 = 320, COL_B = 384,
-                            COL_Z = 448;
+  static constexpr uint32_t COL_D1 = 0, COL_ST = 64, COL_D2 = 192, COL_D3 = 320, COL_W = 384;
   static_assert(TOTAL <= 227u * 1024u, "shared memory plan too large");
-  static_assert(OFF_KQ32 % 1024 == 0 && OFF_V % 1024 == 0 && OFF_I % 1024 == 0 &&
-                    OFF_T % 1024 == 0 && OFF_P % 1024 == 0,
+  static_assert(OFF_V % 1024 == 0 && OFF_T % 1024 == 0 && OFF_P % 1024 == 0 &&
+                    OFF_OUT % 128 == 0,
                 "operand alignment");
 };
+
+// 2^x from the hardware approximation (relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 // (hi, lo) bf16 splits of two consecutive K elements, packed low-first as a
 // 32-bit TMEM column of a bf16 A operand.
@@ -1071,10 +1079,13 @@ __device__ __forceinline__ bool bar_group_or(int id, bool flag) {
   return r != 0;
 }
 
+constexpr int kTeamA = 6, kTeamB = 7;
+
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ Ag,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ Ag,
                        const float* __restrict__ Wg, const float* __restrict__ Rg,
                        const float* S0, const float* __restrict__ P0, float* __restrict__ O,
                        float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
@@ -1090,37 +1101,35 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   const int nchunks = (T + kC - 1) / kC;
   const uint32_t sbase = smem_u32(smem);
 
-  // scalar area (floats); [2][64] arrays are indexed by chunk parity
+  // scalar area (floats); [4][64] arrays are indexed by chunk & 3
   float* scf = reinterpret_cast<float*>(smem + P::OFF_SC);
-  float* sc_a = scf;            // decay a_t
-  float* sc_w = scf + 128;      // process noise w_t
-  float* sc_r = scf + 256;      // observation noise r_t
-  float* sc_n = scf + 384;      // [2 halves][64] partial ||k_t||^2
-  float* sc_beta = scf + 512;   // beta_t
-  float* sc_lg = scf + 640;     // log2 of the in-chunk cumulative decay
-  float* sc_gam = scf + 768;    // gamma_t
-  float* sc_coef = scf + 896;   // state-update coefficient
-  float* sc_gC = scf + 1024;    // [2] gamma of the whole chunk
-  float* sc_pcar = scf + 1026;  // carried variance
-  volatile float* sc_abort = scf + 1027;
+  float* sc_a = scf;             // decay a_t
+  float* sc_w = scf + 256;       // process noise w_t
+  float* sc_r = scf + 512;       // observation noise r_t
+  float* sc_beta = scf + 768;    // beta_t
+  float* sc_lg = scf + 1024;     // log2 of the in-chunk cumulative decay
+  float* sc_gam = scf + 1280;    // gamma_t
+  float* sc_coef = scf + 1536;   // state-update coefficient
+  float* sc_n = scf + 1792;      // [2 halves][64] partial ||k_t||^2 of one chunk
+  float* sc_gC = scf + 1920;     // [4] gamma of the whole chunk
+  float* sc_pcar = scf + 1924;   // carried variance
+  volatile float* sc_abort = scf + 1925;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
-  uint64_t* full_kq = bars;         // [2] K/Q tiles of a stage landed
-  uint64_t* full_v = bars + 2;      // V tile landed
-  uint64_t* mma1_bar = bars + 3;    // MMA1 finished (D1)
-  uint64_t* mma2_bar = bars + 4;    // MMA2 finished: fp32 K/Q copy and V free
-  uint64_t* mma3_bar = bars + 5;    // MMA3 finished: T free
-  uint64_t* mma4_bar = bars + 6;    // MMA4 finished: P free, output ready
-  uint64_t* mma5_bar = bars + 7;    // MMA5 finished: state updated, stage free
-  uint64_t* kq32_ready = bars + 8;  // fp32 K/Q copy and decay scalars written
-  uint64_t* t_ready = bars + 9;     // T and the update coefficients written
-  uint64_t* p_ready = bars + 10;    // P written
+  uint64_t* full_kq = bars;        // [kStages] K/Q tiles of a stage landed
+  uint64_t* full_v = bars + 3;     // V tile landed
+  uint64_t* mma1_bar = bars + 4;   // MMA1 finished (D1)
+  uint64_t* mma2_bar = bars + 5;   // MMA2 finished
+  uint64_t* mma3_bar = bars + 6;   // MMA3 finished: T free
+  uint64_t* mma4_bar = bars + 7;   // MMA4 finished: P free, output ready
+  uint64_t* mma5_bar = bars + 8;   // MMA5 finished: state updated, stage free
+  uint64_t* t_ready = bars + 9;    // T written
+  uint64_t* p_ready = bars + 10;   // P and the next chunk's scalars written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  float* sOut = reinterpret_cast<float*>(smem + P::OFF_OUT);
   float* AT = reinterpret_cast<float*>(smem + P::OFF_AT);
   float* X = reinterpret_cast<float*>(smem + P::OFF_X);
-  uint8_t* sKQ32 = smem + P::OFF_KQ32;
   uint8_t* sT = smem + P::OFF_T;
   uint8_t* sP = smem + P::OFF_P;
-  uint8_t* sI = smem + P::OFF_I;
   uint8_t* sV = smem + P::OFF_V;
 
   if (tid == 0) {
@@ -1129,16 +1138,9 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     *sc_abort = 0.f;
     sc_pcar[0] = P0 ? P0[bh] : 1.f;
   }
-  // [I; 0]: bf16 K-major rows L of 64 u, 1.0 at u = L for L < 64
-  for (int i = tid; i < 1024; i += kThreads) {
-    const int L = i >> 3, q = i & 7;
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (L < 64 && (L >> 3) == q) w[(L & 7) >> 1] = 0x3F80u << (16 * (L & 1));
-    *reinterpret_cast<uint4*>(sI + chunk_off((uint32_t)L, (uint32_t)q)) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-    // T operand (hi, lo): blocks above the diagonal are never written again
+  // T operand (hi, lo): blocks above the diagonal are never written again
+  for (int i = tid; i < 1024; i += kThreads)
     *reinterpret_cast<uint4*>(sT + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
-  }
   fence_async_smem();
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -1151,7 +1153,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   // Bounded wait; once any thread has recorded a timeout every later wait
   // fails at once, so an aborting CTA ends within a few wait limits.
-  auto fail1 = [&](uint64_t* bar_, uint32_t parity) -> bool {
+  auto fail = [&](uint64_t* bar_, uint32_t parity) -> bool {
     if (*sc_abort != 0.f) return true;
     if (!mbar_wait(bar_, parity)) {
       atomicOr(err, DEV_TIMEOUT);
@@ -1160,47 +1162,195 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     return false;
   };
-  auto fail = fail1;
 
   const int m = 32 * (warp & 3) + lane;  // TMEM lane of this thread
   const uint32_t tm_lane = (uint32_t)(32 * (warp & 3)) << 16;
+
+  // ---- the prep group's per-chunk scalars
+  // a, w, r of chunk c (one warp): loaded a chunk ahead into registers
+  float ps_a[2], ps_r[2], ps_w[2];
+  auto fetch_scalars = [&](int c) {
+    const int t0 = c * kC, valid = min(kC, T - t0);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int t = lane + 32 * i;
+      const bool in = t < valid;
+      const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+      ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
+      ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
+      ps_w[i] = in ? __ldg(Wg + tok) : 0.f;
+    }
+  };
+  auto store_scalars = [&](int c) {
+    const int sl = c & 3;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int t = lane + 32 * i;
+      sc_a[64 * sl + t] = ps_a[i];
+      sc_r[64 * sl + t] = ps_r[i];
+      sc_w[64 * sl + t] = ps_w[i];
+    }
+  };
+  // partial ||k_t||^2 of chunk c over d in [64 half, 64 half + 64), 128 threads
+  auto key_norms = [&](int c, int pt) {
+    const int t = pt & 63, half = pt >> 6;
+    const uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + half * 16384;
+    float acc = 0.f;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+      float x[8];
+      ld_bf16x8(kt, (uint32_t)t, (uint32_t)cc, x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(x[e], x[e], acc);
+    }
+    sc_n[64 * half + t] = acc;
+  };
+  // decay prefix and Mobius scan of the variance of chunk c (one warp, two
+  // tokens per lane): lg, gamma, gamma_C, beta, the update coefficients, carry
+  auto decay_and_variance = [&](int c) {
+    const int sl = c & 3;
+    const float* a_s = sc_a + 64 * sl;
+    const float* w_s = sc_w + 64 * sl;
+    const float* r_s = sc_r + 64 * sl;
+    const int ta = 2 * lane, tb = ta + 1;
+    const float a0 = a_s[ta], a1 = a_s[tb];
+    const float l0 = __log2f(a0), l1 = __log2f(a1);
+    float incl = l0 + l1;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const float o = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += o;
+    }
+    const float lg0 = incl - l1, lg1 = incl;
+    const float lg_last = __shfl_sync(0xffffffffu, lg1, 31);
+    sc_lg[64 * sl + ta] = lg0;
+    sc_lg[64 * sl + tb] = lg1;
+    sc_gam[64 * sl + ta] = exp2f(lg0);
+    sc_gam[64 * sl + tb] = exp2f(lg1);
+    if (lane == 31) sc_gC[sl] = exp2f(lg1);
+    const float n0 = sc_n[ta] + sc_n[64 + ta], n1 = sc_n[tb] + sc_n[64 + tb];
+    const float w0 = w_s[ta], w1 = w_s[tb], r0 = r_s[ta], r1 = r_s[tb];
+    const float c0 = kappa * n0, c1 = kappa * n1;
+    const Mat2 M0 = {r0 * a0 * a0, r0 * w0, c0 * a0 * a0, fmaf(c0, w0, r0)};
+    const Mat2 M1 = {r1 * a1 * a1, r1 * w1, c1 * a1 * a1, fmaf(c1, w1, r1)};
+    Mat2 Pm = mnorm(mmul(M1, M0));
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      Mat2 o;
+      o.a = __shfl_up_sync(0xffffffffu, Pm.a, d);
+      o.b = __shfl_up_sync(0xffffffffu, Pm.b, d);
+      o.c = __shfl_up_sync(0xffffffffu, Pm.c, d);
+      o.d = __shfl_up_sync(0xffffffffu, Pm.d, d);
+      if (lane >= d) Pm = mnorm(mmul(Pm, o));
+    }
+    Mat2 ex;
+    ex.a = __shfl_up_sync(0xffffffffu, Pm.a, 1);
+    ex.b = __shfl_up_sync(0xffffffffu, Pm.b, 1);
+    ex.c = __shfl_up_sync(0xffffffffu, Pm.c, 1);
+    ex.d = __shfl_up_sync(0xffffffffu, Pm.d, 1);
+    const float carry = sc_pcar[0];
+    float p = lane == 0 ? carry : __fdividef(fmaf(ex.a, carry, ex.b), fmaf(ex.c, carry, ex.d));
+    const float pp0 = fmaf(a0 * a0, p, w0);
+    p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
+    const float pp1 = fmaf(a1 * a1, p, w1);
+    p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
+    const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
+    const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
+    sc_beta[64 * sl + ta] = b0;
+    sc_beta[64 * sl + tb] = b1;
+    sc_coef[64 * sl + ta] = b0 * exp2f(lg_last - lg0);
+    sc_coef[64 * sl + tb] = b1 * exp2f(lg_last - lg1);
+    const float pnext = __shfl_sync(0xffffffffu, p, 31);
+    __syncwarp();
+    if (lane == 0) sc_pcar[0] = pnext;
+  };
+
+  const bool issuer = (warp == 0 && lane == 0);       // chain: MMAs and copies
+  const bool mma1_issuer = (warp == 15 && lane == 0);  // prep: MMA1
+  constexpr uint32_t ID_1 = umma_idesc(128, 64, 1, 0, 0);
+  int pend_kq[P::kStages] = {-1, -1, -1}, pend_v = -1, pend_mma1 = -1;  // (issuers) not yet seen done
+  auto kq_parity = [](int c) { return (uint32_t)((c / P::kStages) & 1); };
+  auto issue_kq = [&](int c) {
+    const int st = c % P::kStages, t0 = c * kC;
+    uint8_t* kqd = smem + P::OFF_KQ + st * P::KQ_BYTES;
+    mbar_expect_tx(&full_kq[st], P::KQ_BYTES);
+    for (int kb = 0; kb < 2; ++kb) {
+      tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, t0, b);
+      tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, t0, b);
+    }
+    pend_kq[st] = (int)kq_parity(c);
+  };
+  auto issue_v = [&](int c) {
+    mbar_expect_tx(full_v, 16384);
+    tma_load_4d(sV, &tm_v, full_v, 0, h, c * kC, b);
+    tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
+    pend_v = c & 1;
+  };
+  // D1 = [K;Q] K^T of chunk c (A: the stage's key rows then query rows per d block)
+  auto issue_mma1 = [&](int c) {
+    const uint32_t kq_a = sbase + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES;
+    tc_fence_after();
+    for (int kb = 0; kb < 2; ++kb)
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t d = umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024);
+        umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
+      }
+    umma_commit(mma1_bar);
+    pend_mma1 = c & 1;
+  };
+
+  // ---- prologue: copies, chunk 0's scalars and MMA1
+  bool bad = false;
+  if (issuer) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+    issue_kq(0);
+    issue_v(0);
+    for (int c = 1; c < P::kStages && c < nchunks; ++c) issue_kq(c);
+  }
+  if (warp >= 8) {
+    if (warp == 13) {
+      fetch_scalars(0);
+      store_scalars(0);
+      if (nchunks > 1) fetch_scalars(1);
+    }
+    if (fail(&full_kq[0], kq_parity(0))) bad = true;
+    if (mma1_issuer && !bad) issue_mma1(0);
+    if (warp >= 12) {
+      key_norms(0, tid - 384);
+      named_bar<kTeamB, 128>();
+      if (warp == 12) decay_and_variance(0);
+    }
+  }
+  __syncthreads();  // chunk 0's scalars are in place
 
   if (warp < 8) {
     // ================================================================ chain
     const int ch = warp >> 2;  // tokens [32 ch, 32 ch + 32), state columns [64 ch, 64 ch + 64)
     const int v = m;           // value index of this lane
-    const bool issuer = (warp == 0 && lane == 0);
-    constexpr uint32_t ID_V = umma_idesc(128, 128, 1, 1, 0);   // bf16, A MN-major
-    constexpr uint32_t ID_2 = umma_idesc(128, 128, 2, 0, 0);   // tf32
+    constexpr uint32_t ID_2 = umma_idesc(128, 128, 1, 0, 0);   // bf16
     constexpr uint32_t ID_3 = umma_idesc(128, 64, 1, 0, 0);    // bf16
     constexpr uint32_t ID_4 = umma_idesc(128, 64, 2, 0, 0);    // tf32
     constexpr uint32_t ID_5 = umma_idesc(128, 128, 1, 0, 1);   // bf16, B MN-major
 
-    int pend_kq[2] = {-1, -1}, pend_v = -1;  // copies not yet seen landed (issuer)
-    auto issue_kq = [&](int c) {
-      const int st = c & 1, t0 = c * kC;
-      uint8_t* kqd = smem + P::OFF_KQ + st * P::KQ_BYTES;
-      mbar_expect_tx(&full_kq[st], P::KQ_BYTES);
-      for (int kb = 0; kb < 2; ++kb) {
-        tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, t0, b);
-        tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, t0, b);
+    // S'^T [v][k], k in [64 ch, 64 ch + 64), as the bf16 hi/lo A operand of
+    // MMA2 in W: k pairs per column, hi then lo
+    auto split_state = [&]() {
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int h32 = 0; h32 < 2; ++h32) {
+        float x[32];
+        tmem_ld32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          split_pack2(x[2 * i], x[2 * i + 1], hi[16 * h32 + i], lo[16 * h32 + i]);
       }
-      pend_kq[st] = (c >> 1) & 1;
+      tmem_st32(tmem + tm_lane + P::COL_W + 32 * ch, hi);
+      tmem_st32(tmem + tm_lane + P::COL_W + 64 + 32 * ch, lo);
     };
-    auto issue_v = [&](int c) {
-      mbar_expect_tx(full_v, 16384);
-      tma_load_4d(sV, &tm_v, full_v, 0, h, c * kC, b);
-      tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
-      pend_v = c & 1;
-    };
-    if (issuer) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      issue_kq(0);
-      issue_v(0);
-      if (nchunks > 1) issue_kq(1);
-    }
 
     // S'^T [v][k] into TMEM, k in [64 ch, 64 ch + 64)
     const size_t s_row = ((size_t)bh * DV + v) * kDK + 64 * ch;
@@ -1219,55 +1369,67 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_st32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, r);
     }
     tmem_wait_st();
+    split_state();
+    tmem_wait_st();
     tc_fence_before();
     bar_group(kChainBar);
 
     int pend_mma2 = -1, pend_mma3 = -1, pend_mma4 = -1, pend_mma5 = -1;
-    bool bad = false;
     for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1;
+      const int s = c % P::kStages, sl = c & 3;
       const int t0 = c * kC;
       const uint32_t kq_a = sbase + P::OFF_KQ + s * P::KQ_BYTES;
-      if (fail(kq32_ready, (uint32_t)(c & 1))) bad = true;
-      if (fail(full_v, (uint32_t)(c & 1))) bad = true;
-      else if (issuer) pend_v = -1;
+      // ---- MMA2: D2 = S'^T [K; Q]^T (S' hi, then lo; B: the stage's key rows
+      // then query rows per d block, K-major)
       if (issuer) {
-        if (fail1(&full_kq[s], (uint32_t)((c >> 1) & 1))) bad = true;
+        if (fail(&full_kq[s], kq_parity(c))) bad = true;
         else pend_kq[s] = -1;
       }
-      // ---- MMA2: D2 = V^T [I;0] + S'^T [-gamma K; gamma Q]^T
       if (issuer && !bad) {
         tc_fence_after();
-        for (int ks = 0; ks < 4; ++ks)
-          umma_bf16(tmem + P::COL_D2, umma_desc_sw128(sbase + P::OFF_V + ks * 2048, 8192, 1024),
-                    umma_desc_sw128(sbase + P::OFF_I + ks * 32, 16, 1024), ID_V,
-                    ks > 0 ? 1u : 0u);
-        for (int ks = 0; ks < 16; ++ks)
-          umma_tf32_ts(tmem + P::COL_D2, tmem + P::COL_ST + 8 * ks,
-                       umma_desc_sw128(sbase + P::OFF_KQ32 + (ks >> 2) * 16384 + (ks & 3) * 32,
-                                       16, 1024),
-                       ID_2, 1u);
+        for (int hl = 0; hl < 2; ++hl)
+          for (int kb = 0; kb < 2; ++kb)
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16_ts(tmem + P::COL_D2, tmem + P::COL_W + 64 * hl + 32 * kb + 8 * ks,
+                           umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024), ID_2,
+                           (hl > 0 || kb > 0 || ks > 0) ? 1u : 0u);
         umma_commit(mma2_bar);
         pend_mma2 = c & 1;
       }
+      if (fail(full_v, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_v = -1;
       if (fail(mma2_bar, (uint32_t)(c & 1))) bad = true;
       else if (issuer) pend_mma2 = -1;
       tc_fence_after();
-      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
 
-      // ---- Z^T as bf16 hi/lo token pairs; the state decays by gamma_C
+      // ---- Z^T = V^T - gamma (K S')^T as bf16 hi/lo token pairs (in W, which
+      // MMA2 has read); gamma (Q S')^T in place; the state decays by gamma_C
       {
-        float z[32];
+        float z[32], qs[32];
         uint32_t hi[16], lo[16];
         tmem_ld32(tmem + tm_lane + P::COL_D2 + 32 * ch, z);
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qs);
         tmem_wait_ld();
+        const uint8_t* vt = sV + (v >> 6) * 8192;
+        const float* gm = sc_gam + 64 * sl + 32 * ch;
+        uint32_t qr[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const uint16_t vb =
+              *reinterpret_cast<const uint16_t*>(vt + sw128_offset((uint32_t)(32 * ch + i),
+                                                                   (uint32_t)(v & 63)));
+          const float g = gm[i];
+          z[i] = fmaf(-g, z[i], __uint_as_float((uint32_t)vb << 16));
+          qr[i] = __float_as_uint(g * qs[i]);
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) split_pack2(z[2 * i], z[2 * i + 1], hi[i], lo[i]);
-        tmem_st16u(tmem + tm_lane + P::COL_Z + 16 * ch, hi);
-        tmem_st16u(tmem + tm_lane + P::COL_Z + 32 + 16 * ch, lo);
+        tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);
+        tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);
+        tmem_st32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qr);
       }
       {
-        const float gC = sc_gC[s];
+        const float gC = sc_gC[sl];
 #pragma unroll
         for (int h32 = 0; h32 < 2; ++h32) {
           float x[32];
@@ -1282,6 +1444,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_st();
       tc_fence_before();
       bar_group(kChainBar);
+      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
 
       // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
       if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
@@ -1289,7 +1452,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         for (int term = 0; term < 3; ++term)
           for (int ks = 0; ks < 4; ++ks)
-            umma_bf16_ts(tmem + P::COL_D3, tmem + P::COL_Z + (term == 1 ? 32 : 0) + 8 * ks,
+            umma_bf16_ts(tmem + P::COL_D3, tmem + P::COL_W + (term == 1 ? 32 : 0) + 8 * ks,
                          umma_desc_sw128(sbase + P::OFF_T + (term == 2 ? 8192 : 0) + ks * 32, 16,
                                          1024),
                          ID_3, (term > 0 || ks > 0) ? 1u : 0u);
@@ -1300,29 +1463,37 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       else if (issuer) pend_mma3 = -1;
       tc_fence_after();
 
-      // ---- B^T = coef U^T as bf16 hi/lo pairs (token pairs packed per column)
+      // ---- B^T = coef U^T as bf16 hi/lo token pairs
       {
         float u[32];
         tmem_ld32(tmem + tm_lane + P::COL_D3 + 32 * ch, u);
         tmem_wait_ld();
-        const float* cf = sc_coef + 64 * s + 32 * ch;
+        const float* cf = sc_coef + 64 * sl + 32 * ch;
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 cc = *reinterpret_cast<const float2*>(cf + 2 * i);
           split_pack2(cc.x * u[2 * i], cc.y * u[2 * i + 1], hi[i], lo[i]);
         }
-        tmem_st16u(tmem + tm_lane + P::COL_B + 16 * ch, hi);
-        tmem_st16u(tmem + tm_lane + P::COL_B + 32 + 16 * ch, lo);
+        tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);  // Z has been read
+        tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);
       }
+      if (issuer) bulk_wait_read_all();  // the previous output tile has been read
       tmem_wait_st();
       tc_fence_before();
       bar_group(kChainBar);
 
-      // ---- MMA4: output += U^T P^T; MMA5: state += B^T K
+      // ---- MMA5: state += B^T K; MMA4: output += U^T P^T
       if (fail(p_ready, (uint32_t)(c & 1))) bad = true;
       if (issuer && !bad) {
         tc_fence_after();
+        // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
+        for (int hl = 0; hl < 2; ++hl)
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_W + 32 * hl + 8 * ks,
+                         umma_desc_sw128(kq_a + ks * 2048, 16384, 1024), ID_5, 1u);
+        umma_commit(mma5_bar);
+        pend_mma5 = c & 1;
         for (int ks = 0; ks < 8; ++ks)
           umma_tf32_ts(tmem + P::COL_D2 + 64, tmem + P::COL_D3 + 8 * ks,
                        umma_desc_sw128(sbase + P::OFF_P + (ks >> 2) * 8192 + (ks & 3) * 32, 16,
@@ -1330,37 +1501,37 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        ID_4, 1u);
         umma_commit(mma4_bar);
         pend_mma4 = c & 1;
-        // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
-        for (int hl = 0; hl < 2; ++hl)
-          for (int ks = 0; ks < 4; ++ks)
-            umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_B + 32 * hl + 8 * ks,
-                         umma_desc_sw128(kq_a + ks * 2048, 16384, 1024), ID_5, 1u);
-        umma_commit(mma5_bar);
-        pend_mma5 = c & 1;
       }
+      // ---- the state's operand for the next chunk (MMA5 has read B)
+      if (fail(mma5_bar, (uint32_t)(c & 1))) bad = true;
+      else if (issuer) pend_mma5 = -1;
+      tc_fence_after();
+      if (c + 1 < nchunks) split_state();
+      // ---- o^T of this chunk's tokens [32 ch, 32 ch + 32)
       if (fail(mma4_bar, (uint32_t)(c & 1))) bad = true;
       else if (issuer) pend_mma4 = -1;
       tc_fence_after();
-
-      // ---- o^T of this chunk's tokens [32 ch, 32 ch + 32)
+      // (into the staging tile [t][v]; one bulk tensor store per chunk writes
+      // it, rows past T excluded)
       {
         float x[32];
         tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
         tmem_wait_ld();
-        const int nvalid = min(32, T - t0 - 32 * ch);
-        float* dst = O + (((size_t)b * T + t0 + 32 * ch) * H + h) * DV + v;
-        const size_t tstride = (size_t)H * DV;
+        float* dst = sOut + (32 * ch) * DV + v;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (i < nvalid) dst[i * tstride] = x[i];
+        for (int i = 0; i < 32; ++i) dst[i * DV] = x[i];
       }
-      if (fail(mma5_bar, (uint32_t)(c & 1))) bad = true;
-      else if (issuer) pend_mma5 = -1;
-      if (issuer && !bad && c + 2 < nchunks) issue_kq(c + 2);  // stage s is free
+      fence_async_smem();
+      if (issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);  // stage s is free
+      tmem_wait_st();
       tc_fence_before();
       if (bar_group_or(kChainBar, bad || *sc_abort != 0.f)) {
         bad = true;
         break;
+      }
+      if (issuer) {
+        tma_store_4d(&tm_o, sOut, 0, h, t0, b);
+        bulk_commit();
       }
     }
     // abort path: bounded waits for this group's MMAs and copies in flight
@@ -1369,9 +1540,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (pend_mma3 >= 0) (void)mbar_wait(mma3_bar, (uint32_t)pend_mma3);
       if (pend_mma4 >= 0) (void)mbar_wait(mma4_bar, (uint32_t)pend_mma4);
       if (pend_mma5 >= 0) (void)mbar_wait(mma5_bar, (uint32_t)pend_mma5);
-      for (int st = 0; st < 2; ++st)
+      for (int st = 0; st < P::kStages; ++st)
         if (pend_kq[st] >= 0) (void)mbar_wait(&full_kq[st], (uint32_t)pend_kq[st]);
       if (pend_v >= 0) (void)mbar_wait(full_v, (uint32_t)pend_v);
+      bulk_wait_all();  // output stores complete
     }
     if (!bad) {
       tc_fence_after();
@@ -1389,169 +1561,18 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else {
     // ================================================================= prep
     const int ptid = tid - kGroup;
-    const int pch = (warp - 8) >> 2;  // D1 columns [32 pch, 32 pch + 32)
-    const bool mma_issuer = (warp == 9 && lane == 0);
+    const int pw = warp - 8;
+    const int pch = pw >> 2;          // D1 columns [32 pch, 32 pch + 32)
     const bool qrow = m >= 64;        // D1 row: query (P) or key (A) of token tk
     const int tk = m & 63;
-    constexpr uint32_t ID_1 = umma_idesc(128, 64, 1, 0, 0);
-    int pend_mma1 = -1;
-    bool pbad = false;
-    // per-token scalars (warp 14): loaded one chunk ahead into registers
-    float ps_a[2], ps_r[2], ps_w[2];
-    auto fetch_scalars = [&](int c) {
-      const int t0 = c * kC, valid = min(kC, T - t0);
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int t = lane + 32 * i;
-        const bool in = t < valid;
-        const size_t tok = ((size_t)b * T + t0 + t) * H + h;
-        ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
-        ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
-        ps_w[i] = in ? __ldg(Wg + tok) : 0.f;
-      }
-    };
-    auto store_scalars = [&](int c) {
-      const int st = c & 1;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int t = lane + 32 * i;
-        sc_a[64 * st + t] = ps_a[i];
-        sc_r[64 * st + t] = ps_r[i];
-        sc_w[64 * st + t] = ps_w[i];
-      }
-    };
-    if (warp == 14) {
-      fetch_scalars(0);
-      store_scalars(0);
-    }
-    bar_group(kPrepBar);
-
     for (int c = 0; c < nchunks; ++c) {
-      const int s = c & 1;
-      const uint32_t kq_a = sbase + P::OFF_KQ + s * P::KQ_BYTES;
-      const uint8_t* kq = smem + P::OFF_KQ + s * P::KQ_BYTES;
-      if (warp == 14 && c + 1 < nchunks) fetch_scalars(c + 1);
-      if (fail(&full_kq[s], (uint32_t)((c >> 1) & 1))) pbad = true;
-      if (mma_issuer && !pbad) {
-        // D1 = [K;Q] K^T (A: the stage's K rows then Q rows per d block)
-        tc_fence_after();
-        for (int kb = 0; kb < 2; ++kb)
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t d = umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024);
-            umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
-          }
-        umma_commit(mma1_bar);
-        pend_mma1 = c & 1;
-      }
-      if (warp == 8) {
-        // log2-decay prefix, gamma_t and gamma_C (two tokens per lane)
-        const float* a_s = sc_a + 64 * s;
-        const int ta = 2 * lane, tb = ta + 1;
-        const float l0 = __log2f(a_s[ta]), l1 = __log2f(a_s[tb]);
-        float incl = l0 + l1;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          const float o = __shfl_up_sync(0xffffffffu, incl, d);
-          if (lane >= d) incl += o;
-        }
-        const float lg0 = incl - l1, lg1 = incl;
-        sc_lg[64 * s + ta] = lg0;
-        sc_lg[64 * s + tb] = lg1;
-        sc_gam[64 * s + ta] = exp2f(lg0);
-        sc_gam[64 * s + tb] = exp2f(lg1);
-        if (lane == 31) sc_gC[s] = exp2f(lg1);
-      }
-      bar_group(kPrepBar);
-
-      // ---- fp32 copies -gamma_t k_t (rows 0-63), gamma_t q_t (rows 64-127),
-      // once MMA2 of the previous chunk released the buffer; ||k_t||^2 halves
-      if (c > 0 && fail(mma2_bar, (uint32_t)((c - 1) & 1))) pbad = true;
-      {
-        const int L = ptid & 127, half = ptid >> 7;  // d in [64 half, 64 half + 64)
-        const int t = L & 63;
-        const bool isq = L >= 64;
-        const float g = sc_gam[64 * s + t];
-        const float scale = isq ? g : -g;
-        const uint8_t* src = kq + half * 16384 + (isq ? 8192 : 0);
-        uint8_t* dst0 = sKQ32 + (2 * half) * 16384;
-        float acc = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float x[8];
-          ld_bf16x8(src, (uint32_t)t, (uint32_t)cc, x);
-          uint32_t w[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            acc = fmaf(x[e], x[e], acc);
-            w[e] = rna_tf32(scale * x[e]);
-          }
-          uint8_t* dst = dst0 + (cc >> 2) * 16384;
-          const uint32_t q0 = 2u * (uint32_t)(cc & 3);
-          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)L, q0)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)L, q0 + 1)) =
-              make_uint4(w[4], w[5], w[6], w[7]);
-        }
-        if (!isq) sc_n[64 * half + t] = acc;
-      }
-      fence_async_smem();
-      bar_group(kPrepBar);
-      if (ptid == 0) mbar_arrive(kq32_ready);
-      if (warp == 8) {
-        // Mobius scan of the variance: beta_t, the update coefficients, the carry
-        const float* w_s = sc_w + 64 * s;
-        const float* r_s = sc_r + 64 * s;
-        const float* a_s = sc_a + 64 * s;
-        const int ta = 2 * lane, tb = ta + 1;
-        const float a0 = a_s[ta], a1 = a_s[tb];
-        const float n0 = sc_n[ta] + sc_n[64 + ta], n1 = sc_n[tb] + sc_n[64 + tb];
-        const float w0 = w_s[ta], w1 = w_s[tb], r0 = r_s[ta], r1 = r_s[tb];
-        const float c0 = kappa * n0, c1 = kappa * n1;
-        const Mat2 M0 = {r0 * a0 * a0, r0 * w0, c0 * a0 * a0, fmaf(c0, w0, r0)};
-        const Mat2 M1 = {r1 * a1 * a1, r1 * w1, c1 * a1 * a1, fmaf(c1, w1, r1)};
-        Mat2 Pm = mnorm(mmul(M1, M0));
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          Mat2 o;
-          o.a = __shfl_up_sync(0xffffffffu, Pm.a, d);
-          o.b = __shfl_up_sync(0xffffffffu, Pm.b, d);
-          o.c = __shfl_up_sync(0xffffffffu, Pm.c, d);
-          o.d = __shfl_up_sync(0xffffffffu, Pm.d, d);
-          if (lane >= d) Pm = mnorm(mmul(Pm, o));
-        }
-        Mat2 ex;
-        ex.a = __shfl_up_sync(0xffffffffu, Pm.a, 1);
-        ex.b = __shfl_up_sync(0xffffffffu, Pm.b, 1);
-        ex.c = __shfl_up_sync(0xffffffffu, Pm.c, 1);
-        ex.d = __shfl_up_sync(0xffffffffu, Pm.d, 1);
-        const float carry = sc_pcar[0];
-        float p = lane == 0 ? carry
-                            : __fdividef(fmaf(ex.a, carry, ex.b), fmaf(ex.c, carry, ex.d));
-        const float pp0 = fmaf(a0 * a0, p, w0);
-        p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
-        const float pp1 = fmaf(a1 * a1, p, w1);
-        p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
-        const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
-        const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
-        const float lg0 = sc_lg[64 * s + ta], lg1 = sc_lg[64 * s + tb];
-        const float lg_last = __shfl_sync(0xffffffffu, lg1, 31);
-        sc_beta[64 * s + ta] = b0;
-        sc_beta[64 * s + tb] = b1;
-        sc_coef[64 * s + ta] = b0 * exp2f(lg_last - lg0);
-        sc_coef[64 * s + tb] = b1 * exp2f(lg_last - lg1);
-        const float pnext = __shfl_sync(0xffffffffu, p, 31);
-        __syncwarp();
-        if (lane == 0) sc_pcar[0] = pnext;
-      }
-      if (warp == 14 && c + 1 < nchunks) store_scalars(c + 1);
-      bar_group(kPrepBar);
-
+      const int sl = c & 3;
       // ---- D1 epilogue: A (key rows) into AT; P (query rows) kept
-      if (fail(mma1_bar, (uint32_t)(c & 1))) pbad = true;
-      else if (mma_issuer) pend_mma1 = -1;
+      if (fail(mma1_bar, (uint32_t)(c & 1))) bad = true;
+      else if (mma1_issuer) pend_mma1 = -1;
       tc_fence_after();
-      const float* lg_c = sc_lg + 64 * s;
-      const float* beta_c = sc_beta + 64 * s;
+      const float* lg_c = sc_lg + 64 * sl;
+      const float* beta_c = sc_beta + 64 * sl;
       float preg[32];
       {
         float d1[32];
@@ -1568,7 +1589,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float bv[4] = {bj.x, bj.y, bj.z, bj.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float val = exp2f(lg_t - lj[e]) * bv[e] * d1[4 * i4 + e];
+            const float val = ex2_approx(lg_t - lj[e]) * bv[e] * d1[4 * i4 + e];
             preg[4 * i4 + e] = (j0 + e < lim) ? val : 0.f;
           }
         }
@@ -1582,54 +1603,58 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
               make_float4(preg[4 * i4], preg[4 * i4 + 1], preg[4 * i4 + 2], preg[4 * i4 + 3]);
       }
       bar_group(kPrepBar);
-
-      // ---- T = (I + A)^-1 into AT (for the solve) and as the bf16 hi/lo B
-      // operand [t][j] of MMA3, once MMA3 of the previous chunk released it.
-      // AT keeps A below the diagonal blocks; T's blocks below the diagonal go
-      // to the transposed places above it (T_ib[r][c] at AT[16 b + c][16 i + r]).
-      if (c > 0 && fail(mma3_bar, (uint32_t)((c - 1) & 1))) pbad = true;
-      if (ptid < 64) {
-        const int blk = ptid >> 4, cc = ptid & 15;
-        const float* Ab = AT + 16 * blk * kLd + 16 * blk;
-        float x[16], acc[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l) {
-          x[l] = (l == cc) ? 1.f : (l < cc ? 0.f : -acc[l]);
-#pragma unroll
-          for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kLd + l], x[l], acc[i]);
-        }
-        named_bar<kPhase1Bar, 64>();  // all A columns read
-#pragma unroll
-        for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
+      // MMA1 of the next chunk: D1 has been read
+      if (mma1_issuer && !bad && c + 1 < nchunks) {
+        if (fail(&full_kq[(c + 1) % P::kStages], kq_parity(c + 1))) bad = true;
+        else issue_mma1(c + 1);
       }
-      bar_group(kPrepBar);
-      {
-        const int pw = warp - 8;
+
+      if (pw < 4) {
+        // ---- T = (I + A)^-1 (warps 8-11) into AT and as the bf16 hi/lo B
+        // operand [t][j] of MMA3, once MMA3 of the previous chunk released it.
+        // AT keeps A below the diagonal blocks; T's blocks below the diagonal
+        // go to the transposed places above it (T_ib[r][c] at AT[16 b + c][16 i + r]).
+        if (c > 0 && fail(mma3_bar, (uint32_t)((c - 1) & 1))) bad = true;
+        if (ptid < 64) {
+          const int blk = ptid >> 4, cc = ptid & 15;
+          const float* Ab = AT + 16 * blk * kLd + 16 * blk;
+          float x[16], acc[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            x[l] = (l == cc) ? 1.f : (l < cc ? 0.f : -acc[l]);
+#pragma unroll
+            for (int i = l + 1; i < 16; ++i) acc[i] = fmaf(Ab[i * kLd + l], x[l], acc[i]);
+          }
+          named_bar<kPhase1Bar, 64>();  // all A columns read
+#pragma unroll
+          for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
+        }
+        named_bar<kTeamA, 128>();
         auto Ael = [&](int i, int l, int r, int k) { return AT[(16 * i + r) * kLd + 16 * l + k]; };
         auto Tdg = [&](int i, int r, int k) { return AT[(16 * i + r) * kLd + 16 * i + k]; };
-        auto Tlo = [&](int i, int b, int r, int k) { return AT[(16 * b + k) * kLd + 16 * i + r]; };
-        auto Tset = [&](int i, int b, int r, int k, float v0, float v1) {
-          AT[(16 * b + k) * kLd + 16 * i + r] = v0;
-          AT[(16 * b + k + 1) * kLd + 16 * i + r] = v1;
+        auto Tlo = [&](int i, int bb, int r, int k) { return AT[(16 * bb + k) * kLd + 16 * i + r]; };
+        auto Tset = [&](int i, int bb, int r, int k, float v0, float v1) {
+          AT[(16 * bb + k) * kLd + 16 * i + r] = v0;
+          AT[(16 * bb + k + 1) * kLd + 16 * i + r] = v1;
         };
-        auto Top = [&](int i, int b, int r, int k, float v0, float v1) {
-          // T[16 i + r][16 b + k, +1] as bf16 hi/lo pairs
+        auto Top = [&](int i, int bb, int r, int k, float v0, float v1) {
+          // T[16 i + r][16 bb + k, +1] as bf16 hi/lo pairs
           uint32_t hi, lo;
           split_pack2(v0, v1, hi, lo);
-          const uint32_t row = (uint32_t)(16 * i + r), col = (uint32_t)(16 * b + k);
+          const uint32_t row = (uint32_t)(16 * i + r), col = (uint32_t)(16 * bb + k);
           const uint32_t off = chunk_off(row, col >> 3) + ((col & 7u) << 1);
           *reinterpret_cast<uint32_t*>(sT + off) = hi;
           *reinterpret_cast<uint32_t*>(sT + 8192 + off) = lo;
         };
         if (pw < 2) {
           // T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_bb inside each 32-block (b = 0, 2)
-          const int b = 2 * pw, i = b + 1;
+          const int bb = 2 * pw, i = bb + 1;
           float* xs = X + pw * 320;
           float acc[3][2][4] = {};
-          warp_mm16(acc, [&](int r, int k) { return Ael(i, b, r, k); },
-                    [&](int k, int n) { return Tdg(b, k, n); }, lane);
+          warp_mm16(acc, [&](int r, int k) { return Ael(i, bb, r, k); },
+                    [&](int k, int n) { return Tdg(bb, k, n); }, lane);
           warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
             *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
           __syncwarp();
@@ -1637,23 +1662,27 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           warp_mm16(acc2, [&](int r, int k) { return Tdg(i, r, k); },
                     [&](int k, int n) { return xs[k * 20 + n]; }, lane);
           warp_put16(acc2, -1.f, [&](int r, int k, float v0, float v1) {
-            Tset(i, b, r, k, v0, v1);
-            Top(i, b, r, k, v0, v1); }, lane);
-        } else if (pw < 6) {
-          // the diagonal blocks into the operand: lane -> row r, 8 columns
-          const int i = pw - 2, r = lane >> 1, half = lane & 1;
-          const float* src = AT + (16 * i + r) * kLd + 16 * i + 8 * half;
-          const float4 x0 = *reinterpret_cast<const float4*>(src);
-          const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
-          const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-          st_split8(sT, (uint32_t)(16 * i + r), sT + 8192, (uint32_t)(16 * i + r),
-                    (uint32_t)(2 * i + half), x);
+            Tset(i, bb, r, k, v0, v1);
+            Top(i, bb, r, k, v0, v1); }, lane);
+        } else {
+          // the diagonal blocks into the operand (two per warp): lane -> row r, 8 columns
+          const int r = lane >> 1, half = lane & 1;
+#pragma unroll
+          for (int bi = 0; bi < 2; ++bi) {
+            const int i = 2 * (pw - 2) + bi;
+            const float* src = AT + (16 * i + r) * kLd + 16 * i + 8 * half;
+            const float4 x0 = *reinterpret_cast<const float4*>(src);
+            const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
+            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            st_split8(sT, (uint32_t)(16 * i + r), sT + 8192, (uint32_t)(16 * i + r),
+                      (uint32_t)(2 * i + half), x);
+          }
         }
-        bar_group(kPrepBar);
+        named_bar<kTeamA, 128>();
         // the 32x32 block below the diagonal: T^(10) = -T^(1) (A^(10) T^(0)),
-        // first X2 = A^(10) T^(0) by four warps, one 16x16 block each
+        // first X2 = A^(10) T^(0), one 16x16 block per warp
         const int i2 = 2 + (pw >> 1), b2 = pw & 1;
-        if (pw < 4) {
+        {
           float acc[3][2][4] = {};
           if (b2 == 0) {
             warp_mm16(acc, [&](int r, int k) { return Ael(i2, 0, r, k); },
@@ -1668,10 +1697,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
             *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
         }
-        bar_group(kPrepBar);
-        if (pw < 4) {
+        named_bar<kTeamA, 128>();
+        {
+          // X2 block (mm, b2) sits in X slot 2 (mm - 2) + b2
           float acc[3][2][4] = {};
-          // X2 block (m, b2) sits in X slot 2 (m - 2) + b2
           if (i2 == 2) {
             warp_mm16(acc, [&](int r, int k) { return Tdg(2, r, k); },
                       [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
@@ -1684,14 +1713,24 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           warp_put16(acc, -1.f, [&](int r, int k, float v0, float v1) {
             Top(i2, b2, r, k, v0, v1); }, lane);
         }
+        fence_async_smem();
+        named_bar<kTeamA, 128>();
+        if (ptid == 0) mbar_arrive(t_ready);
+      } else if (c + 1 < nchunks) {
+        // ---- the next chunk's scalars (warps 12-15)
+        if (warp == 13) {
+          store_scalars(c + 1);
+          if (c + 2 < nchunks) fetch_scalars(c + 2);
+        }
+        if (fail(&full_kq[(c + 1) % P::kStages], kq_parity(c + 1))) bad = true;
+        key_norms(c + 1, ptid - 128);
+        named_bar<kTeamB, 128>();
+        if (warp == 12) decay_and_variance(c + 1);
       }
-      fence_async_smem();
-      bar_group(kPrepBar);
-      if (ptid == 0) mbar_arrive(t_ready);
 
       // ---- P as the tf32 B operand [t][j], once MMA4 of the previous chunk
       // released the buffer
-      if (c > 0 && fail(mma4_bar, (uint32_t)((c - 1) & 1))) pbad = true;
+      if (c > 0 && fail(mma4_bar, (uint32_t)((c - 1) & 1))) bad = true;
       if (qrow) {
         uint8_t* dst = sP + pch * 8192;
 #pragma unroll
@@ -1701,14 +1740,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                          rna_tf32(preg[4 * q + 2]), rna_tf32(preg[4 * q + 3]));
       }
       fence_async_smem();
-      if (bar_group_or(kPrepBar, pbad || *sc_abort != 0.f)) {
-        pbad = true;
+      if (bar_group_or(kPrepBar, bad || *sc_abort != 0.f)) {
+        bad = true;
         break;
       }
       if (ptid == 0) mbar_arrive(p_ready);
     }
-    if (mma_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
-    if (ptid == 0 && !pbad) P_out[bh] = sc_pcar[0];
+    if (mma1_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
+    if (ptid == 0 && !bad) P_out[bh] = sc_pcar[0];
   }
   tc_fence_before();
   __syncthreads();
@@ -1740,6 +1779,19 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int 
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [B, T, H, d] fp32 output, boxes of (d columns, 1 head, box_t tokens, 1 batch)
+bool make_out_map(CUtensorMap* m, void* base, int B, int T, int H, int d, int box_t) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
+  cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_t, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <bool DIAG, int NV>
@@ -1781,9 +1833,9 @@ kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a
                      float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
                      cudaStream_t s) {
   using P = WsPlan;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, B, T, H, kDK, 64) || !make_map(&mk, k, B, T, H, kDK, 64) ||
-      !make_map(&mv, v, B, T, H, 128, 64))
+      !make_map(&mv, v, B, T, H, 128, 64) || !make_out_map(&mo, o, B, T, H, 128, 64))
     return KDN_ERR_CUDA;
   static bool attr_set = false;
   if (!attr_set) {
@@ -1794,7 +1846,7 @@ kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a
   }
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
   chunk_engine_ws_kernel<<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
-      mq, mk, mv, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa, static_cast<uint32_t*>(ws));
+      mq, mk, mv, mo, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa, static_cast<uint32_t*>(ws));
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 

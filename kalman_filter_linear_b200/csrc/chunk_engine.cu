@@ -1290,9 +1290,12 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto issue_mma1 = [&](int c) {
     const uint32_t kq_a = sbase + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES;
     tc_fence_after();
+    const uint64_t d0 = umma_desc_sw128(kq_a, 16, 1024);
+#pragma unroll
     for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t d = umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024);
+        const uint64_t d = d0 + (uint64_t)((kb * 16384 + ks * 32) >> 4);
         umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
       }
     umma_commit(mma1_bar);
@@ -1387,11 +1390,16 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (issuer && !bad) {
         tc_fence_after();
+        // descriptor start addresses advance by (byte offset >> 4)
+        const uint64_t dkq = umma_desc_sw128(kq_a, 16, 1024);
+#pragma unroll
         for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
           for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
             for (int ks = 0; ks < 4; ++ks)
               umma_bf16_ts(tmem + P::COL_D2, tmem + P::COL_W + 64 * hl + 32 * kb + 8 * ks,
-                           umma_desc_sw128(kq_a + kb * 16384 + ks * 32, 16, 1024), ID_2,
+                           dkq + (uint64_t)((kb * 16384 + ks * 32) >> 4), ID_2,
                            (hl > 0 || kb > 0 || ks > 0) ? 1u : 0u);
         umma_commit(mma2_bar);
         pend_mma2 = c & 1;
@@ -1403,32 +1411,73 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
 
       // ---- Z^T = V^T - gamma (K S')^T as bf16 hi/lo token pairs (in W, which
-      // MMA2 has read); gamma (Q S')^T in place; the state decays by gamma_C
+      // MMA2 has read)
       {
-        float z[32], qs[32];
+        float z[32];
         uint32_t hi[16], lo[16];
         tmem_ld32(tmem + tm_lane + P::COL_D2 + 32 * ch, z);
-        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qs);
         tmem_wait_ld();
-        const uint8_t* vt = sV + (v >> 6) * 8192;
-        const float* gm = sc_gam + 64 * sl + 32 * ch;
-        uint32_t qr[32];
+        // V[t][v] of the swizzled tile: rows t = 32 ch + i, whose byte offset
+        // within the row depends on t mod 8 = i mod 8 only
+        const uint8_t* vrow = sV + (v >> 6) * 8192 + 4096 * ch;
+        uint32_t voff[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const uint16_t vb =
-              *reinterpret_cast<const uint16_t*>(vt + sw128_offset((uint32_t)(32 * ch + i),
-                                                                   (uint32_t)(v & 63)));
-          const float g = gm[i];
-          z[i] = fmaf(-g, z[i], __uint_as_float((uint32_t)vb << 16));
-          qr[i] = __float_as_uint(g * qs[i]);
+        for (int r8 = 0; r8 < 8; ++r8)
+          voff[r8] = (((((uint32_t)v & 63u) >> 3) ^ (uint32_t)r8) << 4) | (((uint32_t)v & 7u) << 1);
+        const float4* gm4 = reinterpret_cast<const float4*>(sc_gam + 64 * sl + 32 * ch);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 g4 = gm4[i4];
+          const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * i4 + e;
+            const uint16_t vb = *reinterpret_cast<const uint16_t*>(vrow + i * 128 + voff[i & 7]);
+            z[i] = fmaf(-gv[e], z[i], __uint_as_float((uint32_t)vb << 16));
+          }
         }
 #pragma unroll
         for (int i = 0; i < 16; ++i) split_pack2(z[2 * i], z[2 * i + 1], hi[i], lo[i]);
         tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);
         tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);
-        tmem_st32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qr);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      bar_group(kChainBar);
+      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
+
+      // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
+      if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
+      if (issuer && !bad) {
+        tc_fence_after();
+        const uint64_t dt = umma_desc_sw128(sbase + P::OFF_T, 16, 1024);
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16_ts(tmem + P::COL_D3, tmem + P::COL_W + (term == 1 ? 32 : 0) + 8 * ks,
+                         dt + (uint64_t)(((term == 2 ? 8192 : 0) + ks * 32) >> 4), ID_3,
+                         (term > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(mma3_bar);
+        pend_mma3 = c & 1;
+      }
+      // ---- while MMA3 runs: gamma (Q S')^T in place (before MMA4 adds to it)
+      // and the state decay by gamma_C (before MMA5 adds to it)
       {
+        float qs[32];
+        uint32_t qr[32];
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qs);
+        tmem_wait_ld();
+        const float4* gm4 = reinterpret_cast<const float4*>(sc_gam + 64 * sl + 32 * ch);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 g4 = gm4[i4];
+          qr[4 * i4] = __float_as_uint(g4.x * qs[4 * i4]);
+          qr[4 * i4 + 1] = __float_as_uint(g4.y * qs[4 * i4 + 1]);
+          qr[4 * i4 + 2] = __float_as_uint(g4.z * qs[4 * i4 + 2]);
+          qr[4 * i4 + 3] = __float_as_uint(g4.w * qs[4 * i4 + 3]);
+        }
+        tmem_st32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qr);
         const float gC = sc_gC[sl];
 #pragma unroll
         for (int h32 = 0; h32 < 2; ++h32) {
@@ -1441,24 +1490,6 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_st32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, r);
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      bar_group(kChainBar);
-      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
-
-      // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
-      if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
-      if (issuer && !bad) {
-        tc_fence_after();
-        for (int term = 0; term < 3; ++term)
-          for (int ks = 0; ks < 4; ++ks)
-            umma_bf16_ts(tmem + P::COL_D3, tmem + P::COL_W + (term == 1 ? 32 : 0) + 8 * ks,
-                         umma_desc_sw128(sbase + P::OFF_T + (term == 2 ? 8192 : 0) + ks * 32, 16,
-                                         1024),
-                         ID_3, (term > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(mma3_bar);
-        pend_mma3 = c & 1;
-      }
       if (fail(mma3_bar, (uint32_t)(c & 1))) bad = true;
       else if (issuer) pend_mma3 = -1;
       tc_fence_after();
@@ -1468,12 +1499,13 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         float u[32];
         tmem_ld32(tmem + tm_lane + P::COL_D3 + 32 * ch, u);
         tmem_wait_ld();
-        const float* cf = sc_coef + 64 * sl + 32 * ch;
+        const float4* cf4 = reinterpret_cast<const float4*>(sc_coef + 64 * sl + 32 * ch);
         uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 cc = *reinterpret_cast<const float2*>(cf + 2 * i);
-          split_pack2(cc.x * u[2 * i], cc.y * u[2 * i + 1], hi[i], lo[i]);
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 c4 = cf4[i4];
+          split_pack2(c4.x * u[4 * i4], c4.y * u[4 * i4 + 1], hi[2 * i4], lo[2 * i4]);
+          split_pack2(c4.z * u[4 * i4 + 2], c4.w * u[4 * i4 + 3], hi[2 * i4 + 1], lo[2 * i4 + 1]);
         }
         tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);  // Z has been read
         tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);
@@ -1488,17 +1520,20 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (issuer && !bad) {
         tc_fence_after();
         // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
+        const uint64_t dk = umma_desc_sw128(kq_a, 16384, 1024);
+#pragma unroll
         for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_W + 32 * hl + 8 * ks,
-                         umma_desc_sw128(kq_a + ks * 2048, 16384, 1024), ID_5, 1u);
+                         dk + (uint64_t)((ks * 2048) >> 4), ID_5, 1u);
         umma_commit(mma5_bar);
         pend_mma5 = c & 1;
+        const uint64_t dp = umma_desc_sw128(sbase + P::OFF_P, 16, 1024);
+#pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           umma_tf32_ts(tmem + P::COL_D2 + 64, tmem + P::COL_D3 + 8 * ks,
-                       umma_desc_sw128(sbase + P::OFF_P + (ks >> 2) * 8192 + (ks & 3) * 32, 16,
-                                       1024),
-                       ID_4, 1u);
+                       dp + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), ID_4, 1u);
         umma_commit(mma4_bar);
         pend_mma4 = c & 1;
       }

@@ -156,11 +156,12 @@ __device__ __forceinline__ Mat2 mnorm(const Mat2& x) {
   return x;
 }
 
-// Named barriers use the non-aligned form: threads of a warp may arrive
-// separately (single-lane issue blocks and bounded waits diverge a warp), and
-// each thread is counted on its own.
+// Named barriers are the aligned form, which needs the whole warp to arrive
+// together: single-lane issue blocks and bounded waits diverge warps, so each
+// barrier first reconverges its warp.
 __device__ __forceinline__ void bar_compute() {
-  asm volatile("barrier.sync 1, %0;" ::"n"(kCompute) : "memory");
+  __syncwarp();
+  asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory");
 }
 
 // `steps` consecutive K=16 MMAs; descriptor start addresses advance by
@@ -180,7 +181,8 @@ __device__ __forceinline__ void mma_steps(uint32_t tmem_d, uint64_t a0, uint64_t
 // bound is a compile-time constant.
 template <int BAR, int NT>
 __device__ __forceinline__ void named_bar() {
-  asm volatile("barrier.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+  __syncwarp();
+  asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
 }
 
 // Every level uses at most 256 threads (tid < 256); BAR / NT name the barrier
@@ -1061,17 +1063,19 @@ __device__ __forceinline__ void warp_put16(const float (&acc)[3][2][4], float s,
 constexpr int kChainBar = 3, kPrepBar = 4, kPhase1Bar = 5, kGroup = 256;
 
 __device__ __forceinline__ void bar_group(int id) {
-  asm volatile("barrier.sync %0, %1;" ::"r"(id), "n"(kGroup) : "memory");
+  __syncwarp();
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "n"(kGroup) : "memory");
 }
 
 // Barrier of one 256-thread group that also ORs a flag over the group, so an
 // abort decision taken after it is the same in every thread of the group.
 __device__ __forceinline__ bool bar_group_or(int id, bool flag) {
   uint32_t r;
+  __syncwarp();
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "barrier.red.or.pred q, %2, %3, p;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)flag), "r"(id), "n"(kGroup)

@@ -27,6 +27,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -57,6 +58,29 @@ def layer_bytes(variant, B, T, H, dk, dv, in_bytes=2):
     o = B * T * H * dv * 4
     st = B * H * dv * dk * 4 + B * H * (dk if variant == 'diag' else 1) * 4
     return qkv + ar + w + o + st
+
+
+PROFILE = os.path.join(ROOT, 'profiles', 'chunk_engine_ws_iso_B4_T4096_H16_d128.md')
+ENGINE_SOURCES = [os.path.join(ROOT, 'kalman_filter_linear_b200', 'csrc', f)
+                  for f in ('chunk_engine.cu', 'kdn_common.cuh')]
+
+
+def captured_traffic(heads):
+    """DRAM bytes (read + write) of one launch over `heads` heads, scaled from
+    the committed ncu capture of the isotropic engine -- or None when the
+    engine's sources changed since that capture (its counters no longer
+    describe the kernel that runs)."""
+    import hashlib
+    try:
+        text = open(PROFILE).read()
+        per_head = float(re.search(r'^traffic-bytes-per-head: (\d+)', text, re.M).group(1))
+        digest = re.search(r'^source-sha256-16: ([0-9a-f]+)', text, re.M).group(1)
+    except (OSError, AttributeError):
+        return None
+    h = hashlib.sha256()
+    for f in ENGINE_SOURCES:
+        h.update(open(f, 'rb').read())
+    return per_head * heads if h.hexdigest()[:16] == digest else None
 
 
 def decode_bytes(B, H, dk, dv):
@@ -334,7 +358,7 @@ def main():
                    'l2': 'inputs (403 MB q/k/v) larger than the 126 MB L2; no flush',
                    'parallelism': f'dp{world} (independent replicas, no collective)'},
         'roofline': {'bound': 'hbm', 'achieved': achieved, 'peak': hbm_peak, 'unit': 'GB/s',
-                     'frac': achieved / hbm_peak, 'traffic': None,
+                     'frac': achieved / hbm_peak, 'traffic': captured_traffic(B * H),
                      'algorithmic_bytes': alg, 'peak_source': peak_kind},
         'e2e': {'value': e2e_value, 'unit': 'tokens/s', 'h2d_bytes_per_step': h2d,
                 'd2h_bytes_per_step': d2h},

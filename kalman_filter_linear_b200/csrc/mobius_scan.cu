@@ -28,6 +28,7 @@
 // All products have non-negative entries (no cancellation).  They are
 // renormalised by powers of two, which is exact, so renormalisation adds no
 // rounding.
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -87,54 +88,28 @@ struct ScanWs {
 __device__ __forceinline__ float4 as_f4(const Mat2& m) { return make_float4(m.a, m.b, m.c, m.d); }
 __device__ __forceinline__ Mat2 as_mat(const float4& f) { return {f.x, f.y, f.z, f.w}; }
 
-__global__ void __launch_bounds__(kThreads)
-mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
-                   const float* __restrict__ R, const float* __restrict__ Nsq,
-                   const float* __restrict__ lambda0, float info_scale,
-                   float* __restrict__ lam_out, float* __restrict__ prior_out,
-                   float* __restrict__ gain_out, int64_t N, int64_t T, int64_t tiles_per_lane,
-                   ScanWs ws, int vec_ok, int64_t debug_skip_tile) {
-  __shared__ Mat2 s_warp[kThreads / 32];
-  __shared__ Mat2 s_tile_prefix;
-  __shared__ uint32_t s_tile;
+struct TileShared {
+  Mat2 warp_incl[kThreads / 32];
+  Mat2 tile_prefix;
+};
 
+// Steps 1-4 for one tile, given this thread's 8 inputs (a, w, r, n).
+__device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const float (&w)[kPerThread],
+                                          const float (&r)[kPerThread], const float (&n)[kPerThread],
+                                          int64_t tile, const float* __restrict__ lambda0,
+                                          float info_scale, float* __restrict__ lam_out,
+                                          float* __restrict__ prior_out,
+                                          float* __restrict__ gain_out, int64_t N, int64_t T,
+                                          const ScanWs& ws, int vec_ok, int64_t debug_skip_tile,
+                                          TileShared& sh) {
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-
-  if (tid == 0) s_tile = atomicAdd(ws.counter, 1u);
-  __syncthreads();
-  const int64_t tile = s_tile;
   const int64_t j = tile / N;    // tile index within the lane
   const int64_t seq = tile % N;  // lane
   const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
   const int64_t base = seq * T;
-
-  // ---- 1. load and compose this thread's maps
-  float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
-  if (vec_ok && t0 + kPerThread <= T) {
-    const float4* a4 = reinterpret_cast<const float4*>(A + base + t0);
-    const float4* w4 = reinterpret_cast<const float4*>(W + base + t0);
-    const float4* r4 = reinterpret_cast<const float4*>(R + base + t0);
-    const float4* n4 = reinterpret_cast<const float4*>(Nsq + base + t0);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float4 x = __ldg(a4 + h), y = __ldg(w4 + h), z = __ldg(r4 + h), u = __ldg(n4 + h);
-      a[4 * h] = x.x; a[4 * h + 1] = x.y; a[4 * h + 2] = x.z; a[4 * h + 3] = x.w;
-      w[4 * h] = y.x; w[4 * h + 1] = y.y; w[4 * h + 2] = y.z; w[4 * h + 3] = y.w;
-      r[4 * h] = z.x; r[4 * h + 1] = z.y; r[4 * h + 2] = z.z; r[4 * h + 3] = z.w;
-      n[4 * h] = u.x; n[4 * h + 1] = u.y; n[4 * h + 2] = u.z; n[4 * h + 3] = u.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < kPerThread; ++i) {
-      const bool in = t0 + i < T;
-      a[i] = in ? __ldg(A + base + t0 + i) : 1.f;
-      w[i] = in ? __ldg(W + base + t0 + i) : 0.f;
-      r[i] = in ? __ldg(R + base + t0 + i) : 1.f;
-      n[i] = in ? __ldg(Nsq + base + t0 + i) : 0.f;
-    }
-  }
+  Mat2* s_warp = sh.warp_incl;
 
   Mat2 P = identity();
 #pragma unroll
@@ -169,7 +144,8 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
   }
   __syncthreads();
 
-  // ---- 3. decoupled look-back (thread 0)
+  // ---- 3. decoupled look-back (thread 0).  The release store of a flag
+  // orders this thread's earlier stores of the prefix data before it.
   if (tid == 0) {
     const Mat2 agg = s_warp[kThreads / 32 - 1];
     Mat2 excl = identity();
@@ -177,44 +153,51 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
     if (j == 0) {
       if (!skip_publish) {
         ws.incl[tile] = as_f4(agg);
-        __threadfence();
         st_release_u32(ws.flag + tile, 2u);
       }
     } else {
-      if (!skip_publish) {
-        ws.agg[tile] = as_f4(agg);
-        __threadfence();
-        st_release_u32(ws.flag + tile, 1u);
-      }
-      const uint64_t start = globaltimer_ns();
-      bool timed_out = false;
-      for (int64_t p = j - 1; p >= 0 && !timed_out;) {
-        const int64_t pt = p * N + seq;
-        uint32_t f = ld_acquire_u32(ws.flag + pt);
-        while (f == 0u) {
-          if (globaltimer_ns() - start > kWaitLimitNs) {
-            timed_out = true;
+      // Usually the predecessor has finished: take its inclusive prefix and
+      // publish only this tile's.  Otherwise publish the aggregate first and
+      // look back tile by tile.
+      const int64_t pt0 = (j - 1) * N + seq;
+      uint32_t f0 = ld_acquire_u32(ws.flag + pt0);
+      if (f0 != 2u) {
+        if (!skip_publish) {
+          ws.agg[tile] = as_f4(agg);
+          st_release_u32(ws.flag + tile, 1u);
+        }
+        const uint64_t start = globaltimer_ns();
+        bool timed_out = false;
+        for (int64_t p = j - 1; p >= 0 && !timed_out;) {
+          const int64_t pt = p * N + seq;
+          uint32_t f = (p == j - 1) ? f0 : ld_acquire_u32(ws.flag + pt);
+          while (f == 0u) {
+            if (globaltimer_ns() - start > kWaitLimitNs) {
+              timed_out = true;
+              break;
+            }
+            __nanosleep(64);
+            f = ld_acquire_u32(ws.flag + pt);
+          }
+          if (timed_out) break;
+          if (f == 2u) {
+            excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
             break;
           }
-          __nanosleep(64);
-          f = ld_acquire_u32(ws.flag + pt);
+          excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
+          f0 = 0u;
+          --p;
         }
-        if (timed_out) break;
-        if (f == 2u) {
-          excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
-          break;
-        }
-        excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
-        --p;
+        if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
+      } else {
+        excl = as_mat(__ldcg(ws.incl + pt0));
       }
-      if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
       if (!skip_publish) {
         ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
-        __threadfence();
         st_release_u32(ws.flag + tile, 2u);
       }
     }
-    s_tile_prefix = excl;
+    sh.tile_prefix = excl;
   }
   __syncthreads();
 
@@ -222,7 +205,7 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
   Mat2 thread_excl = shfl_up(incl, 1);
   if (lane == 0) thread_excl = identity();
   if (warp > 0) thread_excl = mul(thread_excl, s_warp[warp - 1]);
-  thread_excl = renorm(mul(renorm(thread_excl), s_tile_prefix));
+  thread_excl = renorm(mul(renorm(thread_excl), sh.tile_prefix));
   const float lam0 = lambda0 ? __ldg(lambda0 + seq) : 1.f;
   float lam = apply(thread_excl, lam0);
 
@@ -260,6 +243,146 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
       }
     }
   }
+}
+
+// One tile per CTA, inputs straight from global memory (any T).
+__global__ void __launch_bounds__(kThreads)
+mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
+                   const float* __restrict__ R, const float* __restrict__ Nsq,
+                   const float* __restrict__ lambda0, float info_scale,
+                   float* __restrict__ lam_out, float* __restrict__ prior_out,
+                   float* __restrict__ gain_out, int64_t N, int64_t T, ScanWs ws, int vec_ok,
+                   int64_t debug_skip_tile) {
+  __shared__ TileShared sh;
+  __shared__ uint32_t s_tile;
+  const int tid = threadIdx.x;
+  if (tid == 0) s_tile = atomicAdd(ws.counter, 1u);
+  __syncthreads();
+  const int64_t tile = s_tile;
+  const int64_t j = tile / N, seq = tile % N;
+  const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
+  const int64_t base = seq * T;
+  float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
+  if (vec_ok && t0 + kPerThread <= T) {
+    const float4* a4 = reinterpret_cast<const float4*>(A + base + t0);
+    const float4* w4 = reinterpret_cast<const float4*>(W + base + t0);
+    const float4* r4 = reinterpret_cast<const float4*>(R + base + t0);
+    const float4* n4 = reinterpret_cast<const float4*>(Nsq + base + t0);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float4 x = __ldg(a4 + h), y = __ldg(w4 + h), z = __ldg(r4 + h), u = __ldg(n4 + h);
+      a[4 * h] = x.x; a[4 * h + 1] = x.y; a[4 * h + 2] = x.z; a[4 * h + 3] = x.w;
+      w[4 * h] = y.x; w[4 * h + 1] = y.y; w[4 * h + 2] = y.z; w[4 * h + 3] = y.w;
+      r[4 * h] = z.x; r[4 * h + 1] = z.y; r[4 * h + 2] = z.z; r[4 * h + 3] = z.w;
+      n[4 * h] = u.x; n[4 * h + 1] = u.y; n[4 * h + 2] = u.z; n[4 * h + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const bool in = t0 + i < T;
+      a[i] = in ? __ldg(A + base + t0 + i) : 1.f;
+      w[i] = in ? __ldg(W + base + t0 + i) : 0.f;
+      r[i] = in ? __ldg(R + base + t0 + i) : 1.f;
+      n[i] = in ? __ldg(Nsq + base + t0 + i) : 0.f;
+    }
+  }
+  scan_tile(a, w, r, n, tile, lambda0, info_scale, lam_out, prior_out, gain_out, N, T, ws, vec_ok,
+            debug_skip_tile, sh);
+}
+
+// Persistent form for T a multiple of 4: each CTA takes tiles in counter
+// order.  Once its threads have moved a tile's inputs into registers, it
+// copies the next tile's inputs into the shared-memory buffer (bulk async
+// copies) while it scans the current tile, so input traffic is in flight
+// during the look-back and the recursion.  A CTA takes the next tile before
+// it finishes the current one; every tile it waits on has a smaller index and
+// was taken earlier, so some CTA is working on it.
+constexpr uint32_t kTileBytes = kTile * 4;  // one input array of a tile
+constexpr uint32_t kBufBytes = 4 * kTileBytes;
+constexpr int kPersistentCtasPerSm = 4;
+
+__global__ void __launch_bounds__(kThreads, kPersistentCtasPerSm)
+mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
+                       const float* __restrict__ R, const float* __restrict__ Nsq,
+                       const float* __restrict__ lambda0, float info_scale,
+                       float* __restrict__ lam_out, float* __restrict__ prior_out,
+                       float* __restrict__ gain_out, int64_t N, int64_t T, int64_t ntiles,
+                       ScanWs ws, int64_t debug_skip_tile) {
+  extern __shared__ __align__(128) uint8_t s_in[];  // [a, w, r, n][kTile] fp32
+  __shared__ TileShared sh;
+  __shared__ int64_t s_tile[2];
+  __shared__ uint64_t s_full;
+  const int tid = threadIdx.x;
+  // copies the inputs of `tile` into the buffer (thread 0)
+  auto fetch = [&](int64_t tile) {
+    const float* src[4] = {A, W, R, Nsq};
+    const int64_t j = tile / N, seq = tile % N;
+    const int64_t first = j * kTile;
+    const uint32_t bytes = (uint32_t)(min((int64_t)kTile, T - first) * 4);
+    mbar_expect_tx(&s_full, 4u * bytes);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(smem_u32(s_in + k * kTileBytes)), "l"(src[k] + seq * T + first), "r"(bytes),
+          "r"(smem_u32(&s_full))
+          : "memory");
+    }
+  };
+  if (tid == 0) {
+    mbar_init(&s_full, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const int64_t first = atomicAdd(ws.counter, 1u);
+    s_tile[0] = first;
+    if (first < ntiles) fetch(first);
+  }
+  __syncthreads();
+  for (int it = 0;; ++it) {
+    const int64_t tile = s_tile[it & 1];
+    if (tile >= ntiles) break;
+    // this tile's inputs; if any thread's wait gives up, the CTA records the
+    // timeout and stops
+    const bool late = !mbar_wait(&s_full, (uint32_t)(it & 1));
+    if (__syncthreads_or(late)) {
+      if (tid == 0) atomicOr(ws.error, DEV_TIMEOUT);
+      break;
+    }
+    const int64_t j = tile / N;
+    const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
+    const float* buf = reinterpret_cast<const float*>(s_in);
+    float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float4 x = *reinterpret_cast<const float4*>(buf + 0 * kTile + tid * kPerThread + 4 * h);
+      const float4 y = *reinterpret_cast<const float4*>(buf + 1 * kTile + tid * kPerThread + 4 * h);
+      const float4 z = *reinterpret_cast<const float4*>(buf + 2 * kTile + tid * kPerThread + 4 * h);
+      const float4 u = *reinterpret_cast<const float4*>(buf + 3 * kTile + tid * kPerThread + 4 * h);
+      a[4 * h] = x.x; a[4 * h + 1] = x.y; a[4 * h + 2] = x.z; a[4 * h + 3] = x.w;
+      w[4 * h] = y.x; w[4 * h + 1] = y.y; w[4 * h + 2] = y.z; w[4 * h + 3] = y.w;
+      r[4 * h] = z.x; r[4 * h + 1] = z.y; r[4 * h + 2] = z.z; r[4 * h + 3] = z.w;
+      n[4 * h] = u.x; n[4 * h + 1] = u.y; n[4 * h + 2] = u.z; n[4 * h + 3] = u.w;
+    }
+    __syncthreads();  // the buffer is free: start the next tile's copies
+    if (tid == 0) {
+      const int64_t next = atomicAdd(ws.counter, 1u);
+      s_tile[(it + 1) & 1] = next;
+      if (next < ntiles) fetch(next);
+    }
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i)
+      if (t0 + i >= T) {  // past the end of the lane: identity steps
+        a[i] = 1.f;
+        w[i] = 0.f;
+        r[i] = 1.f;
+        n[i] = 0.f;
+      }
+    scan_tile(a, w, r, n, tile, lambda0, info_scale, lam_out, prior_out, gain_out, N, T, ws, 1,
+              debug_skip_tile, sh);
+    __syncthreads();  // the shared tile state and s_tile are free
+  }
+  // Nothing is in flight at exit: a copy is started only for a tile below
+  // ntiles, which the next iteration waits for (or gives up on, after which
+  // the CTA stops).
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -317,9 +440,29 @@ kdn_status mobius_scan_launch(const float* a, const float* w, const float* r, co
 
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, stream) != cudaSuccess) return KDN_ERR_CUDA;
   const int vec_ok = (T % 4 == 0) ? 1 : 0;
-  mobius_scan_kernel<<<(unsigned)L.ntiles, kThreads, 0, stream>>>(
-      a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out, N, T, L.tiles_per_lane,
-      ws, vec_ok, debug_skip_tile);
+  if (vec_ok) {
+    static int grid_cap = 0;  // CTAs that fit on the device at once
+    if (grid_cap == 0) {
+      int dev = 0, sms = 0, per_sm = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+          cudaFuncSetAttribute(mobius_scan_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               kBufBytes) != cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mobius_scan_persistent, kThreads,
+                                                        kBufBytes) != cudaSuccess ||
+          per_sm < 1)
+        return KDN_ERR_CUDA;
+      grid_cap = sms * per_sm;
+    }
+    const int64_t grid = std::min<int64_t>(L.ntiles, grid_cap);
+    mobius_scan_persistent<<<(unsigned)grid, kThreads, kBufBytes, stream>>>(
+        a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out, N, T, L.ntiles, ws,
+        debug_skip_tile);
+  } else {
+    mobius_scan_kernel<<<(unsigned)L.ntiles, kThreads, 0, stream>>>(
+        a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out, N, T, ws, vec_ok,
+        debug_skip_tile);
+  }
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 

@@ -1907,8 +1907,18 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
   if (dv == 128) {
     // one CTA per head reads p0 and writes p_out: no snapshot needed
     if (!diag) return launch_ws(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s);
-    return diag ? launch<true, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
-                : launch<false, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+    // With few heads, one CTA per head leaves most SMs idle: split each head's
+    // value columns over two CTAs (each repeats the head's input-only work).
+    static int sms = 0;
+    if (sms == 0) {
+      int dev = 0;
+      if (cudaGetDevice(&dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return KDN_ERR_CUDA;
+    }
+    if (2 * B * H <= sms)
+      return launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+    return launch<true, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
   }
   return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
               : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);

@@ -1687,35 +1687,54 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           *reinterpret_cast<uint32_t*>(sT + off) = hi;
           *reinterpret_cast<uint32_t*>(sT + 8192 + off) = lo;
         };
-        if (pw < 2) {
-          // T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_bb inside each 32-block (b = 0, 2)
-          const int bb = 2 * pw, i = bb + 1;
-          float* xs = X + pw * 320;
-          float acc[3][2][4] = {};
-          warp_mm16(acc, [&](int r, int k) { return Ael(i, bb, r, k); },
-                    [&](int k, int n) { return Tdg(bb, k, n); }, lane);
-          warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
-            *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
-          __syncwarp();
-          float acc2[3][2][4] = {};
-          warp_mm16(acc2, [&](int r, int k) { return Tdg(i, r, k); },
-                    [&](int k, int n) { return xs[k * 20 + n]; }, lane);
-          warp_put16(acc2, -1.f, [&](int r, int k, float v0, float v1) {
-            Tset(i, bb, r, k, v0, v1);
-            Top(i, bb, r, k, v0, v1); }, lane);
-        } else {
-          // the diagonal blocks into the operand (two per warp): lane -> row r, 8 columns
-          const int r = lane >> 1, half = lane & 1;
+        // T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_bb inside each 32-block
+        // (b = 0, 2) on the 128 threads: 64 per product, 2x2 outputs each
+        {
+          const int pr = ptid >> 6, e = ptid & 63;
+          const int bb = 2 * pr, i = bb + 1;
+          const int r0 = 2 * (e >> 3), c0 = 2 * (e & 7);
+          float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+          const float* a_r0 = AT + (16 * i + r0) * kLd + 16 * bb;
+          const float* tb = AT + (16 * bb) * kLd + 16 * bb + c0;
 #pragma unroll
-          for (int bi = 0; bi < 2; ++bi) {
-            const int i = 2 * (pw - 2) + bi;
-            const float* src = AT + (16 * i + r) * kLd + 16 * i + 8 * half;
-            const float4 x0 = *reinterpret_cast<const float4*>(src);
-            const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
-            const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-            st_split8(sT, (uint32_t)(16 * i + r), sT + 8192, (uint32_t)(16 * i + r),
-                      (uint32_t)(2 * i + half), x);
+          for (int mm = 0; mm < 16; ++mm) {
+            const float2 tt = *reinterpret_cast<const float2*>(tb + mm * kLd);
+            const float a0v = a_r0[mm], a1v = a_r0[kLd + mm];
+            x00 = fmaf(a0v, tt.x, x00);
+            x01 = fmaf(a0v, tt.y, x01);
+            x10 = fmaf(a1v, tt.x, x10);
+            x11 = fmaf(a1v, tt.y, x11);
           }
+          float* xs = X + pr * 320;
+          *reinterpret_cast<float2*>(xs + r0 * 20 + c0) = make_float2(x00, x01);
+          *reinterpret_cast<float2*>(xs + (r0 + 1) * 20 + c0) = make_float2(x10, x11);
+          named_bar<kTeamA, 128>();
+          const float* t_r0 = AT + (16 * i + r0) * kLd + 16 * i;
+          float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+          for (int mm = 0; mm < 16; ++mm) {
+            const float2 xv = *reinterpret_cast<const float2*>(xs + mm * 20 + c0);
+            const float ta = t_r0[mm], tbv = t_r0[kLd + mm];
+            y00 = fmaf(ta, xv.x, y00);
+            y01 = fmaf(ta, xv.y, y01);
+            y10 = fmaf(tbv, xv.x, y10);
+            y11 = fmaf(tbv, xv.y, y11);
+          }
+          // T_ib rows r0, r0 + 1, columns c0, c0 + 1: AT (transposed) and operand
+          Tset(i, bb, r0, c0, -y00, -y01);
+          Tset(i, bb, r0 + 1, c0, -y10, -y11);
+          Top(i, bb, r0, c0, -y00, -y01);
+          Top(i, bb, r0 + 1, c0, -y10, -y11);
+        }
+        // the diagonal blocks into the operand: item -> row 16 i + r, 8 columns
+        {
+          const int i = ptid >> 5, r = (ptid >> 1) & 15, half = ptid & 1;
+          const float* src = AT + (16 * i + r) * kLd + 16 * i + 8 * half;
+          const float4 x0 = *reinterpret_cast<const float4*>(src);
+          const float4 x1 = *reinterpret_cast<const float4*>(src + 4);
+          const float x[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+          st_split8(sT, (uint32_t)(16 * i + r), sT + 8192, (uint32_t)(16 * i + r),
+                    (uint32_t)(2 * i + half), x);
         }
         named_bar<kTeamA, 128>();
         // the 32x32 block below the diagonal: T^(10) = -T^(1) (A^(10) T^(0)),

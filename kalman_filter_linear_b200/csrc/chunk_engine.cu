@@ -16,8 +16,10 @@
 // exists).  The variance recursion (a Mobius map per token and lane) crosses
 // chunks through one carried value per lane.
 //
-// One CTA owns one (batch, head, block of NV value columns) for the whole
-// sequence: 16 warps.  The K/Q tiles are double-buffered and the V tile is
+// Two engines.  The warp-specialised one further down serves d_v = 128 (both
+// variants).  The lock-step one here serves d_v = 64: one CTA owns one
+// (batch, head, block of NV = 64 value columns) for the whole sequence, 16
+// warps.  The K/Q tiles are double-buffered and the V tile is
 // single-buffered; the copies of chunk c+1 (and its per-token scalars) are
 // issued during chunk c's diagonal-block solve, when 14 of the 16 warps are
 // idle and both buffers are free.  Per chunk:
@@ -937,7 +939,7 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ===========================================================================
-// Warp-specialised isotropic engine (one CTA per head, d_v = 128).
+// Warp-specialised engine (one CTA per head, d_v = 128), both variants.
 //
 // Every product runs transposed, with the value index v on the 128 TMEM lanes,
 // so that the fp32 state S'^T [v][k] stays in TMEM, every operand a lane
@@ -948,28 +950,39 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 //   D3 = Z^T T^T                              U^T (bf16 hi/lo Z and T, three terms)
 //   D2 (query half) += U^T P^T                o^T (tf32: U as the tensor cores
 //                                             truncate it, P rounded)
-//   S'^T = gamma_C S'^T + B^T K,  B = coef U  (bf16 hi/lo B, exact K)
+//   S'^T = gamma_C S'^T + B^T G,  B = coef U  (bf16 hi/lo B; G = K exact, or
+//                                             the diagonal variant's G~ as bf16
+//                                             hi/lo, three terms)
 //
 // Warps 0-7 (the chain) run the part that depends on the state.  Per chunk:
 // MMA2; Z (with gamma_t (Q S')_t and the state decay); MMA3; B = coef U; MMA5
 // and MMA4; the state's bf16 hi/lo operand for the next chunk and the output
-// copy.  Warps 8-15 (prep) run the
-// part that depends only on the chunk's inputs, one chunk ahead: the D1
-// epilogue (A and P) on all eight warps, then T = (I + A)^-1 on warps 8-11
-// while warps 12-15 prepare the next chunk's ||k||^2, decay prefix and
-// variance scan.  MMA1 of the next chunk is issued as soon as D1 is read.
+// (isotropic: a staged tile and one tensor store; diagonal: direct stores).
+// Warps 8-15 (prep) run the part that depends only on the chunk's inputs, one
+// chunk ahead: the D1 epilogue (A, and P once MMA4 of the previous chunk has
+// released its buffer) on all eight warps, then T = (I + A)^-1 on warps 8-11
+// while warps 12-15 prepare the next chunk:
+//   isotropic  ||k||^2, decay prefix and the variance scan; MMA1 of the next
+//              chunk is issued as soon as D1 is read.
+//   diagonal   decay prefix and the per-dimension variance (one thread per
+//              dimension, w copied in 16-token quarters), whose G~ = p^- k is
+//              parked in the free D1 columns until MMA5 of chunk c - 1 has
+//              released the G~ buffer it goes to (two buffers); then MMA1 of
+//              the next chunk, D1 = [K;Q] G~^T.  beta_t = 1 / (k_t.G~_t + r_t)
+//              comes from the diagonal of D1 in the next D1 epilogue.
 // The groups hand over through mbarriers:
 //   t_ready / p_ready   prep -> chain: T / P written, with the chunk's scalars
 //                       and the next chunk's decay
-//   mma3 / mma4         the chain's commits; they also hand T and P back
+//   mma3 / mma4 / mma5  the chain's commits; they also hand T, P and G~ back
 // Per-token scalars live in four slots (chunk index mod 4).
 // TMEM columns: D1 [0,64) (prep); S'^T [64,192); D2 [192,320) (key half, then
 // query half); D3 [320,384); W [384,512) holds in turn S'^T hi [384,448) and lo
 // [448,512) (k pairs), Z^T hi [384,416) and lo [416,448), B^T hi and lo (same).
 // ===========================================================================
+template <bool DIAG>
 struct WsPlan {
   static constexpr uint32_t KQ_BYTES = 32768;           // bf16 [kb 2][K|Q][64 t][64]
-  static constexpr int kStages = 3;
+  static constexpr int kStages = DIAG ? 2 : 3;
   static constexpr uint32_t OFF_KQ = 0;                 // kStages stages
   static constexpr uint32_t OFF_V = kStages * KQ_BYTES; // bf16 [vb 2][64 t][64 v]
   static constexpr uint32_t OFF_T = OFF_V + 16384;      // bf16 hi, lo [64 t][64 j]
@@ -977,14 +990,19 @@ struct WsPlan {
   static constexpr uint32_t OFF_AT = OFF_P + 16384;     // fp32 [64][68]
   static constexpr uint32_t OFF_X = OFF_AT + 64u * kLd * 4u;
   static constexpr uint32_t OFF_SC = OFF_X + 5120u;     // X: fp32 [4][16][20]
-  static constexpr uint32_t OFF_OUT = OFF_SC + 9216u;   // fp32 [64 t][128 v] output tile
-  static constexpr uint32_t OFF_BAR = OFF_OUT + 32768u;
+  // isotropic: fp32 [64 t][128 v] output tile; diagonal: two G~ buffers, each
+  // bf16 hi then lo [kb 2][64 t][64 k]
+  static constexpr uint32_t OFF_OUT = OFF_SC + 9216u;
+  static constexpr uint32_t OFF_G = OFF_OUT;
+  // diagonal: w of 16 tokens, fp32 [16 t][128 k], two buffers
+  static constexpr uint32_t OFF_W = OFF_G + 65536u;
+  static constexpr uint32_t OFF_BAR = DIAG ? OFF_W + 16384u : OFF_OUT + 32768u;
   static constexpr uint32_t TOTAL = OFF_BAR + 256u;
   static constexpr uint32_t ALLOC = TOTAL + 1024u;
   static constexpr uint32_t COL_D1 = 0, COL_ST = 64, COL_D2 = 192, COL_D3 = 320, COL_W = 384;
   static_assert(TOTAL <= 227u * 1024u, "shared memory plan too large");
   static_assert(OFF_V % 1024 == 0 && OFF_T % 1024 == 0 && OFF_P % 1024 == 0 &&
-                    OFF_OUT % 128 == 0,
+                    OFF_OUT % 1024 == 0,
                 "operand alignment");
 };
 
@@ -1085,16 +1103,18 @@ __device__ __forceinline__ bool bar_group_or(int id, bool flag) {
 
 constexpr int kTeamA = 6, kTeamB = 7;
 
+template <bool DIAG>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_o, const float* __restrict__ Ag,
+                       const __grid_constant__ CUtensorMap tm_o,
+                       const __grid_constant__ CUtensorMap tm_w, const float* __restrict__ Ag,
                        const float* __restrict__ Wg, const float* __restrict__ Rg,
                        const float* S0, const float* __restrict__ P0, float* __restrict__ O,
                        float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
                        uint32_t* __restrict__ err) {
-  using P = WsPlan;
+  using P = WsPlan<DIAG>;
   constexpr int DV = 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1116,8 +1136,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   float* sc_coef = scf + 1536;   // state-update coefficient
   float* sc_n = scf + 1792;      // [2 halves][64] partial ||k_t||^2 of one chunk
   float* sc_gC = scf + 1920;     // [4] gamma of the whole chunk
-  float* sc_pcar = scf + 1924;   // carried variance
-  volatile float* sc_abort = scf + 1925;
+  volatile float* sc_abort = scf + 1924;
+  float* sc_pcar = scf + 1928;   // carried variance (diagonal: [128])
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P::OFF_BAR);
   uint64_t* full_kq = bars;        // [kStages] K/Q tiles of a stage landed
   uint64_t* full_v = bars + 3;     // V tile landed
@@ -1128,6 +1148,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* mma5_bar = bars + 8;   // MMA5 finished: state updated, stage free
   uint64_t* t_ready = bars + 9;    // T written
   uint64_t* p_ready = bars + 10;   // P and the next chunk's scalars written
+  uint64_t* w_full = bars + 11;    // [2] (diagonal) a w buffer landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   float* sOut = reinterpret_cast<float*>(smem + P::OFF_OUT);
   float* AT = reinterpret_cast<float*>(smem + P::OFF_AT);
@@ -1135,13 +1156,15 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* sT = smem + P::OFF_T;
   uint8_t* sP = smem + P::OFF_P;
   uint8_t* sV = smem + P::OFF_V;
+  const float* sW = reinterpret_cast<const float*>(smem + P::OFF_W);
 
   if (tid == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 13; ++i) mbar_init(&bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     *sc_abort = 0.f;
-    sc_pcar[0] = P0 ? P0[bh] : 1.f;
+    if (!DIAG) sc_pcar[0] = P0 ? P0[bh] : 1.f;
   }
+  if (DIAG && tid < kDK) sc_pcar[tid] = P0 ? P0[(size_t)bh * kDK + tid] : 1.f;
   // T operand (hi, lo): blocks above the diagonal are never written again
   for (int i = tid; i < 1024; i += kThreads)
     *reinterpret_cast<uint4*>(sT + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
@@ -1182,7 +1205,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       const size_t tok = ((size_t)b * T + t0 + t) * H + h;
       ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
       ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
-      ps_w[i] = in ? __ldg(Wg + tok) : 0.f;
+      ps_w[i] = (!DIAG && in) ? __ldg(Wg + tok) : 0.f;
     }
   };
   auto store_scalars = [&](int c) {
@@ -1232,6 +1255,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     sc_gam[64 * sl + ta] = exp2f(lg0);
     sc_gam[64 * sl + tb] = exp2f(lg1);
     if (lane == 31) sc_gC[sl] = exp2f(lg1);
+    if constexpr (DIAG) return;  // beta and the coefficients come from D1
     const float n0 = sc_n[ta] + sc_n[64 + ta], n1 = sc_n[tb] + sc_n[64 + tb];
     const float w0 = w_s[ta], w1 = w_s[tb], r0 = r_s[ta], r1 = r_s[tb];
     const float c0 = kappa * n0, c1 = kappa * n1;
@@ -1268,11 +1292,13 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
     if (lane == 0) sc_pcar[0] = pnext;
   };
-
   const bool issuer = (warp == 0 && lane == 0);       // chain: MMAs and copies
   const bool mma1_issuer = (warp == 15 && lane == 0);  // prep: MMA1
   constexpr uint32_t ID_1 = umma_idesc(128, 64, 1, 0, 0);
-  int pend_kq[P::kStages] = {-1, -1, -1}, pend_v = -1, pend_mma1 = -1;  // (issuers) not yet seen done
+  // (issuers) copies and MMAs not yet seen done: pend_kq holds per stage a
+  // pending bit (2 st) and the parity to wait for (2 st + 1)
+  uint32_t pend_kq = 0u;
+  int pend_v = -1, pend_mma1 = -1;
   auto kq_parity = [](int c) { return (uint32_t)((c / P::kStages) & 1); };
   auto issue_kq = [&](int c) {
     const int st = c % P::kStages, t0 = c * kC;
@@ -1282,7 +1308,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, t0, b);
       tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, t0, b);
     }
-    pend_kq[st] = (int)kq_parity(c);
+    pend_kq = (pend_kq & ~(3u << (2 * st))) | ((1u | (kq_parity(c) << 1)) << (2 * st));
   };
   auto issue_v = [&](int c) {
     mbar_expect_tx(full_v, 16384);
@@ -1290,24 +1316,107 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
     pend_v = c & 1;
   };
-  // D1 = [K;Q] K^T of chunk c (A: the stage's key rows then query rows per d block)
+  // (diagonal) w quarter n: tokens [16 n, 16 n + 16) of the sequence
+  uint32_t pend_w = 0u;  // per buffer: pending bit (2 i) and parity (2 i + 1)
+  auto issue_w = [&](int n) {
+    const int bf = n & 1;
+    mbar_expect_tx(&w_full[bf], 8192);
+    tma_load_4d(smem + P::OFF_W + bf * 8192, &tm_w, &w_full[bf], 0, h, 16 * n, b);
+    pend_w = (pend_w & ~(3u << (2 * bf))) | ((1u | ((uint32_t)((n >> 1) & 1) << 1)) << (2 * bf));
+  };
+  // D1 = [K;Q] K^T of chunk c (A: the stage's key rows then query rows per d
+  // block); diagonal: D1 = [K;Q] G~^T (G~ hi, then lo)
   auto issue_mma1 = [&](int c) {
     const uint32_t kq_a = sbase + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES;
     tc_fence_after();
     const uint64_t d0 = umma_desc_sw128(kq_a, 16, 1024);
+    if constexpr (DIAG) {
+      const uint64_t g0 = umma_desc_sw128(sbase + P::OFF_G + (c & 1) * 32768u, 16, 1024);
 #pragma unroll
-    for (int kb = 0; kb < 2; ++kb)
+      for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-        const uint64_t d = d0 + (uint64_t)((kb * 16384 + ks * 32) >> 4);
-        umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
-      }
+        for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            umma_bf16(tmem + P::COL_D1, d0 + (uint64_t)((kb * 16384 + ks * 32) >> 4),
+                      g0 + (uint64_t)((hl * 16384 + kb * 8192 + ks * 32) >> 4), ID_1,
+                      (hl > 0 || kb > 0 || ks > 0) ? 1u : 0u);
+    } else {
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t d = d0 + (uint64_t)((kb * 16384 + ks * 32) >> 4);
+          umma_bf16(tmem + P::COL_D1, d, d, ID_1, (kb > 0 || ks > 0) ? 1u : 0u);
+        }
+    }
     umma_commit(mma1_bar);
     pend_mma1 = c & 1;
   };
 
-  // ---- prologue: copies, chunk 0's scalars and MMA1
   bool bad = false;
+  // diagonal: the variance of dimension d over chunk c (one thread per d,
+  // tokens in order), p^- = a^2 p + w, p = r p^- / (k^2 p^- + r), with the
+  // gain direction G~ = p^- k of each token kept in the free D1 columns (TMEM
+  // lane d) until its smem buffer is released (write_gain). w arrives in
+  // quarters of 16 tokens (quarter n = 4 c + q in buffer n & 1); the whole
+  // team takes part (four team barriers), the w copies are issued by one thread.
+  auto diag_variance = [&](int c, int d) {
+    const int sl = c & 3;
+    const float* a_s = sc_a + 64 * sl;
+    const float* r_s = sc_r + 64 * sl;
+    const uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + (d >> 6) * 16384;
+    const uint32_t col = (uint32_t)(d & 63);
+    float p = sc_pcar[d];
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+      const int n = 4 * c + q;
+      if (fail(&w_full[n & 1], (uint32_t)((n >> 1) & 1))) bad = true;
+      if (!bad) {
+        const float* wq = sW + (n & 1) * 2048 + d;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const float4 a4 = *reinterpret_cast<const float4*>(a_s + 16 * q + 4 * i4);
+          const float4 r4 = *reinterpret_cast<const float4*>(r_s + 16 * q + 4 * i4);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w}, rv[4] = {r4.x, r4.y, r4.z, r4.w};
+          uint32_t g[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float k = ld_bf16(kt, (uint32_t)(16 * q + 4 * i4 + e), col);
+            const float pp = fmaf(av[e] * av[e], p, wq[(4 * i4 + e) * kDK]);
+            g[e] = __float_as_uint(pp * k);
+            p = __fdividef(rv[e] * pp, fmaf(k * k, pp, rv[e]));
+          }
+          tmem_st4u(tmem + tm_lane + P::COL_D1 + 16 * q + 4 * i4, g);
+        }
+      }
+      named_bar<kTeamB, 128>();  // buffer n & 1 has been read
+      if (mma1_issuer && !bad && n + 2 < 4 * nchunks) issue_w(n + 2);
+    }
+    sc_pcar[d] = p;
+    tmem_wait_st();
+  };
+  // G~ of chunk c from TMEM into its buffer c & 1 as bf16 hi/lo [kb][t][k]
+  auto write_gain = [&](int c, int d) {
+    uint8_t* gh = smem + P::OFF_G + (c & 1) * 32768 + (d >> 6) * 8192;
+    const uint32_t col = (uint32_t)(d & 63);
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+      float g[16];
+      tmem_ld16(tmem + tm_lane + P::COL_D1 + 16 * blk, g);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const __nv_bfloat16 g_hi = __float2bfloat16_rn(g[i]);
+        const __nv_bfloat16 g_lo = __float2bfloat16_rn(g[i] - __bfloat162float(g_hi));
+        const uint32_t off = sw128_offset((uint32_t)(16 * blk + i), col);
+        *reinterpret_cast<__nv_bfloat16*>(gh + off) = g_hi;
+        *reinterpret_cast<__nv_bfloat16*>(gh + 16384 + off) = g_lo;
+      }
+    }
+  };
+
+  // ---- prologue: copies, chunk 0's scalars and MMA1
   if (issuer) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -1318,17 +1427,34 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int c = 1; c < P::kStages && c < nchunks; ++c) issue_kq(c);
   }
   if (warp >= 8) {
+    if (DIAG && mma1_issuer) {
+      issue_w(0);
+      issue_w(1);
+    }
     if (warp == 13) {
       fetch_scalars(0);
       store_scalars(0);
       if (nchunks > 1) fetch_scalars(1);
     }
     if (fail(&full_kq[0], kq_parity(0))) bad = true;
-    if (mma1_issuer && !bad) issue_mma1(0);
-    if (warp >= 12) {
-      key_norms(0, tid - 384);
-      named_bar<kTeamB, 128>();
-      if (warp == 12) decay_and_variance(0);
+    if constexpr (DIAG) {
+      if (warp >= 12) {
+        named_bar<kTeamB, 128>();  // chunk 0's scalars
+        diag_variance(0, tid - 384);
+        if (!bad) write_gain(0, tid - 384);
+        if (warp == 12) decay_and_variance(0);
+        fence_async_smem();
+        tc_fence_before();
+        named_bar<kTeamB, 128>();
+        if (mma1_issuer && !bad) issue_mma1(0);
+      }
+    } else {
+      if (mma1_issuer && !bad) issue_mma1(0);
+      if (warp >= 12) {
+        key_norms(0, tid - 384);
+        named_bar<kTeamB, 128>();
+        if (warp == 12) decay_and_variance(0);
+      }
     }
   }
   __syncthreads();  // chunk 0's scalars are in place
@@ -1345,18 +1471,17 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     // S'^T [v][k], k in [64 ch, 64 ch + 64), as the bf16 hi/lo A operand of
     // MMA2 in W: k pairs per column, hi then lo
     auto split_state = [&]() {
-      uint32_t hi[32], lo[32];
 #pragma unroll
       for (int h32 = 0; h32 < 2; ++h32) {
         float x[32];
+        uint32_t hi[16], lo[16];
         tmem_ld32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, x);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          split_pack2(x[2 * i], x[2 * i + 1], hi[16 * h32 + i], lo[16 * h32 + i]);
+        for (int i = 0; i < 16; ++i) split_pack2(x[2 * i], x[2 * i + 1], hi[i], lo[i]);
+        tmem_st16u(tmem + tm_lane + P::COL_W + 32 * ch + 16 * h32, hi);
+        tmem_st16u(tmem + tm_lane + P::COL_W + 64 + 32 * ch + 16 * h32, lo);
       }
-      tmem_st32(tmem + tm_lane + P::COL_W + 32 * ch, hi);
-      tmem_st32(tmem + tm_lane + P::COL_W + 64 + 32 * ch, lo);
     };
 
     // S'^T [v][k] into TMEM, k in [64 ch, 64 ch + 64)
@@ -1390,7 +1515,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       // then query rows per d block, K-major)
       if (issuer) {
         if (fail(&full_kq[s], kq_parity(c))) bad = true;
-        else pend_kq[s] = -1;
+        else pend_kq &= ~(3u << (2 * s));
       }
       if (issuer && !bad) {
         tc_fence_after();
@@ -1452,6 +1577,9 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
       if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
+      // diagonal: stage s is free once MMA1 and the variance of chunk c (both
+      // before t_ready) and MMA2 have read it; MMA5 reads G~ instead of K
+      if (DIAG && issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);
       if (issuer && !bad) {
         tc_fence_after();
         const uint64_t dt = umma_desc_sw128(sbase + P::OFF_T, 16, 1024);
@@ -1514,7 +1642,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);  // Z has been read
         tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);
       }
-      if (issuer) bulk_wait_read_all();  // the previous output tile has been read
+      if (!DIAG && issuer) bulk_wait_read_all();  // the previous output tile has been read
       tmem_wait_st();
       tc_fence_before();
       bar_group(kChainBar);
@@ -1523,14 +1651,26 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (fail(p_ready, (uint32_t)(c & 1))) bad = true;
       if (issuer && !bad) {
         tc_fence_after();
-        // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
-        const uint64_t dk = umma_desc_sw128(kq_a, 16384, 1024);
+        if constexpr (DIAG) {
+          // state += B^T G~: Bhi G~hi + Blo G~hi + Bhi G~lo (G~ [t][k] MN-major:
+          // k blocks 8 KB apart, token groups 1024 B)
+          const uint64_t dg = umma_desc_sw128(sbase + P::OFF_G + (c & 1) * 32768u, 8192, 1024);
 #pragma unroll
-        for (int hl = 0; hl < 2; ++hl)
+          for (int term = 0; term < 3; ++term)
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_W + 32 * hl + 8 * ks,
-                         dk + (uint64_t)((ks * 2048) >> 4), ID_5, 1u);
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_W + (term == 1 ? 32 : 0) + 8 * ks,
+                           dg + (uint64_t)(((term == 2 ? 16384 : 0) + ks * 2048) >> 4), ID_5, 1u);
+        } else {
+          // B = K [t][k] MN-major: k blocks 16 KB apart, token groups 1024 B
+          const uint64_t dk = umma_desc_sw128(kq_a, 16384, 1024);
+#pragma unroll
+          for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              umma_bf16_ts(tmem + P::COL_ST, tmem + P::COL_W + 32 * hl + 8 * ks,
+                           dk + (uint64_t)((ks * 2048) >> 4), ID_5, 1u);
+        }
         umma_commit(mma5_bar);
         pend_mma5 = c & 1;
         const uint64_t dp = umma_desc_sw128(sbase + P::OFF_P, 16, 1024);
@@ -1550,25 +1690,36 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (fail(mma4_bar, (uint32_t)(c & 1))) bad = true;
       else if (issuer) pend_mma4 = -1;
       tc_fence_after();
-      // (into the staging tile [t][v]; one bulk tensor store per chunk writes
-      // it, rows past T excluded)
-      {
+      // (isotropic: into the staging tile [t][v]; one bulk tensor store per
+      // chunk writes it, rows past T excluded. diagonal: straight to memory,
+      // each warp writing 128 contiguous bytes per token)
+      if constexpr (DIAG) {
+        float x[32];
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
+        tmem_wait_ld();
+        const int valid = min(kC, T - t0);
+        float* dst = O + (((size_t)b * T + t0 + 32 * ch) * H + h) * DV + v;
+        const size_t ostride = (size_t)H * DV;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (32 * ch + i < valid) dst[i * ostride] = x[i];
+      } else {
         float x[32];
         tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
         tmem_wait_ld();
         float* dst = sOut + (32 * ch) * DV + v;
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * DV] = x[i];
+        fence_async_smem();
+        if (issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);  // stage s is free
       }
-      fence_async_smem();
-      if (issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);  // stage s is free
       tmem_wait_st();
       tc_fence_before();
       if (bar_group_or(kChainBar, bad || *sc_abort != 0.f)) {
         bad = true;
         break;
       }
-      if (issuer) {
+      if (!DIAG && issuer) {
         tma_store_4d(&tm_o, sOut, 0, h, t0, b);
         bulk_commit();
       }
@@ -1580,9 +1731,9 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (pend_mma4 >= 0) (void)mbar_wait(mma4_bar, (uint32_t)pend_mma4);
       if (pend_mma5 >= 0) (void)mbar_wait(mma5_bar, (uint32_t)pend_mma5);
       for (int st = 0; st < P::kStages; ++st)
-        if (pend_kq[st] >= 0) (void)mbar_wait(&full_kq[st], (uint32_t)pend_kq[st]);
+        if ((pend_kq >> (2 * st)) & 1u) (void)mbar_wait(&full_kq[st], (pend_kq >> (2 * st + 1)) & 1u);
       if (pend_v >= 0) (void)mbar_wait(full_v, (uint32_t)pend_v);
-      bulk_wait_all();  // output stores complete
+      if (!DIAG) bulk_wait_all();  // output stores complete
     }
     if (!bad) {
       tc_fence_after();
@@ -1617,6 +1768,19 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         float d1[32];
         tmem_ld32(tmem + tm_lane + P::COL_D1 + 32 * pch, d1);
         tmem_wait_ld();
+        if constexpr (DIAG) {
+          // beta_t = 1 / (k_t . G~_t + r_t) from the diagonal of D1, then the
+          // state-update coefficients
+          if (!qrow && (tk >> 5) == pch) {
+            float dd = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) dd = (i == (tk & 31)) ? d1[i] : dd;
+            sc_beta[64 * sl + tk] = 1.f / (dd + sc_r[64 * sl + tk]);
+          }
+          bar_group(kPrepBar);
+          if (ptid < 64)
+            sc_coef[64 * sl + ptid] = beta_c[ptid] * exp2f(lg_c[kC - 1] - lg_c[ptid]);
+        }
         const float lg_t = lg_c[tk];
         const int lim = tk + (qrow ? 1 : 0);  // A: j < t; P: j <= t
 #pragma unroll
@@ -1640,10 +1804,20 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int i4 = 0; i4 < 8; ++i4)
           *reinterpret_cast<float4*>(row + 4 * i4) =
               make_float4(preg[4 * i4], preg[4 * i4 + 1], preg[4 * i4 + 2], preg[4 * i4 + 3]);
+      } else {
+        // P as the tf32 B operand [t][j], once MMA4 of the previous chunk
+        // released the buffer
+        if (c > 0 && fail(mma4_bar, (uint32_t)((c - 1) & 1))) bad = true;
+        uint8_t* dst = sP + pch * 8192;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)tk, (uint32_t)q)) =
+              make_uint4(rna_tf32(preg[4 * q]), rna_tf32(preg[4 * q + 1]),
+                         rna_tf32(preg[4 * q + 2]), rna_tf32(preg[4 * q + 3]));
       }
       bar_group(kPrepBar);
-      // MMA1 of the next chunk: D1 has been read
-      if (mma1_issuer && !bad && c + 1 < nchunks) {
+      // MMA1 of the next chunk: D1 has been read (diagonal: once G~ is written)
+      if (!DIAG && mma1_issuer && !bad && c + 1 < nchunks) {
         if (fail(&full_kq[(c + 1) % P::kStages], kq_parity(c + 1))) bad = true;
         else issue_mma1(c + 1);
       }
@@ -1781,22 +1955,25 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (c + 2 < nchunks) fetch_scalars(c + 2);
         }
         if (fail(&full_kq[(c + 1) % P::kStages], kq_parity(c + 1))) bad = true;
-        key_norms(c + 1, ptid - 128);
-        named_bar<kTeamB, 128>();
-        if (warp == 12) decay_and_variance(c + 1);
+        if constexpr (DIAG) {
+          named_bar<kTeamB, 128>();  // the scalars of chunk c + 1
+          tc_fence_after();          // (D1 has been read)
+          diag_variance(c + 1, ptid - 128);
+          if (warp == 12) decay_and_variance(c + 1);
+          // G~ buffer (c + 1) & 1 is free once MMA5 of chunk c - 1 has read it
+          if (c > 0 && fail(mma5_bar, (uint32_t)((c - 1) & 1))) bad = true;
+          if (!bad) write_gain(c + 1, ptid - 128);
+          fence_async_smem();
+          tc_fence_before();
+          named_bar<kTeamB, 128>();
+          if (mma1_issuer && !bad) issue_mma1(c + 1);
+        } else {
+          key_norms(c + 1, ptid - 128);
+          named_bar<kTeamB, 128>();
+          if (warp == 12) decay_and_variance(c + 1);
+        }
       }
 
-      // ---- P as the tf32 B operand [t][j], once MMA4 of the previous chunk
-      // released the buffer
-      if (c > 0 && fail(mma4_bar, (uint32_t)((c - 1) & 1))) bad = true;
-      if (qrow) {
-        uint8_t* dst = sP + pch * 8192;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4*>(dst + chunk_off((uint32_t)tk, (uint32_t)q)) =
-              make_uint4(rna_tf32(preg[4 * q]), rna_tf32(preg[4 * q + 1]),
-                         rna_tf32(preg[4 * q + 2]), rna_tf32(preg[4 * q + 3]));
-      }
       fence_async_smem();
       if (bar_group_or(kPrepBar, bad || *sc_abort != 0.f)) {
         bad = true;
@@ -1805,7 +1982,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ptid == 0) mbar_arrive(p_ready);
     }
     if (mma1_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
-    if (ptid == 0 && !bad) P_out[bh] = sc_pcar[0];
+    if (DIAG && mma1_issuer)
+      for (int bf = 0; bf < 2; ++bf)
+        if ((pend_w >> (2 * bf)) & 1u) (void)mbar_wait(&w_full[bf], (pend_w >> (2 * bf + 1)) & 1u);
+    if constexpr (DIAG) {
+      if (ptid >= 128 && !bad) P_out[(size_t)bh * kDK + ptid - 128] = sc_pcar[ptid - 128];
+    } else {
+      if (ptid == 0 && !bad) P_out[bh] = sc_pcar[0];
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -1840,14 +2024,14 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int 
 }
 
 // [B, T, H, d] fp32 output, boxes of (d columns, 1 head, box_t tokens, 1 batch)
-bool make_out_map(CUtensorMap* m, void* base, int B, int T, int H, int d, int box_t) {
+bool make_out_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int box_t) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
   cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -1886,25 +2070,36 @@ kdn_status launch(const void* q, const void* k, const void* v, const float* a, c
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
+template <bool DIAG>
 kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a,
                      const float* w, const float* r, const float* S0, const float* p0, float* o,
                      float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
                      cudaStream_t s) {
-  using P = WsPlan;
-  CUtensorMap mq, mk, mv, mo;
+  using P = WsPlan<DIAG>;
+  CUtensorMap mq, mk, mv, mo, mw;
   if (!make_map(&mq, q, B, T, H, kDK, 64) || !make_map(&mk, k, B, T, H, kDK, 64) ||
-      !make_map(&mv, v, B, T, H, 128, 64) || !make_out_map(&mo, o, B, T, H, 128, 64))
+      !make_map(&mv, v, B, T, H, 128, 64))
     return KDN_ERR_CUDA;
+  // isotropic: the output tile map; diagonal: the output is written without a
+  // map, and w [B, T, H, 128] is read in boxes of 16 tokens
+  if (DIAG) {
+    mo = mq;
+    if (!make_out_map(&mw, w, B, T, H, kDK, 16)) return KDN_ERR_CUDA;
+  } else {
+    if (!make_out_map(&mo, o, B, T, H, 128, 64)) return KDN_ERR_CUDA;
+    mw = mq;
+  }
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(chunk_engine_ws_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             P::ALLOC) != cudaSuccess)
+    if (cudaFuncSetAttribute(chunk_engine_ws_kernel<DIAG>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, P::ALLOC) != cudaSuccess)
       return KDN_ERR_CUDA;
     attr_set = true;
   }
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
-  chunk_engine_ws_kernel<<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
-      mq, mk, mv, mo, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa, static_cast<uint32_t*>(ws));
+  chunk_engine_ws_kernel<DIAG><<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
+      mq, mk, mv, mo, mw, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa,
+      static_cast<uint32_t*>(ws));
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
@@ -1925,19 +2120,8 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                int T, int H, int dv, float kappa, void* ws, cudaStream_t s) {
   if (dv == 128) {
     // one CTA per head reads p0 and writes p_out: no snapshot needed
-    if (!diag) return launch_ws(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s);
-    // With few heads, one CTA per head leaves most SMs idle: split each head's
-    // value columns over two CTAs (each repeats the head's input-only work).
-    static int sms = 0;
-    if (sms == 0) {
-      int dev = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return KDN_ERR_CUDA;
-    }
-    if (2 * B * H <= sms)
-      return launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
-    return launch<true, 128>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+    return diag ? launch_ws<true>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s)
+                : launch_ws<false>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s);
   }
   return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
               : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);

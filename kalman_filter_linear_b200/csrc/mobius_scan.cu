@@ -77,6 +77,15 @@ __device__ __forceinline__ Mat2 shfl_up(const Mat2& x, int delta) {
           __shfl_up_sync(0xffffffffu, x.c, delta), __shfl_up_sync(0xffffffffu, x.d, delta)};
 }
 
+// (lane, tile index within the lane) of a tile.  Tiles number below 2^31
+// (checked on the host), so 32-bit division does.
+__device__ __forceinline__ void split_tile(int64_t tile, int64_t N, int64_t& j, int64_t& seq) {
+  const uint32_t t = (uint32_t)tile, n = (uint32_t)N;
+  const uint32_t q = t / n;
+  j = q;
+  seq = t - q * n;
+}
+
 struct ScanWs {
   uint32_t* error;    // device error word
   uint32_t* counter;  // next tile to hand out
@@ -105,11 +114,20 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int64_t j = tile / N;    // tile index within the lane
-  const int64_t seq = tile % N;  // lane
+  int64_t j, seq;  // tile index within the lane, lane
+  split_tile(tile, N, j, seq);
   const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
   const int64_t base = seq * T;
   Mat2* s_warp = sh.warp_incl;
+  // The predecessor's inclusive prefix is usually published already: ask for
+  // it now, so that the read overlaps this tile's local scan.
+  const int64_t pt0 = (j - 1) * N + seq;
+  uint32_t f_pre = 0u;
+  float4 incl_pre = make_float4(1.f, 0.f, 0.f, 1.f);
+  if (tid == 0 && j > 0) {
+    f_pre = ld_acquire_u32(ws.flag + pt0);
+    incl_pre = __ldcg(ws.incl + pt0);
+  }
 
   Mat2 P = identity();
 #pragma unroll
@@ -159,8 +177,7 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
       // Usually the predecessor has finished: take its inclusive prefix and
       // publish only this tile's.  Otherwise publish the aggregate first and
       // look back tile by tile.
-      const int64_t pt0 = (j - 1) * N + seq;
-      uint32_t f0 = ld_acquire_u32(ws.flag + pt0);
+      uint32_t f0 = f_pre;
       if (f0 != 2u) {
         if (!skip_publish) {
           ws.agg[tile] = as_f4(agg);
@@ -190,7 +207,7 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
         }
         if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
       } else {
-        excl = as_mat(__ldcg(ws.incl + pt0));
+        excl = as_mat(incl_pre);
       }
       if (!skip_publish) {
         ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
@@ -259,7 +276,8 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
   if (tid == 0) s_tile = atomicAdd(ws.counter, 1u);
   __syncthreads();
   const int64_t tile = s_tile;
-  const int64_t j = tile / N, seq = tile % N;
+  int64_t j, seq;
+  split_tile(tile, N, j, seq);
   const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
   const int64_t base = seq * T;
   float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
@@ -316,7 +334,8 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
   // copies the inputs of `tile` into the buffer (thread 0)
   auto fetch = [&](int64_t tile) {
     const float* src[4] = {A, W, R, Nsq};
-    const int64_t j = tile / N, seq = tile % N;
+    int64_t j, seq;
+    split_tile(tile, N, j, seq);
     const int64_t first = j * kTile;
     const uint32_t bytes = (uint32_t)(min((int64_t)kTile, T - first) * 4);
     mbar_expect_tx(&s_full, 4u * bytes);
@@ -347,7 +366,8 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
       if (tid == 0) atomicOr(ws.error, DEV_TIMEOUT);
       break;
     }
-    const int64_t j = tile / N;
+    int64_t j, seq;
+    split_tile(tile, N, j, seq);
     const int64_t t0 = j * kTile + (int64_t)tid * kPerThread;
     const float* buf = reinterpret_cast<const float*>(s_in);
     float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];

@@ -965,7 +965,8 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 //   isotropic  ||k||^2, decay prefix and the variance scan; MMA1 of the next
 //              chunk is issued as soon as D1 is read.
 //   diagonal   decay prefix and the per-dimension variance (one thread per
-//              dimension, w copied in 16-token quarters), whose G~ = p^- k is
+//              dimension; each warp copies w of its 32 dimensions in 16-token
+//              quarters, two ahead), whose G~ = p^- k (as bf16 hi/lo) is
 //              parked in the free D1 columns until MMA5 of chunk c - 1 has
 //              released the G~ buffer it goes to (two buffers); then MMA1 of
 //              the next chunk, D1 = [K;Q] G~^T.  beta_t = 1 / (k_t.G~_t + r_t)
@@ -994,7 +995,8 @@ struct WsPlan {
   // bf16 hi then lo [kb 2][64 t][64 k]
   static constexpr uint32_t OFF_OUT = OFF_SC + 9216u;
   static constexpr uint32_t OFF_G = OFF_OUT;
-  // diagonal: w of 16 tokens, fp32 [16 t][128 k], two buffers
+  // diagonal: w of 16 tokens, per warp of the variance team two buffers of
+  // fp32 [16 t][32 k] (its 32 dimensions)
   static constexpr uint32_t OFF_W = OFF_G + 65536u;
   static constexpr uint32_t OFF_BAR = DIAG ? OFF_W + 16384u : OFF_OUT + 32768u;
   static constexpr uint32_t TOTAL = OFF_BAR + 256u;
@@ -1148,8 +1150,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint64_t* mma5_bar = bars + 8;   // MMA5 finished: state updated, stage free
   uint64_t* t_ready = bars + 9;    // T written
   uint64_t* p_ready = bars + 10;   // P and the next chunk's scalars written
-  uint64_t* w_full = bars + 11;    // [2] (diagonal) a w buffer landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* w_full = bars + 11;    // [4 warps][2] (diagonal) a w buffer landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   float* sOut = reinterpret_cast<float*>(smem + P::OFF_OUT);
   float* AT = reinterpret_cast<float*>(smem + P::OFF_AT);
   float* X = reinterpret_cast<float*>(smem + P::OFF_X);
@@ -1159,7 +1161,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   const float* sW = reinterpret_cast<const float*>(smem + P::OFF_W);
 
   if (tid == 0) {
-    for (int i = 0; i < 13; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 19; ++i) mbar_init(&bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     *sc_abort = 0.f;
     if (!DIAG) sc_pcar[0] = P0 ? P0[bh] : 1.f;
@@ -1316,12 +1318,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
     pend_v = c & 1;
   };
-  // (diagonal) w quarter n: tokens [16 n, 16 n + 16) of the sequence
+  // (diagonal) w quarter n: tokens [16 n, 16 n + 16) of the sequence, for the
+  // 32 dimensions of variance warp wv (its lane 0 issues them)
   uint32_t pend_w = 0u;  // per buffer: pending bit (2 i) and parity (2 i + 1)
-  auto issue_w = [&](int n) {
+  auto issue_w = [&](int n, int wv) {
     const int bf = n & 1;
-    mbar_expect_tx(&w_full[bf], 8192);
-    tma_load_4d(smem + P::OFF_W + bf * 8192, &tm_w, &w_full[bf], 0, h, 16 * n, b);
+    uint64_t* bar_ = &w_full[2 * wv + bf];
+    mbar_expect_tx(bar_, 2048);
+    tma_load_4d(smem + P::OFF_W + (2 * wv + bf) * 2048, &tm_w, bar_, 32 * wv, h, 16 * n, b);
     pend_w = (pend_w & ~(3u << (2 * bf))) | ((1u | ((uint32_t)((n >> 1) & 1) << 1)) << (2 * bf));
   };
   // D1 = [K;Q] K^T of chunk c (A: the stage's key rows then query rows per d
@@ -1357,23 +1361,29 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   bool bad = false;
   // diagonal: the variance of dimension d over chunk c (one thread per d,
   // tokens in order), p^- = a^2 p + w, p = r p^- / (k^2 p^- + r), with the
-  // gain direction G~ = p^- k of each token kept in the free D1 columns (TMEM
-  // lane d) until its smem buffer is released (write_gain). w arrives in
-  // quarters of 16 tokens (quarter n = 4 c + q in buffer n & 1); the whole
-  // team takes part (four team barriers), the w copies are issued by one thread.
+  // gain direction G~ = p^- k of each token (as a bf16 hi/lo pair) kept in the
+  // free D1 columns (TMEM lane d) until its smem buffer is released
+  // (write_gain).  w arrives in quarters of 16 tokens: quarter n = 4 c + q of
+  // this warp's 32 dimensions in its buffer n & 1, copied two quarters ahead
+  // by the warp's lane 0.
   auto diag_variance = [&](int c, int d) {
     const int sl = c & 3;
     const float* a_s = sc_a + 64 * sl;
     const float* r_s = sc_r + 64 * sl;
     const uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + (d >> 6) * 16384;
     const uint32_t col = (uint32_t)(d & 63);
-    float p = sc_pcar[d];
+    // p = x / y, carried projectively so that no division sits on the
+    // token-to-token chain: with u = a^2 x + w y (= p^- y), one token maps
+    // (x, y) to (r u, k^2 u + r y), the Mobius map's matrix applied to the
+    // pair; p^- k = u k / y is a division off the chain.  (x, y) is rescaled
+    // by the binade of y (exact) every four tokens.
+    float x = sc_pcar[d], y = 1.f;
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
       const int n = 4 * c + q;
-      if (fail(&w_full[n & 1], (uint32_t)((n >> 1) & 1))) bad = true;
+      if (fail(&w_full[2 * (d >> 5) + (n & 1)], (uint32_t)((n >> 1) & 1))) bad = true;
       if (!bad) {
-        const float* wq = sW + (n & 1) * 2048 + d;
+        const float* wq = sW + (2 * (d >> 5) + (n & 1)) * 512 + (d & 31);
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) {
           const float4 a4 = *reinterpret_cast<const float4*>(a_s + 16 * q + 4 * i4);
@@ -1383,20 +1393,33 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float k = ld_bf16(kt, (uint32_t)(16 * q + 4 * i4 + e), col);
-            const float pp = fmaf(av[e] * av[e], p, wq[(4 * i4 + e) * kDK]);
-            g[e] = __float_as_uint(pp * k);
-            p = __fdividef(rv[e] * pp, fmaf(k * k, pp, rv[e]));
+            const float u = fmaf(av[e] * av[e], x, wq[(4 * i4 + e) * 32] * y);
+            // G~ = p^- k as bf16 hi (low half) and lo (high half)
+            const float gf = __fdividef(u * k, y);
+            const __nv_bfloat16 g_hi = __float2bfloat16_rn(gf);
+            const __nv_bfloat16 g_lo = __float2bfloat16_rn(gf - __bfloat162float(g_hi));
+            g[e] = (uint32_t)__bfloat16_as_ushort(g_hi) |
+                   ((uint32_t)__bfloat16_as_ushort(g_lo) << 16);
+            x = rv[e] * u;
+            y = fmaf(k * k, u, rv[e] * y);
           }
           tmem_st4u(tmem + tm_lane + P::COL_D1 + 16 * q + 4 * i4, g);
+          const int ex = (int)((__float_as_uint(y) >> 23) & 0xffu) - 127;
+          if (ex > -100 && ex < 100) {
+            const float sc = __uint_as_float((uint32_t)(127 - ex) << 23);
+            x *= sc;
+            y *= sc;
+          }
         }
       }
-      named_bar<kTeamB, 128>();  // buffer n & 1 has been read
-      if (mma1_issuer && !bad && n + 2 < 4 * nchunks) issue_w(n + 2);
+      __syncwarp();  // this warp's buffer n & 1 has been read
+      if (lane == 0 && !bad && n + 2 < 4 * nchunks) issue_w(n + 2, d >> 5);
     }
-    sc_pcar[d] = p;
+    sc_pcar[d] = x / y;
     tmem_wait_st();
   };
-  // G~ of chunk c from TMEM into its buffer c & 1 as bf16 hi/lo [kb][t][k]
+  // G~ of chunk c (bf16 hi/lo pairs) from TMEM into its buffer c & 1 as
+  // [hi|lo][kb][t][k]
   auto write_gain = [&](int c, int d) {
     uint8_t* gh = smem + P::OFF_G + (c & 1) * 32768 + (d >> 6) * 8192;
     const uint32_t col = (uint32_t)(d & 63);
@@ -1407,11 +1430,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const __nv_bfloat16 g_hi = __float2bfloat16_rn(g[i]);
-        const __nv_bfloat16 g_lo = __float2bfloat16_rn(g[i] - __bfloat162float(g_hi));
+        const uint32_t hl = __float_as_uint(g[i]);
         const uint32_t off = sw128_offset((uint32_t)(16 * blk + i), col);
-        *reinterpret_cast<__nv_bfloat16*>(gh + off) = g_hi;
-        *reinterpret_cast<__nv_bfloat16*>(gh + 16384 + off) = g_lo;
+        *reinterpret_cast<uint16_t*>(gh + off) = (uint16_t)(hl & 0xffffu);
+        *reinterpret_cast<uint16_t*>(gh + 16384 + off) = (uint16_t)(hl >> 16);
       }
     }
   };
@@ -1427,9 +1449,9 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int c = 1; c < P::kStages && c < nchunks; ++c) issue_kq(c);
   }
   if (warp >= 8) {
-    if (DIAG && mma1_issuer) {
-      issue_w(0);
-      issue_w(1);
+    if (DIAG && warp >= 12 && lane == 0) {
+      issue_w(0, warp - 12);
+      issue_w(1, warp - 12);
     }
     if (warp == 13) {
       fetch_scalars(0);
@@ -1982,9 +2004,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (ptid == 0) mbar_arrive(p_ready);
     }
     if (mma1_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);
-    if (DIAG && mma1_issuer)
+    if (DIAG && warp >= 12 && lane == 0)
       for (int bf = 0; bf < 2; ++bf)
-        if ((pend_w >> (2 * bf)) & 1u) (void)mbar_wait(&w_full[bf], (pend_w >> (2 * bf + 1)) & 1u);
+        if ((pend_w >> (2 * bf)) & 1u)
+          (void)mbar_wait(&w_full[2 * (warp - 12) + bf], (pend_w >> (2 * bf + 1)) & 1u);
     if constexpr (DIAG) {
       if (ptid >= 128 && !bad) P_out[(size_t)bh * kDK + ptid - 128] = sc_pcar[ptid - 128];
     } else {
@@ -2023,13 +2046,15 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [B, T, H, d] fp32 output, boxes of (d columns, 1 head, box_t tokens, 1 batch)
-bool make_out_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int box_t) {
+// [B, T, H, d] fp32 tensor, boxes of (box_d columns (default d), 1 head, box_t
+// tokens, 1 batch)
+bool make_out_map(CUtensorMap* m, const void* base, int B, int T, int H, int d, int box_t,
+                  int box_d = 0) {
   auto enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
-  cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_t, 1};
+  cuuint32_t box[4] = {(cuuint32_t)(box_d > 0 ? box_d : d), 1, (cuuint32_t)box_t, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -2084,7 +2109,7 @@ kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a
   // map, and w [B, T, H, 128] is read in boxes of 16 tokens
   if (DIAG) {
     mo = mq;
-    if (!make_out_map(&mw, w, B, T, H, kDK, 16)) return KDN_ERR_CUDA;
+    if (!make_out_map(&mw, w, B, T, H, kDK, 16, 32)) return KDN_ERR_CUDA;
   } else {
     if (!make_out_map(&mo, o, B, T, H, 128, 64)) return KDN_ERR_CUDA;
     mw = mq;

@@ -1782,7 +1782,6 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       // ---- D1 epilogue: A (key rows) into AT; P (query rows) kept
       if (fail(mma1_bar, (uint32_t)(c & 1))) bad = true;
       else if (mma1_issuer) pend_mma1 = -1;
-      __syncwarp();  // the TMEM load below is warp-collective
       tc_fence_after();
       const float* lg_c = sc_lg + 64 * sl;
       const float* beta_c = sc_beta + 64 * sl;

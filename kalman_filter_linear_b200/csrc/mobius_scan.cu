@@ -151,6 +151,9 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
   }
   if (lane == 31) s_warp[warp] = incl;
   __syncthreads();
+  // ---- block scan of the warp totals and 3. the decoupled look-back, both
+  // in warp 0 (the other warps wait at the next barrier).  The release store
+  // of a flag orders this thread's earlier stores of the prefix data before it.
   if (warp == 0) {
     Mat2 x = lane < kThreads / 32 ? s_warp[lane] : identity();
 #pragma unroll
@@ -159,62 +162,62 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
       if (lane >= d) x = renorm(mul(x, prev));
     }
     if (lane < kThreads / 32) s_warp[lane] = x;  // inclusive over warps
-  }
-  __syncthreads();
-
-  // ---- 3. decoupled look-back (thread 0).  The release store of a flag
-  // orders this thread's earlier stores of the prefix data before it.
-  if (tid == 0) {
-    const Mat2 agg = s_warp[kThreads / 32 - 1];
-    Mat2 excl = identity();
-    const bool skip_publish = (tile == debug_skip_tile);  // fault-injection hook
-    if (j == 0) {
-      if (!skip_publish) {
-        ws.incl[tile] = as_f4(agg);
-        st_release_u32(ws.flag + tile, 2u);
-      }
-    } else {
-      // Usually the predecessor has finished: take its inclusive prefix and
-      // publish only this tile's.  Otherwise publish the aggregate first and
-      // look back tile by tile.
-      uint32_t f0 = f_pre;
-      if (f0 != 2u) {
+    const Mat2 tot = {__shfl_sync(0xffffffffu, x.a, kThreads / 32 - 1),
+                      __shfl_sync(0xffffffffu, x.b, kThreads / 32 - 1),
+                      __shfl_sync(0xffffffffu, x.c, kThreads / 32 - 1),
+                      __shfl_sync(0xffffffffu, x.d, kThreads / 32 - 1)};
+    if (tid == 0) {
+      const Mat2 agg = tot;
+      Mat2 excl = identity();
+      const bool skip_publish = (tile == debug_skip_tile);  // fault-injection hook
+      if (j == 0) {
         if (!skip_publish) {
-          ws.agg[tile] = as_f4(agg);
-          st_release_u32(ws.flag + tile, 1u);
+          ws.incl[tile] = as_f4(agg);
+          st_release_u32(ws.flag + tile, 2u);
         }
-        const uint64_t start = globaltimer_ns();
-        bool timed_out = false;
-        for (int64_t p = j - 1; p >= 0 && !timed_out;) {
-          const int64_t pt = p * N + seq;
-          uint32_t f = (p == j - 1) ? f0 : ld_acquire_u32(ws.flag + pt);
-          while (f == 0u) {
-            if (globaltimer_ns() - start > kWaitLimitNs) {
-              timed_out = true;
+      } else {
+        // Usually the predecessor has finished: take its inclusive prefix and
+        // publish only this tile's.  Otherwise publish the aggregate first and
+        // look back tile by tile.
+        uint32_t f0 = f_pre;
+        if (f0 != 2u) {
+          if (!skip_publish) {
+            ws.agg[tile] = as_f4(agg);
+            st_release_u32(ws.flag + tile, 1u);
+          }
+          const uint64_t start = globaltimer_ns();
+          bool timed_out = false;
+          for (int64_t p = j - 1; p >= 0 && !timed_out;) {
+            const int64_t pt = p * N + seq;
+            uint32_t f = (p == j - 1) ? f0 : ld_acquire_u32(ws.flag + pt);
+            while (f == 0u) {
+              if (globaltimer_ns() - start > kWaitLimitNs) {
+                timed_out = true;
+                break;
+              }
+              __nanosleep(64);
+              f = ld_acquire_u32(ws.flag + pt);
+            }
+            if (timed_out) break;
+            if (f == 2u) {
+              excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
               break;
             }
-            __nanosleep(64);
-            f = ld_acquire_u32(ws.flag + pt);
+            excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
+            f0 = 0u;
+            --p;
           }
-          if (timed_out) break;
-          if (f == 2u) {
-            excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
-            break;
-          }
-          excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
-          f0 = 0u;
-          --p;
+          if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
+        } else {
+          excl = as_mat(incl_pre);
         }
-        if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
-      } else {
-        excl = as_mat(incl_pre);
+        if (!skip_publish) {
+          ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
+          st_release_u32(ws.flag + tile, 2u);
+        }
       }
-      if (!skip_publish) {
-        ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
-        st_release_u32(ws.flag + tile, 2u);
-      }
+      sh.tile_prefix = excl;
     }
-    sh.tile_prefix = excl;
   }
   __syncthreads();
 
@@ -398,7 +401,8 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
       }
     scan_tile(a, w, r, n, tile, lambda0, info_scale, lam_out, prior_out, gain_out, N, T, ws, 1,
               debug_skip_tile, sh);
-    __syncthreads();  // the shared tile state and s_tile are free
+    // (the next iteration's first barrier keeps the shared tile state until
+    // every thread is done with it)
   }
   // Nothing is in flight at exit: a copy is started only for a tile below
   // ntiles, which the next iteration waits for (or gives up on, after which

@@ -191,6 +191,46 @@ kdn_status kdn_diag_forward(const void* q, const void* k, const void* v,
                             size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_forward_host -- kdn_iso_forward / kdn_diag_forward (variant) with every
+ * tensor in host memory, for callers whose data is not on the device yet.
+ * The batch goes through the device in slices of slice_b entries (<= 0
+ * selects 1): a slice's inputs are copied in, the forward runs on them and
+ * its o, S_out and p_out are copied back, on two internal streams that
+ * alternate between slices, so that the copies of one slice overlap the
+ * copies of the next and the kernels.  Results equal those of the device
+ * calls on the same data.  The pages have no counterpart of this entry point.
+ *
+ * q, k, v, a, w, r, S0, p0, o, S_out, p_out  as in kdn_iso_forward /
+ *          kdn_diag_forward, but host pointers; pinned (page-locked) memory
+ *          is needed for the copies to overlap.  S0, p0 may be NULL.
+ * info_scale  iso only (as kdn_iso_forward); ignored for KDN_DIAG
+ * workspace   device scratch of >= kdn_forward_host_workspace_size(...)
+ *             bytes, 256-byte aligned: an error word, then two slots of
+ *             one slice's device buffers.  kdn_read_workspace_status() on it
+ *             reports a bounded wait that gave up in any slice.
+ * stream   the work is ordered after earlier work on `stream`, and later
+ *          work on `stream` waits for all of it; synchronise `stream` before
+ *          reading the outputs.  Calls on one device are enqueued one at a
+ *          time (an internal lock); the host buffers must stay valid until
+ *          `stream` has passed the call.
+ * Errors: as kdn_iso_forward.  All checks run before anything is enqueued;
+ * a KDN_ERR_CUDA from a runtime call part-way still leaves `stream` waiting
+ * for what was enqueued.
+ * ---------------------------------------------------------------------- */
+size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T,
+                                       int H, int dk, int dv,
+                                       kdn_dtype in_dtype, int chunk,
+                                       int slice_b);
+kdn_status kdn_forward_host(kdn_variant variant, const void* q, const void* k,
+                            const void* v, kdn_dtype in_dtype, const float* a,
+                            const float* w, const float* r, const float* S0,
+                            const float* p0, float* o, float* S_out,
+                            float* p_out, int B, int T, int H, int dk, int dv,
+                            float info_scale, int chunk, int slice_b,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_decode_step -- one recurrent decoding step for B x H heads, updating
  * the state in place (the constant-memory decoding of "Kalman Delta
  * Networks: Uncertainty-aware Associative Memory", abstract).  The same

@@ -1,7 +1,12 @@
 // extern "C" entry points of libkdn: argument checks, then kernel dispatch.
 // Every check runs before anything is enqueued; a call that returns an error
-// has enqueued nothing.
+// has enqueued nothing (kdn_forward_host: except for KDN_ERR_CUDA from a
+// runtime call part-way, after which the caller's stream still waits for
+// whatever was enqueued).
 #include <cstring>
+
+#include <algorithm>
+#include <mutex>
 
 #include "kdn_common.cuh"
 #include "../../include/kdn_testing.h"
@@ -83,6 +88,60 @@ kdn_status forward_common(bool diag, const void* q, const void* k, const void* v
                                   kappa, workspace, as_stream(stream));
 }
 
+// ------------------------------------------------------------ host buffers
+// kdn_forward_host runs the forward on batch slices whose inputs and outputs
+// live in pinned host memory.  Slice i uses device slot i & 1 and internal
+// stream i & 1, so the copies of one slice (in and out, PCIe is full duplex)
+// overlap those of the next and the kernels; a slot is reused only after the
+// earlier work on its own stream.
+
+__global__ void or_error_word(uint32_t* dst, const uint32_t* src) { atomicOr(dst, *src); }
+
+inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Offsets of one slice's device buffers (of nb batch entries) in a slot.
+struct HostSlot {
+  size_t q, k, v, a, w, r, s0, p0, o, s, p, fws, fws_bytes, bytes;
+};
+
+HostSlot host_slot(bool diag, int nb, int T, int H, int dk, int dv, size_t es, int chunk) {
+  HostSlot L{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t at = off;
+    off = up256(off + n);
+    return at;
+  };
+  const size_t tok = (size_t)nb * T * H;
+  const size_t pdim = diag ? (size_t)dk : 1;
+  L.q = take(tok * dk * es);
+  L.k = take(tok * dk * es);
+  L.v = take(tok * dv * es);
+  L.a = take(tok * 4);
+  L.w = take(tok * pdim * 4);
+  L.r = take(tok * 4);
+  L.s0 = take((size_t)nb * H * dv * dk * 4);
+  L.p0 = take((size_t)nb * H * pdim * 4);
+  L.o = take(tok * dv * 4);
+  L.s = take((size_t)nb * H * dv * dk * 4);
+  L.p = take((size_t)nb * H * pdim * 4);
+  L.fws_bytes = std::max<size_t>(256, kdn_forward_workspace_size(diag ? KDN_DIAG : KDN_ISO, nb, T,
+                                                                  H, dk, dv, chunk));
+  L.fws = take(L.fws_bytes);
+  L.bytes = off;
+  return L;
+}
+
+// Two streams and three events per device, created once.
+struct HostStreams {
+  cudaStream_t st[2];
+  cudaEvent_t start, done[2];
+};
+constexpr int kMaxHostDevices = 64;
+HostStreams g_host_streams[kMaxHostDevices];
+bool g_host_ready[kMaxHostDevices];
+std::mutex g_host_mu;  // also serialises the enqueue of concurrent calls
+
 }  // namespace
 
 extern "C" {
@@ -156,6 +215,114 @@ kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k, co
   const float kappa = info_scale > 0.f ? info_scale : 1.f / (float)dk;
   return kdn::recurrent_launch(variant == KDN_DIAG, in_dtype, q, k, v, a, w, r, S, p, o, S, p, B,
                                1, H, dk, dv, kappa, as_stream(stream));
+}
+
+size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,
+                                       kdn_dtype in_dtype, int chunk, int slice_b) {
+  if (B < 1 || T < 1 || H < 1 || !dims_supported(dk, dv)) return 0;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return 0;
+  const int nb = std::min(B, slice_b > 0 ? slice_b : 1);
+  const size_t es = in_dtype == KDN_BF16 ? 2 : 4;
+  return 256 + 2 * host_slot(variant == KDN_DIAG, nb, T, H, dk, dv, es, chunk).bytes;
+}
+
+kdn_status kdn_forward_host(kdn_variant variant, const void* q, const void* k, const void* v,
+                            kdn_dtype in_dtype, const float* a, const float* w, const float* r,
+                            const float* S0, const float* p0, float* o, float* S_out,
+                            float* p_out, int B, int T, int H, int dk, int dv, float info_scale,
+                            int chunk, int slice_b, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (variant != KDN_ISO && variant != KDN_DIAG) return KDN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !a || !w || !r || !o || !S_out || !p_out) return KDN_ERR_INVALID_ARG;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  if (!(info_scale == info_scale) || info_scale > 3.0e38f) return KDN_ERR_INVALID_ARG;
+  if (!dims_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
+  const int path = select_path(chunk, in_dtype, dk, dv);
+  if (path == -2) return KDN_ERR_INVALID_ARG;
+  if (path == -1) return KDN_ERR_UNSUPPORTED;
+  const bool diag = variant == KDN_DIAG;
+  const int nb = std::min(B, slice_b > 0 ? slice_b : 1);
+  const size_t es = in_dtype == KDN_BF16 ? 2 : 4;
+  const HostSlot L = host_slot(diag, nb, T, H, dk, dv, es, chunk);
+  if (!workspace || workspace_bytes < 256 + 2 * L.bytes) return KDN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDN_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxHostDevices)
+    return KDN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostStreams& hs = g_host_streams[dev];
+  if (!g_host_ready[dev]) {
+    if (cudaStreamCreateWithFlags(&hs.st[0], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hs.st[1], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hs.start, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hs.done[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hs.done[1], cudaEventDisableTiming) != cudaSuccess)
+      return KDN_ERR_CUDA;
+    g_host_ready[dev] = true;
+  }
+  cudaStream_t s0 = as_stream(stream);
+  char* base = static_cast<char*>(workspace);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  // the header error word and both slots' forward error words start clear
+  bool ok = cudaMemsetAsync(err, 0, 4, s0) == cudaSuccess;
+  for (int i = 0; i < 2 && ok; ++i)
+    ok = cudaMemsetAsync(base + 256 + i * L.bytes + L.fws, 0, 4, s0) == cudaSuccess;
+  ok = ok && cudaEventRecord(hs.start, s0) == cudaSuccess &&
+       cudaStreamWaitEvent(hs.st[0], hs.start, 0) == cudaSuccess &&
+       cudaStreamWaitEvent(hs.st[1], hs.start, 0) == cudaSuccess;
+  kdn_status status = ok ? KDN_OK : KDN_ERR_CUDA;
+  const size_t pdim = diag ? (size_t)dk : 1;
+  const auto H2D = cudaMemcpyHostToDevice;
+  const auto D2H = cudaMemcpyDeviceToHost;
+  for (int b0 = 0, i = 0; b0 < B && status == KDN_OK; b0 += nb, ++i) {
+    const int n = std::min(nb, B - b0);
+    cudaStream_t st = hs.st[i & 1];
+    char* sb = base + 256 + (size_t)(i & 1) * L.bytes;
+    const size_t tok0 = (size_t)b0 * T * H, tok = (size_t)n * T * H;
+    const size_t hd0 = (size_t)b0 * H, hd = (size_t)n * H;
+    auto cp = [&](size_t dst_off, const void* src, size_t off_bytes, size_t bytes,
+                  cudaMemcpyKind kind, bool to_dev) {
+      if (status != KDN_OK) return;
+      cudaError_t e = to_dev ? cudaMemcpyAsync(sb + dst_off, static_cast<const char*>(src) + off_bytes,
+                                               bytes, kind, st)
+                             : cudaMemcpyAsync(static_cast<char*>(const_cast<void*>(src)) + off_bytes,
+                                               sb + dst_off, bytes, kind, st);
+      if (e != cudaSuccess) status = KDN_ERR_CUDA;
+    };
+    cp(L.q, q, tok0 * dk * es, tok * dk * es, H2D, true);
+    cp(L.k, k, tok0 * dk * es, tok * dk * es, H2D, true);
+    cp(L.v, v, tok0 * dv * es, tok * dv * es, H2D, true);
+    cp(L.a, a, tok0 * 4, tok * 4, H2D, true);
+    cp(L.w, w, tok0 * pdim * 4, tok * pdim * 4, H2D, true);
+    cp(L.r, r, tok0 * 4, tok * 4, H2D, true);
+    if (S0) cp(L.s0, S0, hd0 * dv * dk * 4, hd * dv * dk * 4, H2D, true);
+    if (p0) cp(L.p0, p0, hd0 * pdim * 4, hd * pdim * 4, H2D, true);
+    if (status != KDN_OK) break;
+    const kdn_status fs = forward_common(
+        diag, sb + L.q, sb + L.k, sb + L.v, in_dtype, reinterpret_cast<float*>(sb + L.a),
+        reinterpret_cast<float*>(sb + L.w), reinterpret_cast<float*>(sb + L.r),
+        S0 ? reinterpret_cast<float*>(sb + L.s0) : nullptr,
+        p0 ? reinterpret_cast<float*>(sb + L.p0) : nullptr, reinterpret_cast<float*>(sb + L.o),
+        reinterpret_cast<float*>(sb + L.s), reinterpret_cast<float*>(sb + L.p), n, T, H, dk, dv,
+        diag ? 1.f : info_scale, chunk, sb + L.fws, L.fws_bytes, st);
+    if (fs != KDN_OK) {
+      status = fs;
+      break;
+    }
+    or_error_word<<<1, 1, 0, st>>>(err, reinterpret_cast<const uint32_t*>(sb + L.fws));
+    if (cudaGetLastError() != cudaSuccess) status = KDN_ERR_CUDA;
+    cp(L.o, o, tok0 * dv * 4, tok * dv * 4, D2H, false);
+    cp(L.s, S_out, hd0 * dv * dk * 4, hd * dv * dk * 4, D2H, false);
+    cp(L.p, p_out, hd0 * pdim * 4, hd * pdim * 4, D2H, false);
+  }
+  // the caller's stream waits for both internal streams, also after an error,
+  // so that no copy outlives the call's stream order
+  for (int j = 0; j < 2; ++j)
+    if (cudaEventRecord(hs.done[j], hs.st[j]) != cudaSuccess ||
+        cudaStreamWaitEvent(s0, hs.done[j], 0) != cudaSuccess)
+      status = KDN_ERR_CUDA;
+  return status;
 }
 
 kdn_status kdn_read_workspace_status(const void* workspace, size_t workspace_bytes,

@@ -1,9 +1,9 @@
 """Thin ctypes binding of libkdn (include/kdn.h).
 
-Argument marshalling only: every function checks that its tensors are CUDA,
-contiguous and of the right dtype, allocates outputs with PyTorch when the
-caller gives none, and passes raw device pointers and the current CUDA stream
-to the C ABI.  All arithmetic happens in the library's kernels.  If
+Argument marshalling only: every function checks that its tensors are CUDA
+(host, for kdn_forward_host), contiguous and of the right dtype, allocates
+outputs with PyTorch when the caller gives none, and passes raw pointers and
+the current CUDA stream to the C ABI.  All arithmetic happens in the library's kernels.  If
 ``libkdn.so`` cannot be loaded the first call raises; there is no fallback.
 Function names match the C entry points.
 """
@@ -57,6 +57,11 @@ def lib():
     L.kdn_iso_forward.restype = _i32
     L.kdn_iso_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + \
         [_f32, _i32, _vp, _sz, _vp]
+    L.kdn_forward_host_workspace_size.restype = _sz
+    L.kdn_forward_host_workspace_size.argtypes = [_i32] * 9
+    L.kdn_forward_host.restype = _i32
+    L.kdn_forward_host.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + \
+        [_f32, _i32, _i32, _vp, _sz, _vp]
     L.kdn_diag_forward.restype = _i32
     L.kdn_diag_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + \
         [_i32, _vp, _sz, _vp]
@@ -230,6 +235,65 @@ def kdn_diag_forward(q, k, v, a, w, r, S0=None, p0=None, chunk=KDN_CHUNK_AUTO, o
                      S_out=None, p_out=None, workspace=None):
     """Diagonal KDN forward.  Returns (o fp32 [B,T,H,dv], S_T, p_T [B,H,dk])."""
     return _forward(KDN_DIAG, q, k, v, a, w, r, S0, p0, 1.0, chunk, o, S_out, p_out, workspace)
+
+
+def _req_host(t, name, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f'{name} must be a host (CPU) tensor')
+    if not t.is_contiguous():
+        raise ValueError(f'{name} must be contiguous')
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f'{name} must be {dtype}, got {t.dtype}')
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f'{name} must have shape {tuple(shape)}, got {tuple(t.shape)}')
+    return t
+
+
+def kdn_forward_host_workspace_size(variant, B, T, H, dk, dv, in_dtype=KDN_BF16,
+                                    chunk=KDN_CHUNK_AUTO, slice_b=0):
+    return int(lib().kdn_forward_host_workspace_size(variant, B, T, H, dk, dv, in_dtype, chunk,
+                                                     slice_b))
+
+
+def kdn_forward_host(variant, q, k, v, a, w, r, S0=None, p0=None, info_scale=0.0,
+                     chunk=KDN_CHUNK_AUTO, slice_b=0, o=None, S_out=None, p_out=None,
+                     workspace=None, device=None):
+    """The forward with host tensors (pinned for overlap); outputs are host
+    tensors, valid once the current stream has been synchronised.  Returns
+    (o, S_T, p_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _in_dtype(q)
+    _req_host(q, 'q', dt)
+    _req_host(k, 'k', dt, (B, T, H, dk))
+    _req_host(v, 'v', dt, (B, T, H, dv))
+    f = torch.float32
+    _req_host(a, 'a', f, (B, T, H))
+    _req_host(r, 'r', f, (B, T, H))
+    pshape = (B, H) if variant == KDN_ISO else (B, H, dk)
+    _req_host(w, 'w', f, (B, T, H) if variant == KDN_ISO else (B, T, H, dk))
+    if S0 is not None:
+        _req_host(S0, 'S0', f, (B, H, dv, dk))
+    if p0 is not None:
+        _req_host(p0, 'p0', f, pshape)
+    o = _req_host(o, 'o', f, (B, T, H, dv)) if o is not None else \
+        torch.empty((B, T, H, dv), dtype=f).pin_memory()
+    S_out = _req_host(S_out, 'S_out', f, (B, H, dv, dk)) if S_out is not None else \
+        torch.empty((B, H, dv, dk), dtype=f).pin_memory()
+    p_out = _req_host(p_out, 'p_out', f, pshape) if p_out is not None else \
+        torch.empty(pshape, dtype=f).pin_memory()
+    need = kdn_forward_host_workspace_size(variant, B, T, H, dk, dv, _in_dtype(q), chunk, slice_b)
+    dev = device if device is not None else torch.device('cuda', torch.cuda.current_device())
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _req(workspace, 'workspace', torch.uint8)
+    st = lib().kdn_forward_host(variant, _ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a),
+                                _ptr(w), _ptr(r), _ptr(S0), _ptr(p0), _ptr(o), _ptr(S_out),
+                                _ptr(p_out), B, T, H, dk, dv, float(info_scale), int(chunk),
+                                int(slice_b), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, 'kdn_forward_host')
+    return o, S_out, p_out
 
 
 def kdn_decode_step(variant, q, k, v, a, w, r, S, p, o=None, info_scale=0.0):

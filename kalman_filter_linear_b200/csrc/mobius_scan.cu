@@ -129,18 +129,17 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
     incl_pre = __ldcg(ws.incl + pt0);
   }
 
+  // (steps past the end of the lane come in as identity steps: a = r = 1,
+  // w = n = 0)
   Mat2 P = identity();
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
-    if (t0 + i < T) {
-      const float c = info_scale * n[i];
-      const float a2 = a[i] * a[i];
-      const Mat2 M = {r[i] * a2, r[i] * w[i], c * a2, fmaf(c, w[i], r[i])};
-      P = mul(M, P);
-      if (i & 1) P = renorm(P);
-    }
+    const float c = info_scale * n[i];
+    const float a2 = a[i] * a[i];
+    const Mat2 M = {r[i] * a2, r[i] * w[i], c * a2, fmaf(c, w[i], r[i])};
+    P = mul(M, P);
+    if (i & 1) P = renorm(P);
   }
-  P = renorm(P);
 
   // ---- 2. warp inclusive scan, then block scan of warp totals
   Mat2 incl = P;
@@ -391,14 +390,17 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
       s_tile[(it + 1) & 1] = next;
       if (next < ntiles) fetch(next);
     }
+    if (t0 + kPerThread > T) {
+      const int nvalid = (int)max((int64_t)0, T - t0);
 #pragma unroll
-    for (int i = 0; i < kPerThread; ++i)
-      if (t0 + i >= T) {  // past the end of the lane: identity steps
-        a[i] = 1.f;
-        w[i] = 0.f;
-        r[i] = 1.f;
-        n[i] = 0.f;
-      }
+      for (int i = 0; i < kPerThread; ++i)
+        if (i >= nvalid) {  // past the end of the lane: identity steps
+          a[i] = 1.f;
+          w[i] = 0.f;
+          r[i] = 1.f;
+          n[i] = 0.f;
+        }
+    }
     scan_tile(a, w, r, n, tile, lambda0, info_scale, lam_out, prior_out, gain_out, N, T, ws, 1,
               debug_skip_tile, sh);
     // (the next iteration's first barrier keeps the shared tile state until

@@ -30,6 +30,24 @@ kdn_status kdn_testing_mobius_scan_unpublished_tile(
     int64_t T, void* workspace, size_t workspace_bytes, int64_t silent_tile,
     void* stream);
 
+/* kdn_iso_forward / kdn_diag_forward (variant) on the chunked engine at
+ * dk = dv = 128, bf16 q/k/v, S0 = 0, p0 = 1, except that the copy of chunk
+ * `skip_chunk`'s V tile is never issued.  The bounded wait for it gives up
+ * (after about one second), records KDN_ERR_TIMEOUT in the workspace error
+ * word, and every CTA takes its abort path: it waits (bounded) for its
+ * copies and MMAs in flight, frees its TMEM and returns.  The call returns
+ * normally; kdn_read_workspace_status() then reports KDN_ERR_TIMEOUT.
+ * Outputs are not meaningful.  1 <= skip_chunk < ceil(T / 64). */
+kdn_status kdn_testing_forward_skip_v_copy(kdn_variant variant, const void* q,
+                                           const void* k, const void* v,
+                                           const float* a, const float* w,
+                                           const float* r, float* o,
+                                           float* S_out, float* p_out, int B,
+                                           int T, int H, int skip_chunk,
+                                           void* workspace,
+                                           size_t workspace_bytes,
+                                           void* stream);
+
 #ifdef __cplusplus
 }
 #endif

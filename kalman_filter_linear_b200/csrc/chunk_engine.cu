@@ -1115,7 +1115,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const float* __restrict__ Wg, const float* __restrict__ Rg,
                        const float* S0, const float* __restrict__ P0, float* __restrict__ O,
                        float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
-                       uint32_t* __restrict__ err) {
+                       uint32_t* __restrict__ err, int debug_skip_v) {
   using P = WsPlan<DIAG>;
   constexpr int DV = 128;
   extern __shared__ uint8_t smem_raw[];
@@ -1595,7 +1595,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       tmem_wait_st();
       tc_fence_before();
       bar_group(kChainBar);
-      if (issuer && !bad && c + 1 < nchunks) issue_v(c + 1);  // the V tile is consumed
+      // (debug_skip_v: a test hook that leaves one chunk's V copy out, so the
+      // bounded wait for it gives up and the CTA takes its abort path)
+      if (issuer && !bad && c + 1 < nchunks && c + 1 != debug_skip_v)
+        issue_v(c + 1);  // the V tile is consumed
 
       // ---- MMA3: D3 = Zhi Thi + Zlo Thi + Zhi Tlo (T from the prep warps)
       if (fail(t_ready, (uint32_t)(c & 1))) bad = true;
@@ -2099,7 +2102,7 @@ template <bool DIAG>
 kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a,
                      const float* w, const float* r, const float* S0, const float* p0, float* o,
                      float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
-                     cudaStream_t s) {
+                     cudaStream_t s, int debug_skip_v) {
   using P = WsPlan<DIAG>;
   CUtensorMap mq, mk, mv, mo, mw;
   if (!make_map(&mq, q, B, T, H, kDK, 64) || !make_map(&mk, k, B, T, H, kDK, 64) ||
@@ -2124,7 +2127,7 @@ kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
   chunk_engine_ws_kernel<DIAG><<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
       mq, mk, mv, mo, mw, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa,
-      static_cast<uint32_t*>(ws));
+      static_cast<uint32_t*>(ws), debug_skip_v);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
@@ -2142,12 +2145,16 @@ size_t chunk_engine_workspace_size(bool diag, int B, int H) {
 kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const void* v,
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
-                               int T, int H, int dv, float kappa, void* ws, cudaStream_t s) {
+                               int T, int H, int dv, float kappa, void* ws, cudaStream_t s,
+                               int debug_skip_v) {
   if (dv == 128) {
     // one CTA per head reads p0 and writes p_out: no snapshot needed
-    return diag ? launch_ws<true>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s)
-                : launch_ws<false>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws, s);
+    return diag ? launch_ws<true>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws,
+                                  s, debug_skip_v)
+                : launch_ws<false>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws,
+                                   s, debug_skip_v);
   }
+  if (debug_skip_v >= 0) return KDN_ERR_UNSUPPORTED;  // the hook exists at d_v = 128 only
   return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
               : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
 }

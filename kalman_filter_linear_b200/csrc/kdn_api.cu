@@ -28,7 +28,7 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
                                int T, int H, int dv, float kappa, void* workspace,
-                               cudaStream_t s);
+                               cudaStream_t s, int debug_skip_v = -1);
 }  // namespace kdn
 
 namespace {
@@ -64,7 +64,8 @@ kdn_status forward_common(bool diag, const void* q, const void* k, const void* v
                           kdn_dtype in_dtype, const float* a, const float* w, const float* r,
                           const float* S0, const float* p0, float* o, float* S_out, float* p_out,
                           int B, int T, int H, int dk, int dv, float info_scale, int chunk,
-                          void* workspace, size_t workspace_bytes, void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream,
+                          int debug_skip_v = -1) {
   if (!q || !k || !v || !a || !w || !r || !o || !S_out || !p_out) return KDN_ERR_INVALID_ARG;
   if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
   if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
@@ -85,7 +86,7 @@ kdn_status forward_common(bool diag, const void* q, const void* k, const void* v
   if (need && (!workspace || workspace_bytes < need)) return KDN_ERR_WORKSPACE;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_INVALID_ARG;
   return kdn::chunk_engine_launch(diag, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv,
-                                  kappa, workspace, as_stream(stream));
+                                  kappa, workspace, as_stream(stream), debug_skip_v);
 }
 
 // ------------------------------------------------------------ host buffers
@@ -333,6 +334,18 @@ kdn_status kdn_read_workspace_status(const void* workspace, size_t workspace_byt
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return KDN_ERR_CUDA;
   return word == kdn::DEV_OK ? KDN_OK : KDN_ERR_TIMEOUT;
+}
+
+kdn_status kdn_testing_forward_skip_v_copy(kdn_variant variant, const void* q, const void* k,
+                                           const void* v, const float* a, const float* w,
+                                           const float* r, float* o, float* S_out, float* p_out,
+                                           int B, int T, int H, int skip_chunk, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  if (variant != KDN_ISO && variant != KDN_DIAG) return KDN_ERR_INVALID_ARG;
+  if (skip_chunk < 1 || skip_chunk >= (T + 63) / 64) return KDN_ERR_INVALID_ARG;
+  return forward_common(variant == KDN_DIAG, q, k, v, KDN_BF16, a, w, r, nullptr, nullptr, o,
+                        S_out, p_out, B, T, H, 128, 128, 0.f, KDN_CHUNK_64, workspace,
+                        workspace_bytes, stream, skip_chunk);
 }
 
 kdn_status kdn_testing_mobius_scan_unpublished_tile(

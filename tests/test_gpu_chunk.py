@@ -123,3 +123,23 @@ def test_chunked_workspace_status_ok_and_small_workspace_rejected():
     with pytest.raises(kdn.KdnError) as e:
         _run('iso', x, workspace=small)
     assert e.value.status == kdn.KDN_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("variant", ["iso", "diag"])
+def test_chunked_bounded_wait_reports_timeout_and_context_survives(variant):
+    """One V copy is left out: the engine's bounded wait gives up, every CTA
+    takes its abort path, the workspace reports KDN_ERR_TIMEOUT, and the next
+    call on the same context is correct again."""
+    B, T, H, d = 1, 256, 2, 128
+    x = to_dev(synth.layer_inputs(B, T, H, d, d, variant, seed=41, dtype='bf16'))
+    var = kdn.KDN_ISO if variant == 'iso' else kdn.KDN_DIAG
+    ws = torch.empty(kdn.kdn_forward_workspace_size(var, B, T, H, d, d, CH), dtype=torch.uint8,
+                     device='cuda')
+    kdn.kdn_testing_forward_skip_v_copy(var, x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], 2,
+                                        ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_ERR_TIMEOUT
+    o, S, p = _run(variant, x, workspace=ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_OK
+    o_r, S_r, p_r = _ref(variant, x)
+    assert rel_maxabs(o, o_r) <= OUT_TOL
+    assert rel_maxabs(S, S_r) <= STATE_TOL

@@ -191,6 +191,44 @@ kdn_status kdn_diag_forward(const void* q, const void* k, const void* v,
                             size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_forward_varlen -- kdn_iso_forward / kdn_diag_forward (variant) over N
+ * packed sequences of different lengths: sequence s is tokens
+ * [cu_seqlens[s], cu_seqlens[s+1]) of tensors laid out [total, H, ...]
+ * (that is [1, total, H, ...]), and it starts from its own S0[s], p0[s] and
+ * ends in its own S_out[s], p_out[s] (the prefill -> decode handoff:
+ * kdn_decode_step continues from them; "Kalman Delta Networks: ..."
+ * abstract, constant-memory decoding).  A sequence may be empty; it then
+ * hands S0, p0 (or zeros, ones) through.
+ *
+ * q, k     [total, H, dk] in_dtype device;  v [total, H, dv]
+ * a, r     [total, H] fp32 device;  w [total, H] (iso) or [total, H, dk]
+ * cu_seqlens  [N + 1] int32 device, cu_seqlens[0] = 0, non-decreasing,
+ *          cu_seqlens[N] = total.  Offsets out of order or out of range are
+ *          clamped and reported through the workspace (KDN_ERR_INVALID_ARG
+ *          from kdn_read_workspace_status).
+ * S0, S_out  [N, H, dv, dk];  p0, p_out  [N, H] (iso) or [N, H, dk] (diag)
+ * o        [total, H, dv] fp32 device
+ * info_scale  iso only, as kdn_iso_forward
+ * chunk    as kdn_iso_forward; the chunked engine serves d_v = 128 here (at
+ *          d_v = 64, KDN_CHUNK_AUTO takes the token-recurrent kernel and
+ *          KDN_CHUNK_64 returns KDN_ERR_UNSUPPORTED)
+ * workspace   device scratch of >= kdn_forward_varlen_workspace_size(...)
+ *             bytes (at least 256), 256-byte aligned
+ * total >= 0, N >= 1.  Other arguments and errors as kdn_iso_forward.
+ * ---------------------------------------------------------------------- */
+size_t kdn_forward_varlen_workspace_size(kdn_variant variant, int N, int H,
+                                         int dk, int dv, int chunk);
+kdn_status kdn_forward_varlen(kdn_variant variant, const void* q,
+                              const void* k, const void* v, kdn_dtype in_dtype,
+                              const float* a, const float* w, const float* r,
+                              const int32_t* cu_seqlens, const float* S0,
+                              const float* p0, float* o, float* S_out,
+                              float* p_out, int N, int total, int H, int dk,
+                              int dv, float info_scale, int chunk,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_forward_host -- kdn_iso_forward / kdn_diag_forward (variant) with every
  * tensor in host memory, for callers whose data is not on the device yet.
  * The batch goes through the device in slices of slice_b entries (<= 0
@@ -254,9 +292,11 @@ kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k,
 
 /* ------------------------------------------------------------------------
  * kdn_read_workspace_status -- synchronise `stream`, then report the device
- * error word a previous call left in `workspace`: KDN_OK, or KDN_ERR_TIMEOUT
- * if a bounded on-device wait gave up.  Also returns KDN_ERR_CUDA if the
- * stream reports an error.  This is the only call that blocks the host.
+ * error word a previous call left in `workspace`: KDN_OK, KDN_ERR_TIMEOUT
+ * if a bounded on-device wait gave up, or KDN_ERR_INVALID_ARG if packed-
+ * sequence offsets were out of order or out of range.  Also returns
+ * KDN_ERR_CUDA if the stream reports an error.  This is the only call that
+ * blocks the host.
  * ---------------------------------------------------------------------- */
 kdn_status kdn_read_workspace_status(const void* workspace,
                                      size_t workspace_bytes, void* stream);

@@ -1105,7 +1105,9 @@ __device__ __forceinline__ bool bar_group_or(int id, bool flag) {
 
 constexpr int kTeamA = 6, kTeamB = 7;
 
-template <bool DIAG>
+// PACKED: the B "batch entries" are packed sequences given by cu_seqlens (the
+// instantiation for ordinary [B, T, H, d] tensors carries none of its code).
+template <bool DIAG, bool PACKED>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -1115,7 +1117,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const float* __restrict__ Wg, const float* __restrict__ Rg,
                        const float* S0, const float* __restrict__ P0, float* __restrict__ O,
                        float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
-                       uint32_t* __restrict__ err, int debug_skip_v) {
+                       uint32_t* __restrict__ err, int debug_skip_v,
+                       const int* __restrict__ cu_seqlens) {
   using P = WsPlan<DIAG>;
   constexpr int DV = 128;
   extern __shared__ uint8_t smem_raw[];
@@ -1123,9 +1126,29 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x;
-  const int b = bh / H, h = bh % H;
-  const int nchunks = (T + kC - 1) / kC;
+  const int h = bh % H;
+  // This CTA's sequence: batch entry b of [B, T, H, d] tensors, or (packed
+  // sequences, cu_seqlens given) tokens [tbeg, tbeg + Tn) of [1, T, H, d] ones.
+  int b = bh / H, tbeg = 0, Tn = T;
+  if constexpr (PACKED) {
+    const int s0 = cu_seqlens[bh / H], s1 = cu_seqlens[bh / H + 1];
+    b = 0;
+    tbeg = min(max(s0, 0), T);
+    Tn = min(max(s1, tbeg), T) - tbeg;
+    if (threadIdx.x == 0 && (s0 < 0 || s1 < s0 || s1 > T)) atomicOr(err, DEV_BAD_ARG);
+  }
+  const int nchunks = (Tn + kC - 1) / kC;
   const uint32_t sbase = smem_u32(smem);
+  if (PACKED && Tn == 0) {
+    // an empty sequence hands its initial state and variance through
+    const size_t n = (size_t)DV * kDK;
+    for (size_t i = threadIdx.x; i < n; i += kThreads)
+      S_out[(size_t)bh * n + i] = S0 ? S0[(size_t)bh * n + i] : 0.f;
+    const int np = DIAG ? kDK : 1;
+    for (int i = threadIdx.x; i < np; i += kThreads)
+      P_out[(size_t)bh * np + i] = P0 ? P0[(size_t)bh * np + i] : 1.f;
+    return;
+  }
 
   // scalar area (floats); [4][64] arrays are indexed by chunk & 3
   float* scf = reinterpret_cast<float*>(smem + P::OFF_SC);
@@ -1158,7 +1181,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* sT = smem + P::OFF_T;
   uint8_t* sP = smem + P::OFF_P;
   uint8_t* sV = smem + P::OFF_V;
-  const float* sW = reinterpret_cast<const float*>(smem + P::OFF_W);
+  float* sW = reinterpret_cast<float*>(smem + P::OFF_W);
 
   if (tid == 0) {
     for (int i = 0; i < 19; ++i) mbar_init(&bars[i], 1);
@@ -1199,12 +1222,12 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   // a, w, r of chunk c (one warp): loaded a chunk ahead into registers
   float ps_a[2], ps_r[2], ps_w[2];
   auto fetch_scalars = [&](int c) {
-    const int t0 = c * kC, valid = min(kC, T - t0);
+    const int t0 = c * kC, valid = min(kC, Tn - t0);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int t = lane + 32 * i;
       const bool in = t < valid;
-      const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+      const size_t tok = ((size_t)b * T + tbeg + t0 + t) * H + h;
       ps_a[i] = in ? __ldg(Ag + tok) : 1.f;
       ps_r[i] = in ? __ldg(Rg + tok) : 1.f;
       ps_w[i] = (!DIAG && in) ? __ldg(Wg + tok) : 0.f;
@@ -1224,6 +1247,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto key_norms = [&](int c, int pt) {
     const int t = pt & 63, half = pt >> 6;
     const uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + half * 16384;
+    // (packed sequences: the tile runs on into the next one)
+    const bool in = !PACKED || t < Tn - c * kC;
     float acc = 0.f;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
@@ -1232,7 +1257,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc = fmaf(x[e], x[e], acc);
     }
-    sc_n[64 * half + t] = acc;
+    sc_n[64 * half + t] = in ? acc : 0.f;
   };
   // decay prefix and Mobius scan of the variance of chunk c (one warp, two
   // tokens per lane): lg, gamma, gamma_C, beta, the update coefficients, carry
@@ -1284,8 +1309,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     p = __fdividef(r0 * pp0, fmaf(c0, pp0, r0));
     const float pp1 = fmaf(a1 * a1, p, w1);
     p = __fdividef(r1 * pp1, fmaf(c1, pp1, r1));
-    const float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
-    const float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
+    // (tokens past the sequence end write nothing: beta = 0)
+    float b0 = __fdividef(pp0, fmaf(pp0, n0, r0));
+    float b1 = __fdividef(pp1, fmaf(pp1, n1, r1));
+    if constexpr (PACKED) {
+      const int vld = Tn - c * kC;
+      b0 = ta < vld ? b0 : 0.f;
+      b1 = tb < vld ? b1 : 0.f;
+    }
     sc_beta[64 * sl + ta] = b0;
     sc_beta[64 * sl + tb] = b1;
     sc_coef[64 * sl + ta] = b0 * exp2f(lg_last - lg0);
@@ -1307,15 +1338,15 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint8_t* kqd = smem + P::OFF_KQ + st * P::KQ_BYTES;
     mbar_expect_tx(&full_kq[st], P::KQ_BYTES);
     for (int kb = 0; kb < 2; ++kb) {
-      tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, t0, b);
-      tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, t0, b);
+      tma_load_4d(kqd + kb * 16384, &tm_k, &full_kq[st], kb * 64, h, tbeg + t0, b);
+      tma_load_4d(kqd + kb * 16384 + 8192, &tm_q, &full_kq[st], kb * 64, h, tbeg + t0, b);
     }
     pend_kq = (pend_kq & ~(3u << (2 * st))) | ((1u | (kq_parity(c) << 1)) << (2 * st));
   };
   auto issue_v = [&](int c) {
     mbar_expect_tx(full_v, 16384);
-    tma_load_4d(sV, &tm_v, full_v, 0, h, c * kC, b);
-    tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, c * kC, b);
+    tma_load_4d(sV, &tm_v, full_v, 0, h, tbeg + c * kC, b);
+    tma_load_4d(sV + 8192, &tm_v, full_v, 64, h, tbeg + c * kC, b);
     pend_v = c & 1;
   };
   // (diagonal) w quarter n: tokens [16 n, 16 n + 16) of the sequence, for the
@@ -1325,7 +1356,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int bf = n & 1;
     uint64_t* bar_ = &w_full[2 * wv + bf];
     mbar_expect_tx(bar_, 2048);
-    tma_load_4d(smem + P::OFF_W + (2 * wv + bf) * 2048, &tm_w, bar_, 32 * wv, h, 16 * n, b);
+    tma_load_4d(smem + P::OFF_W + (2 * wv + bf) * 2048, &tm_w, bar_, 32 * wv, h, tbeg + 16 * n, b);
     pend_w = (pend_w & ~(3u << (2 * bf))) | ((1u | ((uint32_t)((n >> 1) & 1) << 1)) << (2 * bf));
   };
   // D1 = [K;Q] K^T of chunk c (A: the stage's key rows then query rows per d
@@ -1370,8 +1401,12 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int sl = c & 3;
     const float* a_s = sc_a + 64 * sl;
     const float* r_s = sc_r + 64 * sl;
-    const uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + (d >> 6) * 16384;
+    uint8_t* kt = smem + P::OFF_KQ + (c % P::kStages) * P::KQ_BYTES + (d >> 6) * 16384;
     const uint32_t col = (uint32_t)(d & 63);
+    // tokens past the end of a packed sequence (its tiles run on into the
+    // next one) become identity steps: their k and w are zeroed in place
+    // (in this thread's own column) before use
+    const int vld = Tn - c * kC;
     // p = x / y, carried projectively so that no division sits on the
     // token-to-token chain: with u = a^2 x + w y (= p^- y), one token maps
     // (x, y) to (r u, k^2 u + r y), the Mobius map's matrix applied to the
@@ -1383,7 +1418,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int n = 4 * c + q;
       if (fail(&w_full[2 * (d >> 5) + (n & 1)], (uint32_t)((n >> 1) & 1))) bad = true;
       if (!bad) {
-        const float* wq = sW + (2 * (d >> 5) + (n & 1)) * 512 + (d & 31);
+        float* wq = sW + (2 * (d >> 5) + (n & 1)) * 512 + (d & 31);
+        if (PACKED && vld < 16 * q + 16) {
+          for (int e = max(vld - 16 * q, 0); e < 16; ++e) {
+            wq[e * 32] = 0.f;
+            *reinterpret_cast<__nv_bfloat16*>(kt + sw128_offset((uint32_t)(16 * q + e), col)) =
+                __float2bfloat16_rn(0.f);
+          }
+        }
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) {
           const float4 a4 = *reinterpret_cast<const float4*>(a_s + 16 * q + 4 * i4);
@@ -1718,12 +1760,15 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       // (isotropic: into the staging tile [t][v]; one bulk tensor store per
       // chunk writes it, rows past T excluded. diagonal: straight to memory,
       // each warp writing 128 contiguous bytes per token)
-      if constexpr (DIAG) {
+      // (also the isotropic variant for the last, partial chunk of a packed
+      // sequence: a tile store there would run into the next sequence)
+      const bool direct = DIAG || (PACKED && Tn - t0 < kC);
+      if (direct) {
         float x[32];
         tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
         tmem_wait_ld();
-        const int valid = min(kC, T - t0);
-        float* dst = O + (((size_t)b * T + t0 + 32 * ch) * H + h) * DV + v;
+        const int valid = min(kC, Tn - t0);
+        float* dst = O + (((size_t)b * T + tbeg + t0 + 32 * ch) * H + h) * DV + v;
         const size_t ostride = (size_t)H * DV;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -1736,7 +1781,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * DV] = x[i];
         fence_async_smem();
-        if (issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);  // stage s is free
+        // stage s is free (a chunk with the direct store above is the last)
+        if (issuer && !bad && c + P::kStages < nchunks) issue_kq(c + P::kStages);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -1744,8 +1790,8 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         bad = true;
         break;
       }
-      if (!DIAG && issuer) {
-        tma_store_4d(&tm_o, sOut, 0, h, t0, b);
+      if (!direct && issuer) {
+        tma_store_4d(&tm_o, sOut, 0, h, tbeg + t0, b);
         bulk_commit();
       }
     }
@@ -2098,36 +2144,39 @@ kdn_status launch(const void* q, const void* k, const void* v, const float* a, c
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
+// (cu_seqlens: B packed sequences in [1, T, H, d] tensors, T = total tokens)
 template <bool DIAG>
 kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a,
                      const float* w, const float* r, const float* S0, const float* p0, float* o,
                      float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
-                     cudaStream_t s, int debug_skip_v) {
+                     cudaStream_t s, int debug_skip_v, const int* cu_seqlens) {
+  const int Bm = cu_seqlens ? 1 : B;  // batch extent of the tensor maps
   using P = WsPlan<DIAG>;
   CUtensorMap mq, mk, mv, mo, mw;
-  if (!make_map(&mq, q, B, T, H, kDK, 64) || !make_map(&mk, k, B, T, H, kDK, 64) ||
-      !make_map(&mv, v, B, T, H, 128, 64))
+  if (!make_map(&mq, q, Bm, T, H, kDK, 64) || !make_map(&mk, k, Bm, T, H, kDK, 64) ||
+      !make_map(&mv, v, Bm, T, H, 128, 64))
     return KDN_ERR_CUDA;
   // isotropic: the output tile map; diagonal: the output is written without a
   // map, and w [B, T, H, 128] is read in boxes of 16 tokens
   if (DIAG) {
     mo = mq;
-    if (!make_out_map(&mw, w, B, T, H, kDK, 16, 32)) return KDN_ERR_CUDA;
+    if (!make_out_map(&mw, w, Bm, T, H, kDK, 16, 32)) return KDN_ERR_CUDA;
   } else {
-    if (!make_out_map(&mo, o, B, T, H, 128, 64)) return KDN_ERR_CUDA;
+    if (!make_out_map(&mo, o, Bm, T, H, 128, 64)) return KDN_ERR_CUDA;
     mw = mq;
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(chunk_engine_ws_kernel<DIAG>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, P::ALLOC) != cudaSuccess)
+  static bool attr_set[2] = {false, false};
+  auto kern = cu_seqlens ? chunk_engine_ws_kernel<DIAG, true> : chunk_engine_ws_kernel<DIAG, false>;
+  if (!attr_set[cu_seqlens ? 1 : 0]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, P::ALLOC) !=
+        cudaSuccess)
       return KDN_ERR_CUDA;
-    attr_set = true;
+    attr_set[cu_seqlens ? 1 : 0] = true;
   }
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
-  chunk_engine_ws_kernel<DIAG><<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
+  kern<<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
       mq, mk, mv, mo, mw, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa,
-      static_cast<uint32_t*>(ws), debug_skip_v);
+      static_cast<uint32_t*>(ws), debug_skip_v, cu_seqlens);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
@@ -2146,15 +2195,16 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
                                int T, int H, int dv, float kappa, void* ws, cudaStream_t s,
-                               int debug_skip_v) {
+                               int debug_skip_v, const int* cu_seqlens) {
   if (dv == 128) {
     // one CTA per head reads p0 and writes p_out: no snapshot needed
     return diag ? launch_ws<true>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws,
-                                  s, debug_skip_v)
+                                  s, debug_skip_v, cu_seqlens)
                 : launch_ws<false>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws,
-                                   s, debug_skip_v);
+                                   s, debug_skip_v, cu_seqlens);
   }
-  if (debug_skip_v >= 0) return KDN_ERR_UNSUPPORTED;  // the hook exists at d_v = 128 only
+  // the hook and packed sequences exist at d_v = 128 only
+  if (debug_skip_v >= 0 || cu_seqlens) return KDN_ERR_UNSUPPORTED;
   return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
               : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
 }

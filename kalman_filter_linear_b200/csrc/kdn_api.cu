@@ -21,14 +21,16 @@ kdn_status mobius_scan_launch(const float* a, const float* w, const float* r, co
 kdn_status recurrent_launch(bool diag, kdn_dtype dt, const void* q, const void* k, const void* v,
                             const float* a, const float* w, const float* r, const float* S0,
                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
-                            int H, int dk, int dv, float kappa, cudaStream_t s);
+                            int H, int dk, int dv, float kappa, cudaStream_t s,
+                            const int* cu_seqlens = nullptr, uint32_t* err = nullptr);
 bool chunk_engine_supported(kdn_dtype dt, int dk, int dv);
 size_t chunk_engine_workspace_size(bool diag, int B, int H);
 kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const void* v,
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
                                int T, int H, int dv, float kappa, void* workspace,
-                               cudaStream_t s, int debug_skip_v = -1);
+                               cudaStream_t s, int debug_skip_v = -1,
+                               const int* cu_seqlens = nullptr);
 }  // namespace kdn
 
 namespace {
@@ -65,28 +67,44 @@ kdn_status forward_common(bool diag, const void* q, const void* k, const void* v
                           const float* S0, const float* p0, float* o, float* S_out, float* p_out,
                           int B, int T, int H, int dk, int dv, float info_scale, int chunk,
                           void* workspace, size_t workspace_bytes, void* stream,
-                          int debug_skip_v = -1) {
+                          int debug_skip_v = -1, const int* cu_seqlens = nullptr) {
   if (!q || !k || !v || !a || !w || !r || !o || !S_out || !p_out) return KDN_ERR_INVALID_ARG;
   if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
-  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  // (packed sequences: B sequences of T tokens in all, T >= 0)
+  if (!shape_ok(B, cu_seqlens ? std::max(T, 1) : T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
   if (!(info_scale == info_scale) || info_scale > 3.0e38f) return KDN_ERR_INVALID_ARG;
   if (!al16(q) || !al16(k) || !al16(v) || !al16(a) || !al16(w) || !al16(r) || !al16(o) ||
       !al16(S_out) || !al16(p_out) || !al16_or_null(S0) || !al16_or_null(p0))
     return KDN_ERR_INVALID_ARG;
   if (!dims_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
-  const int path = select_path(chunk, in_dtype, dk, dv);
+  int path = select_path(chunk, in_dtype, dk, dv);
   if (path == -2) return KDN_ERR_INVALID_ARG;
   if (path == -1) return KDN_ERR_UNSUPPORTED;
+  if (cu_seqlens) {
+    // packed sequences: the chunked engine at d_v = 128, otherwise the
+    // token-recurrent kernel; a workspace always carries the error word
+    if (path == 1 && (dv != 128 || T == 0)) {
+      if (chunk == KDN_CHUNK_64 && dv != 128) return KDN_ERR_UNSUPPORTED;
+      path = 0;
+    }
+    if (!workspace || workspace_bytes < 256) return KDN_ERR_WORKSPACE;
+  }
   const float kappa = info_scale > 0.f ? info_scale : 1.f / (float)dk;
   if (path == 0) {
+    uint32_t* err = nullptr;
+    if (cu_seqlens) {
+      if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDN_ERR_INVALID_ARG;
+      err = static_cast<uint32_t*>(workspace);
+      if (cudaMemsetAsync(err, 0, 4, as_stream(stream)) != cudaSuccess) return KDN_ERR_CUDA;
+    }
     return kdn::recurrent_launch(diag, in_dtype, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T,
-                                 H, dk, dv, kappa, as_stream(stream));
+                                 H, dk, dv, kappa, as_stream(stream), cu_seqlens, err);
   }
   const size_t need = kdn::chunk_engine_workspace_size(diag, B, H);
   if (need && (!workspace || workspace_bytes < need)) return KDN_ERR_WORKSPACE;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_INVALID_ARG;
   return kdn::chunk_engine_launch(diag, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv,
-                                  kappa, workspace, as_stream(stream), debug_skip_v);
+                                  kappa, workspace, as_stream(stream), debug_skip_v, cu_seqlens);
 }
 
 // ------------------------------------------------------------ host buffers
@@ -198,6 +216,26 @@ kdn_status kdn_diag_forward(const void* q, const void* k, const void* v, kdn_dty
                             size_t workspace_bytes, void* stream) {
   return forward_common(true, q, k, v, in_dtype, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk,
                         dv, 1.0f, chunk, workspace, workspace_bytes, stream);
+}
+
+size_t kdn_forward_varlen_workspace_size(kdn_variant variant, int N, int H, int dk, int dv,
+                                         int chunk) {
+  if (N < 1 || H < 1 || !dims_supported(dk, dv)) return 0;
+  const size_t need = kdn_forward_workspace_size(variant, N, 1, H, dk, dv, chunk);
+  return need > 256 ? need : 256;
+}
+
+kdn_status kdn_forward_varlen(kdn_variant variant, const void* q, const void* k, const void* v,
+                              kdn_dtype in_dtype, const float* a, const float* w, const float* r,
+                              const int32_t* cu_seqlens, const float* S0, const float* p0,
+                              float* o, float* S_out, float* p_out, int N, int total, int H,
+                              int dk, int dv, float info_scale, int chunk, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (variant != KDN_ISO && variant != KDN_DIAG) return KDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || total < 0) return KDN_ERR_INVALID_ARG;
+  return forward_common(variant == KDN_DIAG, q, k, v, in_dtype, a, w, r, S0, p0, o, S_out, p_out,
+                        N, total, H, dk, dv, variant == KDN_DIAG ? 1.f : info_scale, chunk,
+                        workspace, workspace_bytes, stream, -1, cu_seqlens);
 }
 
 kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k, const void* v,
@@ -333,7 +371,8 @@ kdn_status kdn_read_workspace_status(const void* workspace, size_t workspace_byt
   uint32_t word = 0;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
     return KDN_ERR_CUDA;
-  return word == kdn::DEV_OK ? KDN_OK : KDN_ERR_TIMEOUT;
+  if (word & kdn::DEV_TIMEOUT) return KDN_ERR_TIMEOUT;
+  return word == kdn::DEV_OK ? KDN_OK : KDN_ERR_INVALID_ARG;
 }
 
 kdn_status kdn_testing_forward_skip_v_copy(kdn_variant variant, const void* q, const void* k,

@@ -13,8 +13,9 @@
 
 namespace kdn {
 
-// Device error word codes written into a workspace (first 4 bytes).
-enum : uint32_t { DEV_OK = 0u, DEV_TIMEOUT = 1u };
+// Device error word bits written into a workspace (first 4 bytes): a bounded
+// wait gave up; packed-sequence offsets out of order or out of range.
+enum : uint32_t { DEV_OK = 0u, DEV_TIMEOUT = 1u, DEV_BAD_ARG = 2u };
 
 // Wall-clock limit of every bounded on-device wait, in nanoseconds.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s

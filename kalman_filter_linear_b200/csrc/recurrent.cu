@@ -68,10 +68,21 @@ recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT
                  const float* __restrict__ A, const float* __restrict__ Wn,
                  const float* __restrict__ R, const float* S0, const float* P0,
                  float* __restrict__ O, float* S_out, float* P_out, int T, int H, int dv,
-                 float kappa) {
+                 float kappa, const int* __restrict__ cu_seqlens, uint32_t* err) {
   constexpr int DK = CPL * 32;
   const int bh = blockIdx.x;
-  const int b = bh / H, h = bh % H;
+  const int h = bh % H;
+  // this CTA's tokens: rows [row0, row0 + Tn) of the [rows, H, ...] tensors
+  // (batch entry bh / H, or packed sequence bh / H when cu_seqlens is given)
+  size_t row0 = (size_t)(bh / H) * T;
+  int Tn = T;
+  if (cu_seqlens) {
+    const int s0 = cu_seqlens[bh / H], s1 = cu_seqlens[bh / H + 1];
+    const int tbeg = min(max(s0, 0), T);
+    Tn = min(max(s1, tbeg), T) - tbeg;
+    row0 = (size_t)tbeg;
+    if (err && threadIdx.x == 0 && (s0 < 0 || s1 < s0 || s1 > T)) atomicOr(err, DEV_BAD_ARG);
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   // ---- state into registers
@@ -99,8 +110,8 @@ recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT
     p[0] = P0 ? P0[bh] : 1.f;
   }
 
-  for (int t = 0; t < T; ++t) {
-    const size_t tok = ((size_t)b * T + t) * H + h;
+  for (int t = 0; t < Tn; ++t) {
+    const size_t tok = (row0 + t) * H + h;
     float k[CPL], q[CPL];
     load_vec<CPL>(K + tok * DK, lane, k);
     load_vec<CPL>(Q + tok * DK, lane, q);
@@ -208,10 +219,11 @@ recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT
 template <bool DIAG, int CPL, typename InT>
 kdn_status launch_t(const void* q, const void* k, const void* v, const float* a, const float* w,
                     const float* r, const float* S0, const float* p0, float* o, float* S_out,
-                    float* p_out, int B, int T, int H, int dv, float kappa, cudaStream_t s) {
+                    float* p_out, int B, int T, int H, int dv, float kappa, cudaStream_t s,
+                    const int* cu, uint32_t* err) {
   recurrent_kernel<DIAG, CPL, InT><<<B * H, kWarps * 32, 0, s>>>(
       static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w, r,
-      S0, p0, o, S_out, p_out, T, H, dv, kappa);
+      S0, p0, o, S_out, p_out, T, H, dv, kappa, cu, err);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
@@ -219,11 +231,11 @@ template <bool DIAG, typename InT>
 kdn_status launch_dk(const void* q, const void* k, const void* v, const float* a, const float* w,
                      const float* r, const float* S0, const float* p0, float* o, float* S_out,
                      float* p_out, int B, int T, int H, int dk, int dv, float kappa,
-                     cudaStream_t s) {
+                     cudaStream_t s, const int* cu, uint32_t* err) {
   switch (dk) {
-    case 32: return launch_t<DIAG, 1, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s);
-    case 64: return launch_t<DIAG, 2, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s);
-    case 128: return launch_t<DIAG, 4, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s);
+    case 32: return launch_t<DIAG, 1, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
+    case 64: return launch_t<DIAG, 2, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
+    case 128: return launch_t<DIAG, 4, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
     default: return KDN_ERR_UNSUPPORTED;
   }
 }
@@ -235,15 +247,16 @@ kdn_status launch_dk(const void* q, const void* k, const void* v, const float* a
 kdn_status recurrent_launch(bool diag, kdn_dtype dt, const void* q, const void* k, const void* v,
                             const float* a, const float* w, const float* r, const float* S0,
                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
-                            int H, int dk, int dv, float kappa, cudaStream_t s) {
+                            int H, int dk, int dv, float kappa, cudaStream_t s,
+                            const int* cu_seqlens, uint32_t* err) {
   if (diag) {
     return dt == KDN_BF16
-               ? launch_dk<true, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s)
-               : launch_dk<true, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s);
+               ? launch_dk<true, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err)
+               : launch_dk<true, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err);
   }
   return dt == KDN_BF16
-             ? launch_dk<false, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s)
-             : launch_dk<false, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s);
+             ? launch_dk<false, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err)
+             : launch_dk<false, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err);
 }
 
 }  // namespace kdn

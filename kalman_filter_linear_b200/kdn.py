@@ -57,6 +57,11 @@ def lib():
     L.kdn_iso_forward.restype = _i32
     L.kdn_iso_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + \
         [_f32, _i32, _vp, _sz, _vp]
+    L.kdn_forward_varlen_workspace_size.restype = _sz
+    L.kdn_forward_varlen_workspace_size.argtypes = [_i32] * 6
+    L.kdn_forward_varlen.restype = _i32
+    L.kdn_forward_varlen.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 9 + [_i32] * 5 + \
+        [_f32, _i32, _vp, _sz, _vp]
     L.kdn_forward_host_workspace_size.restype = _sz
     L.kdn_forward_host_workspace_size.argtypes = [_i32] * 9
     L.kdn_forward_host.restype = _i32
@@ -237,6 +242,49 @@ def kdn_diag_forward(q, k, v, a, w, r, S0=None, p0=None, chunk=KDN_CHUNK_AUTO, o
                      S_out=None, p_out=None, workspace=None):
     """Diagonal KDN forward.  Returns (o fp32 [B,T,H,dv], S_T, p_T [B,H,dk])."""
     return _forward(KDN_DIAG, q, k, v, a, w, r, S0, p0, 1.0, chunk, o, S_out, p_out, workspace)
+
+
+def kdn_forward_varlen_workspace_size(variant, N, H, dk, dv, chunk=KDN_CHUNK_AUTO):
+    return int(lib().kdn_forward_varlen_workspace_size(variant, N, H, dk, dv, chunk))
+
+
+def kdn_forward_varlen(variant, q, k, v, a, w, r, cu_seqlens, S0=None, p0=None, info_scale=0.0,
+                       chunk=KDN_CHUNK_AUTO, o=None, S_out=None, p_out=None, workspace=None):
+    """The forward over packed sequences: q, k [total, H, dk], v [total, H, dv],
+    a, r [total, H], w [total, H] (iso) or [total, H, dk] (diag), cu_seqlens
+    [N + 1] int32.  Returns (o [total, H, dv], S_T [N, H, dv, dk], p_T)."""
+    total, H, dk = q.shape
+    dv = v.shape[-1]
+    N = cu_seqlens.numel() - 1
+    dt = q.dtype
+    _in_dtype(q)
+    _req(q, 'q', dt)
+    _req(k, 'k', dt, (total, H, dk))
+    _req(v, 'v', dt, (total, H, dv))
+    f = torch.float32
+    _req(a, 'a', f, (total, H))
+    _req(r, 'r', f, (total, H))
+    pshape = (N, H) if variant == KDN_ISO else (N, H, dk)
+    _req(w, 'w', f, (total, H) if variant == KDN_ISO else (total, H, dk))
+    _req(cu_seqlens, 'cu_seqlens', torch.int32, (N + 1,))
+    _opt(S0, 'S0', f, (N, H, dv, dk))
+    _opt(p0, 'p0', f, pshape)
+    dev = q.device
+    o = _req(o, 'o', f, (total, H, dv)) if o is not None else \
+        torch.empty((total, H, dv), dtype=f, device=dev)
+    S_out = _req(S_out, 'S_out', f, (N, H, dv, dk)) if S_out is not None else \
+        torch.empty((N, H, dv, dk), dtype=f, device=dev)
+    p_out = _req(p_out, 'p_out', f, pshape) if p_out is not None else \
+        torch.empty(pshape, dtype=f, device=dev)
+    need = kdn_forward_varlen_workspace_size(variant, N, H, dk, dv, chunk)
+    workspace = _workspace(need, dev, workspace)
+    st = lib().kdn_forward_varlen(variant, _ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a),
+                                  _ptr(w), _ptr(r), _ptr(cu_seqlens), _ptr(S0), _ptr(p0), _ptr(o),
+                                  _ptr(S_out), _ptr(p_out), N, total, H, dk, dv,
+                                  float(info_scale), int(chunk), _ptr(workspace),
+                                  workspace.numel(), _stream())
+    _check(st, 'kdn_forward_varlen')
+    return o, S_out, p_out
 
 
 def _req_host(t, name, dtype=None, shape=None):

@@ -12,7 +12,9 @@ L2, so no flush is needed between steps.  Prints ONE JSON line (rank 0).
 
 Also measured on the same run and reported under "secondary": the Diagonal
 KDN forward at the same shape, the standalone variance scan (4096 x 65536),
-the long-context diagonal forward (B1 T65536) and the decode step (batch 256).
+the long-context diagonal forward (B1 T65536), the decode step (batch 256) and
+the isotropic forward over 32768 tokens packed from sequences of mixed length
+(kdn_forward_varlen).
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores.
@@ -25,6 +27,7 @@ CUDA-event time.
 from __future__ import annotations
 
 import argparse
+import itertools
 import json
 import os
 import re
@@ -252,7 +255,7 @@ def main():
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
-    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode'],
+    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen'],
                     help='run only this kernel (for profiler captures) and print its timing')
     ap.add_argument('--B', type=int, default=None, help='batch override for --only')
     ap.add_argument('--T', type=int, default=None, help='length override for --only')
@@ -403,6 +406,8 @@ def run_only(args):
         f = lambda: kdn.kdn_mobius_scan(xs['a'], xs['w'], xs['r'], xs['n'], None,
                                         c['info_scale'], lambda_out=lam, workspace=wss)
         units, alg = N * T, N * T * 20
+    elif args.only == 'varlen':
+        f, units, alg, _ = varlen_case(kdn, synth, dev)
     else:
         c = synth.WORKLOADS['diag_long']
         B = args.B or c['decode_batch']
@@ -417,6 +422,31 @@ def run_only(args):
     ms = time_launches(f, args.steps, args.warmup, stream) / max(args.steps, 1)
     print(json.dumps({'only': args.only, 'ms': ms, 'units_per_s': units / ms * 1e3,
                       'achieved_gbs': alg / ms / 1e6, 'algorithmic_bytes': alg}))
+
+
+def varlen_case(kdn, synth, dev):
+    """The packed isotropic forward: (launch fn, tokens, algorithmic bytes,
+    description)."""
+    import torch
+    c = synth.WORKLOADS['iso_varlen']
+    lengths = synth.packed_lengths(c['total'], c['seed'], c['min_len'], c['max_len'])
+    total, H, d, N = c['total'], c['H'], c['dk'], len(lengths)
+    x = synth.layer_inputs(1, total, H, d, d, 'iso', c['seed'], c['dtype'])
+    x = {k: v[0].to(dev) for k, v in x.items()}
+    cu = torch.tensor([0] + list(itertools.accumulate(lengths)),
+                      dtype=torch.int32, device=dev)
+    ws = torch.empty(kdn.kdn_forward_varlen_workspace_size(kdn.KDN_ISO, N, H, d, d),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty((total, H, d), dtype=torch.float32, device=dev)
+    S = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    p = torch.empty((N, H), dtype=torch.float32, device=dev)
+    f = lambda: kdn.kdn_forward_varlen(kdn.KDN_ISO, x['q'], x['k'], x['v'], x['a'], x['w'],
+                                       x['r'], cu, o=o, S_out=S, p_out=p, workspace=ws)
+    # tokens move as in one B1 T=total launch; the final state is per sequence
+    alg = layer_bytes('iso', 1, total, H, d, d) + (N - 1) * H * (d * d + 1) * 4
+    desc = {'sequences': N, 'tokens': total, 'max_len': max(lengths),
+            'min_len': min(lengths), 'H': H, 'd': d}
+    return f, total, alg, desc
 
 
 def measure_secondary(kdn, synth, dev, stream, hbm_peak):
@@ -483,6 +513,14 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     alg = decode_bytes(Bd, H, d, d)
     out['decode'] = {'tokens_per_s': Bd / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
                      'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg}
+    del Sd, pd, xd, od
+    # packed variable-length isotropic forward, 32768 tokens
+    f, units, alg, desc = varlen_case(kdn, synth, dev)
+    n = 10
+    ms = time_launches(f, n, 3, stream) / n
+    out['iso_varlen'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
+                         'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                         'algorithmic_bytes': alg, **desc}
     return out
 
 

@@ -198,7 +198,10 @@ kdn_status kdn_diag_forward(const void* q, const void* k, const void* v,
  * ends in its own S_out[s], p_out[s] (the prefill -> decode handoff:
  * kdn_decode_step continues from them; "Kalman Delta Networks: ..."
  * abstract, constant-memory decoding).  A sequence may be empty; it then
- * hands S0, p0 (or zeros, ones) through.
+ * hands S0, p0 (or zeros, ones) through.  On the chunked engine, when the
+ * N x H (sequence, head) problems outnumber the SMs, a one-block kernel first
+ * orders the sequences longest first (by chunk count) into the workspace and
+ * the engine starts them in that order; results do not depend on the order.
  *
  * q, k     [total, H, dk] in_dtype device;  v [total, H, dv]
  * a, r     [total, H] fp32 device;  w [total, H] (iso) or [total, H, dk]
@@ -213,7 +216,8 @@ kdn_status kdn_diag_forward(const void* q, const void* k, const void* v,
  *          d_v = 64, KDN_CHUNK_AUTO takes the token-recurrent kernel and
  *          KDN_CHUNK_64 returns KDN_ERR_UNSUPPORTED)
  * workspace   device scratch of >= kdn_forward_varlen_workspace_size(...)
- *             bytes (at least 256), 256-byte aligned
+ *             bytes (at least 256), 256-byte aligned: the error word, then
+ *             (chunked engine) the sequence order
  * total >= 0, N >= 1.  Other arguments and errors as kdn_iso_forward.
  * ---------------------------------------------------------------------- */
 size_t kdn_forward_varlen_workspace_size(kdn_variant variant, int N, int H,

@@ -1105,6 +1105,71 @@ __device__ __forceinline__ bool bar_group_or(int id, bool flag) {
 
 constexpr int kTeamA = 6, kTeamB = 7;
 
+// Longest-first order of packed sequences.  The engine holds one CTA per SM,
+// so when there are more (sequence, head) problems than SMs the hardware
+// starts them in waves; a long sequence that starts in a late wave sets the
+// end of the launch.  Starting them longest first (list scheduling by longest
+// processing time, Graham 1969) bounds the launch by 4/3 of the best schedule.
+// One CTA counting-sorts the sequences by their number of chunks, descending;
+// equal counts land in any order, which changes no result (a sequence's
+// arithmetic does not depend on the CTA that runs it).  order[] receives a
+// permutation of [0, N) whatever cu_seqlens holds: lengths are clamped as
+// the engine clamps them, and the engine reports bad offsets itself.
+constexpr int kOrderBuckets = 4096, kOrderThreads = 1024;
+
+__device__ __forceinline__ int order_bucket(const int* __restrict__ cu, int s, int T) {
+  const int s0 = min(max(cu[s], 0), T);
+  const int n = min(max(cu[s + 1], s0), T) - s0;
+  return kOrderBuckets - 1 - min((n + kC - 1) / kC, kOrderBuckets - 1);  // 0: longest
+}
+
+__global__ void __launch_bounds__(kOrderThreads)
+varlen_order_kernel(const int* __restrict__ cu, int N, int T, int* __restrict__ order) {
+  constexpr int kPer = kOrderBuckets / kOrderThreads;
+  __shared__ int start[kOrderBuckets];
+  __shared__ int wsum[kOrderThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  for (int i = tid; i < kOrderBuckets; i += kOrderThreads) start[i] = 0;
+  __syncthreads();
+  for (int s = tid; s < N; s += kOrderThreads) atomicAdd(&start[order_bucket(cu, s, T)], 1);
+  __syncthreads();
+  // exclusive prefix sum of the bucket counts: kPer buckets per thread, then
+  // a warp scan and a scan of the warp totals
+  int c[kPer], run = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    c[j] = start[tid * kPer + j];
+    run += c[j];
+  }
+  int x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int y = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int z = __shfl_up_sync(0xffffffffu, y, o);
+      if (lane >= o) y += z;
+    }
+    wsum[lane] = y;
+  }
+  __syncthreads();
+  int base = x - run + (wid ? wsum[wid - 1] : 0);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    start[tid * kPer + j] = base;
+    base += c[j];
+  }
+  __syncthreads();
+  for (int s = tid; s < N; s += kOrderThreads)
+    order[atomicAdd(&start[order_bucket(cu, s, T)], 1)] = s;
+}
+
 // PACKED: the B "batch entries" are packed sequences given by cu_seqlens (the
 // instantiation for ordinary [B, T, H, d] tensors carries none of its code).
 template <bool DIAG, bool PACKED>
@@ -1118,14 +1183,16 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const float* S0, const float* __restrict__ P0, float* __restrict__ O,
                        float* S_out, float* __restrict__ P_out, int T, int H, float kappa,
                        uint32_t* __restrict__ err, int debug_skip_v,
-                       const int* __restrict__ cu_seqlens) {
+                       const int* __restrict__ cu_seqlens, const int* __restrict__ order) {
   using P = WsPlan<DIAG>;
   constexpr int DV = 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x;
+  // packed sequences may be taken longest first: CTA i runs sequence order[i / H]
+  const int bh = PACKED && order ? order[blockIdx.x / H] * H + (int)(blockIdx.x % H)
+                                 : (int)blockIdx.x;
   const int h = bh % H;
   // This CTA's sequence: batch entry b of [B, T, H, d] tensors, or (packed
   // sequences, cu_seqlens given) tokens [tbeg, tbeg + Tn) of [1, T, H, d] ones.
@@ -2174,9 +2241,22 @@ kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a
     attr_set[cu_seqlens ? 1 : 0] = true;
   }
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
+  // packed sequences: longest first once the problems outnumber the SMs (the
+  // order goes after the error word; the workspace holds B * H floats there)
+  int* order = nullptr;
+  if (cu_seqlens) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return KDN_ERR_CUDA;
+    if (B * H > sms) {
+      order = reinterpret_cast<int*>(static_cast<char*>(ws) + 256);
+      varlen_order_kernel<<<1, kOrderThreads, 0, s>>>(cu_seqlens, B, T, order);
+    }
+  }
   kern<<<(unsigned)(B * H), kThreads, P::ALLOC, s>>>(
       mq, mk, mv, mo, mw, a, w, r, S0, p0, o, S_out, p_out, T, H, kappa,
-      static_cast<uint32_t*>(ws), debug_skip_v, cu_seqlens);
+      static_cast<uint32_t*>(ws), debug_skip_v, cu_seqlens, order);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 

@@ -23,6 +23,9 @@ The named workloads mirror the five benchmark configurations of this library:
   'diag_long'   diagonal layer, bf16, B1 T65536 H16 d128, seed 4, followed by
                 512 decode steps at batch 256 from S ~ N(0, 0.02^2),
                 p ~ U(0.1, 1)
+  'iso_varlen'  isotropic layer, bf16, H16 d128, 32768 tokens packed from
+                sequences of log-uniform length in [64, 4096] (``packed_lengths``,
+                seed 5), the same token count as 'iso_1p3b'
 """
 from __future__ import annotations
 
@@ -35,6 +38,8 @@ WORKLOADS = {
     'diag_1p3b': dict(variant='diag', B=8, T=4096, H=16, dk=128, dv=128, dtype='bf16', seed=3),
     'diag_long': dict(variant='diag', B=1, T=65536, H=16, dk=128, dv=128, dtype='bf16', seed=4,
                       decode_batch=256, decode_steps=512),
+    'iso_varlen': dict(variant='iso', total=32768, H=16, dk=128, dv=128, dtype='bf16', seed=5,
+                       min_len=64, max_len=4096),
 }
 
 _DT = {'f32': torch.float32, 'bf16': torch.bfloat16}
@@ -108,3 +113,24 @@ def decode_inputs(B, H, dk, dv, variant='diag', seed=0, dtype='bf16'):
     [B,H,dk]."""
     x = layer_inputs(B, 1, H, dk, dv, variant, seed, dtype)
     return {name: t[:, 0] for name, t in x.items()}
+
+
+def packed_lengths(total, seed=0, min_len=64, max_len=4096):
+    """Sequence lengths for a packed batch of ``total`` tokens.
+
+    Lengths are drawn log-uniform in [min_len, max_len] (a long-tailed mix of
+    short and long documents), rounded down to integers, until the next one
+    would pass ``total``; the last sequence takes what is left, so the list
+    sums to ``total`` exactly and only its last entry may be below
+    ``min_len``.  Returns a list of ints.
+    """
+    import math
+    g = _gen(seed)
+    lo, hi = math.log(min_len), math.log(max_len)
+    out, left = [], int(total)
+    while left > 0:
+        u = float(torch.rand((), generator=g, dtype=torch.float64))
+        n = min(int(math.exp(lo + u * (hi - lo))), left)
+        out.append(n)
+        left -= n
+    return out

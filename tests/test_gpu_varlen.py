@@ -83,6 +83,62 @@ def test_varlen_equal_lengths_agree_with_dense(variant):
     torch.testing.assert_close(p_v, p_d, rtol=1e-6, atol=0)
 
 
+def _sm_count():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("variant", ["iso", "diag"])
+def test_varlen_many_sequences_longest_first(variant):
+    """More (sequence, head) problems than SMs: the engine takes the
+    sequences longest first, and every sequence still lands in its own rows
+    of o, S_T and p_T.  Lengths mix zeros, ragged tails and full chunks."""
+    H, d = 2, 128
+    N = _sm_count() // H + 12
+    g = np.random.default_rng(41)
+    lengths = [int(n) for n in g.integers(0, 150, size=N)]
+    lengths[3] = 0
+    lengths[N - 1] = 300  # the longest one last in the packing
+    x, cu = _packed(variant, lengths, H, d, d, 'bf16', seed=43)
+    gt = torch.Generator().manual_seed(44)
+    S0 = 0.05 * torch.randn(N, H, d, d, generator=gt)
+    p0 = torch.rand((N, H) if variant == 'iso' else (N, H, d), generator=gt) + 0.2
+    xd = {k: v.cuda() for k, v in x.items()}
+    var = kdn.KDN_ISO if variant == 'iso' else kdn.KDN_DIAG
+    ws = torch.empty(kdn.kdn_forward_varlen_workspace_size(var, N, H, d, d), dtype=torch.uint8,
+                     device='cuda')
+    o, S, p = kdn.kdn_forward_varlen(var, xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'],
+                                     cu.cuda(), S0.cuda(), p0.cuda(), workspace=ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_OK
+    o_r, S_r, p_r = _oracle(variant, x, cu, S0, p0)
+    assert rel_maxabs(o, o_r) <= OUT_TOL
+    for s in range(N):  # per sequence, so that a swapped pair of rows fails
+        assert rel_maxabs(S[s], S_r[s]) <= STATE_TOL, s
+    np.testing.assert_allclose(f64(p), p_r, rtol=1e-5)
+    assert torch.equal(S[3].cpu(), S0[3]) and torch.equal(p[3].cpu(), p0[3])
+
+
+@pytest.mark.parametrize("variant", ["iso", "diag"])
+def test_varlen_longest_first_is_bitwise_the_dense_result(variant):
+    """With the launch order permuted (more problems than SMs, unequal
+    lengths), each sequence's results are bit for bit those of the dense
+    call on that sequence alone: the order moves work, not arithmetic."""
+    H, d = 2, 128
+    N = _sm_count() // H + 4
+    lengths = [64 + 37 * (i % 5) for i in range(N)]
+    x, cu = _packed(variant, lengths, H, d, d, 'bf16', seed=47)
+    xd = {k: v.cuda() for k, v in x.items()}
+    var = kdn.KDN_ISO if variant == 'iso' else kdn.KDN_DIAG
+    o, S, p = kdn.kdn_forward_varlen(var, xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'],
+                                     cu.cuda())
+    fwd = kdn.kdn_iso_forward if variant == 'iso' else kdn.kdn_diag_forward
+    for s in (0, 1, 2, 3, 4, N - 1):
+        lo, hi = int(cu[s]), int(cu[s + 1])
+        one = {k: v[lo:hi][None].clone() for k, v in xd.items()}  # aligned copies
+        o1, S1, p1 = fwd(one['q'], one['k'], one['v'], one['a'], one['w'], one['r'])
+        assert torch.equal(o[lo:hi], o1[0]), s
+        assert torch.equal(S[s], S1[0]) and torch.equal(p[s], p1[0]), s
+
+
 def test_varlen_bad_offsets_are_clamped_and_reported():
     """Offsets out of order are clamped (the sequence is empty) and the
     workspace reports KDN_ERR_INVALID_ARG."""

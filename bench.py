@@ -14,7 +14,8 @@ Also measured on the same run and reported under "secondary": the Diagonal
 KDN forward at the same shape, the standalone variance scan (4096 x 65536),
 the long-context diagonal forward (B1 T65536), the decode step (batch 256) and
 the isotropic forward over 32768 tokens packed from sequences of mixed length
-(kdn_forward_varlen).
+(kdn_forward_varlen), and the dense (full-covariance) filter at d_k = d_v = 64
+(kdn_exact_forward).
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores.
@@ -255,7 +256,7 @@ def main():
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
-    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen'],
+    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact'],
                     help='run only this kernel (for profiler captures) and print its timing')
     ap.add_argument('--B', type=int, default=None, help='batch override for --only')
     ap.add_argument('--T', type=int, default=None, help='length override for --only')
@@ -408,6 +409,8 @@ def run_only(args):
         units, alg = N * T, N * T * 20
     elif args.only == 'varlen':
         f, units, alg, _ = varlen_case(kdn, synth, dev)
+    elif args.only == 'exact':
+        f, units, alg, _ = exact_case(kdn, synth, dev, args.B, args.T)
     else:
         c = synth.WORKLOADS['diag_long']
         B = args.B or c['decode_batch']
@@ -447,6 +450,29 @@ def varlen_case(kdn, synth, dev):
     desc = {'sequences': N, 'tokens': total, 'max_len': max(lengths),
             'min_len': min(lengths), 'H': H, 'd': d}
     return f, total, alg, desc
+
+
+def exact_bytes(B, T, H, dk, dv, in_bytes=2):
+    """Algorithmic HBM bytes of the dense filter (W = w I): read q, k, v, a,
+    w, r; write o (fp32), S_T and P_T."""
+    return (B * T * H * ((2 * dk + dv) * in_bytes + 3 * 4 + dv * 4) +
+            B * H * (dv * dk + dk * dk) * 4)
+
+
+def exact_case(kdn, synth, dev, B=None, T=None):
+    """The dense filter: (launch fn, tokens, algorithmic bytes, description)."""
+    import torch
+    c = synth.WORKLOADS['exact_d64']
+    B, T = B or c['B'], T or c['T']
+    H, dk, dv = c['H'], c['dk'], c['dv']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, dk, dv, c['variant'], c['seed'],
+                                                     c['dtype']).items()}
+    o = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    S = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    P = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    f = lambda: kdn.kdn_exact_forward(c['variant'], x['q'], x['k'], x['v'], x['a'], x['w'],
+                                      x['r'], o=o, S_out=S, P_out=P)
+    return f, B * T, exact_bytes(B, T, H, dk, dv), {'B': B, 'T': T, 'H': H, 'dk': dk, 'dv': dv}
 
 
 def measure_secondary(kdn, synth, dev, stream, hbm_peak):
@@ -521,6 +547,13 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     out['iso_varlen'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
                          'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                          'algorithmic_bytes': alg, **desc}
+    # dense (full-covariance) filter, B8 T4096 H16 d64
+    f, units, alg, desc = exact_case(kdn, synth, dev)
+    n = 3
+    ms = time_launches(f, n, 3, stream) / n
+    out['exact_d64'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
+                        'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                        'algorithmic_bytes': alg, **desc}
     return out
 
 

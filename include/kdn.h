@@ -295,6 +295,41 @@ kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k,
                            float info_scale, void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_exact_forward -- the dense (full-covariance) Kalman filter of the same
+ * memory model, for small d_k: every row of S shares one d_k x d_k covariance
+ * P, carried exactly by the Riccati recursion instead of being projected to a
+ * scalar or a diagonal.  The pages name this exact filter as what the KDN
+ * projection approximates ("Kalman Delta Networks: Uncertainty-aware
+ * Associative Memory", abstract; "Kalman Delta Networks: 不确定性感知的联想
+ * 记忆", 局限), so this call measures the projection's error.  Per token:
+ *   P- = a^2 P + W,  u = P- k,  s = k.u + r,  g = u / s,
+ *   S <- a S + (v - a S k) g^T,  o = S q,  P = P- - u u^T / s
+ * with W = w I (variant KDN_ISO) or diag(w) (KDN_DIAG).  There is no
+ * information scale: nothing is projected.
+ *
+ * q, k     [B, T, H, dk] in_dtype device;  v [B, T, H, dv] in_dtype device
+ * a, r     [B, T, H] fp32 device
+ * w        [B, T, H] (iso) or [B, T, H, dk] (diag) fp32 device
+ * S0       [B, H, dv, dk] fp32 device, or NULL for zeros
+ * P0       [B, H, dk, dk] fp32 device, or NULL for the identity; only its
+ *          symmetric part (P0 + P0^T) / 2 is used
+ * o        [B, T, H, dv] fp32 device output
+ * S_out    [B, H, dv, dk];  P_out [B, H, dk, dk] fp32 device outputs; they
+ *          may alias S0 and P0 (each head reads its state before writing)
+ * Supported: dk in {32, 64}; 8 <= dv <= 128 with dv a multiple of 8; every
+ * pointer 16-byte aligned.  KDN_ERR_UNSUPPORTED for other sizes.  One CTA
+ * per (b, h) runs the T tokens in order; no workspace, no on-device waits.
+ * Errors: KDN_ERR_INVALID_ARG (NULL, shape, alignment, variant or dtype),
+ * KDN_ERR_CUDA (launch).
+ * ---------------------------------------------------------------------- */
+kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k,
+                             const void* v, kdn_dtype in_dtype, const float* a,
+                             const float* w, const float* r, const float* S0,
+                             const float* P0, float* o, float* S_out,
+                             float* P_out, int B, int T, int H, int dk, int dv,
+                             void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_read_workspace_status -- synchronise `stream`, then report the device
  * error word a previous call left in `workspace`: KDN_OK, KDN_ERR_TIMEOUT
  * if a bounded on-device wait gave up, or KDN_ERR_INVALID_ARG if packed-

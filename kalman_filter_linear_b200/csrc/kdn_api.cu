@@ -31,6 +31,11 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
                                int T, int H, int dv, float kappa, void* workspace,
                                cudaStream_t s, int debug_skip_v = -1,
                                const int* cu_seqlens = nullptr);
+bool exact_kalman_supported(int dk, int dv);
+kdn_status exact_kalman_launch(bool diag, kdn_dtype dt, const void* q, const void* k,
+                               const void* v, const float* a, const float* w, const float* r,
+                               const float* S0, const float* P0, float* o, float* S_out,
+                               float* P_out, int B, int T, int H, int dk, int dv, cudaStream_t s);
 }  // namespace kdn
 
 namespace {
@@ -254,6 +259,22 @@ kdn_status kdn_decode_step(kdn_variant variant, const void* q, const void* k, co
   const float kappa = info_scale > 0.f ? info_scale : 1.f / (float)dk;
   return kdn::recurrent_launch(variant == KDN_DIAG, in_dtype, q, k, v, a, w, r, S, p, o, S, p, B,
                                1, H, dk, dv, kappa, as_stream(stream));
+}
+
+kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k, const void* v,
+                             kdn_dtype in_dtype, const float* a, const float* w, const float* r,
+                             const float* S0, const float* P0, float* o, float* S_out,
+                             float* P_out, int B, int T, int H, int dk, int dv, void* stream) {
+  if (!q || !k || !v || !a || !w || !r || !o || !S_out || !P_out) return KDN_ERR_INVALID_ARG;
+  if (variant != KDN_ISO && variant != KDN_DIAG) return KDN_ERR_INVALID_ARG;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(a) || !al16(w) || !al16(r) || !al16(o) ||
+      !al16(S_out) || !al16(P_out) || !al16_or_null(S0) || !al16_or_null(P0))
+    return KDN_ERR_INVALID_ARG;
+  if (!kdn::exact_kalman_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
+  return kdn::exact_kalman_launch(variant == KDN_DIAG, in_dtype, q, k, v, a, w, r, S0, P0, o,
+                                  S_out, P_out, B, T, H, dk, dv, as_stream(stream));
 }
 
 size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,

@@ -73,6 +73,8 @@ def lib():
     L.kdn_decode_step.restype = _i32
     L.kdn_decode_step.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 6 + [_i32] * 4 + \
         [_f32, _vp]
+    L.kdn_exact_forward.restype = _i32
+    L.kdn_exact_forward.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
     L.kdn_read_workspace_status.restype = _i32
     L.kdn_read_workspace_status.argtypes = [_vp, _sz, _vp]
     L.kdn_testing_mobius_scan_unpublished_tile.restype = _i32
@@ -368,6 +370,39 @@ def kdn_decode_step(variant, q, k, v, a, w, r, S, p, o=None, info_scale=0.0):
                                float(info_scale), _stream())
     _check(st, 'kdn_decode_step')
     return o
+
+
+def kdn_exact_forward(variant, q, k, v, a, w, r, S0=None, P0=None, o=None, S_out=None,
+                      P_out=None):
+    """The dense (full-covariance) Kalman filter: q, k [B,T,H,dk], v [B,T,H,dv],
+    a, r [B,T,H], w [B,T,H] (iso: W = w I) or [B,T,H,dk] (diag: W = diag(w)).
+    Returns (o [B,T,H,dv], S_T [B,H,dv,dk], P_T [B,H,dk,dk])."""
+    var = KDN_DIAG if variant in ('diag', KDN_DIAG) else KDN_ISO
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _in_dtype(q)
+    _req(q, 'q', dt)
+    _req(k, 'k', dt, (B, T, H, dk))
+    _req(v, 'v', dt, (B, T, H, dv))
+    f = torch.float32
+    _req(a, 'a', f, (B, T, H))
+    _req(r, 'r', f, (B, T, H))
+    _req(w, 'w', f, (B, T, H) if var == KDN_ISO else (B, T, H, dk))
+    _opt(S0, 'S0', f, (B, H, dv, dk))
+    _opt(P0, 'P0', f, (B, H, dk, dk))
+    dev = q.device
+    o = _req(o, 'o', f, (B, T, H, dv)) if o is not None else \
+        torch.empty((B, T, H, dv), dtype=f, device=dev)
+    S_out = _req(S_out, 'S_out', f, (B, H, dv, dk)) if S_out is not None else \
+        torch.empty((B, H, dv, dk), dtype=f, device=dev)
+    P_out = _req(P_out, 'P_out', f, (B, H, dk, dk)) if P_out is not None else \
+        torch.empty((B, H, dk, dk), dtype=f, device=dev)
+    st = lib().kdn_exact_forward(var, _ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w),
+                                 _ptr(r), _ptr(S0), _ptr(P0), _ptr(o), _ptr(S_out), _ptr(P_out),
+                                 B, T, H, dk, dv, _stream())
+    _check(st, 'kdn_exact_forward')
+    return o, S_out, P_out
 
 
 def kdn_read_workspace_status(workspace):

@@ -26,6 +26,8 @@ The named workloads mirror the five benchmark configurations of this library:
   'iso_varlen'  isotropic layer, bf16, H16 d128, 32768 tokens packed from
                 sequences of log-uniform length in [64, 4096] (``packed_lengths``,
                 seed 5), the same token count as 'iso_1p3b'
+  'exact_d64'   dense (full-covariance) filter, bf16, B8 T4096 H16 d_k = d_v = 64,
+                W = w I, seed 6
 """
 from __future__ import annotations
 
@@ -40,6 +42,7 @@ WORKLOADS = {
                       decode_batch=256, decode_steps=512),
     'iso_varlen': dict(variant='iso', total=32768, H=16, dk=128, dv=128, dtype='bf16', seed=5,
                        min_len=64, max_len=4096),
+    'exact_d64': dict(variant='iso', B=8, T=4096, H=16, dk=64, dv=64, dtype='bf16', seed=6),
 }
 
 _DT = {'f32': torch.float32, 'bf16': torch.bfloat16}

@@ -115,3 +115,22 @@ def test_decode_rejects_bad_arguments(L):
     assert d(H=0) == kdn.KDN_ERR_INVALID_ARG
     assert d(dk=48) == kdn.KDN_ERR_UNSUPPORTED
     assert L.kdn_read_workspace_status(None, 0, None) == kdn.KDN_ERR_INVALID_ARG
+
+
+def test_exact_forward_rejects_bad_arguments(L):
+    base = dict(var=kdn.KDN_ISO, q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_F32, a=FAKE, w=FAKE, r=FAKE,
+                S0=None, P0=None, o=FAKE, S=FAKE, P=FAKE, B=1, T=8, H=1, dk=64, dv=64,
+                stream=None)
+    x = lambda **kw: L.kdn_exact_forward(*dict(base, **kw).values())
+    assert x(q=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(P=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(var=7) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dt=9) == kdn.KDN_ERR_INVALID_ARG
+    assert x(T=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(B=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(P0=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert x(o=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dk=128) == kdn.KDN_ERR_UNSUPPORTED   # small d_k only
+    assert x(dk=16) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(dv=12) == kdn.KDN_ERR_UNSUPPORTED    # d_v a multiple of 8
+    assert x(dv=136) == kdn.KDN_ERR_UNSUPPORTED

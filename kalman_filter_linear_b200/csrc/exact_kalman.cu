@@ -14,24 +14,31 @@
 //   P  = P- - u u^T / s
 // It is the reference for the projection's approximation error at small d_k.
 //
-// One CTA of 8 warps per (b, h).  Warp w holds rows w, w + 8, ... of S and of
-// P in registers; lane l holds columns [l CPL, (l + 1) CPL), CPL = d_k / 32.
-//  - u = P- k is formed as column sums (P- is symmetric): each warp sums its
-//    own rows and the 8 partial vectors meet in shared memory, the one block
-//    barrier per token.
-//  - P stays exactly symmetric: P-_ij and P-_ji are computed from the same
-//    operands, and so are u_i u_j and u_j u_i; s is the same in every warp.
-//  - The row sums S k and S q of a warp's rows are reduced across the lanes
-//    by recursive halving (each exchange step halves the values a lane keeps),
-//    2 RPW values in about 2 RPW shuffles rather than 5 per value.
-//  - Inputs come into shared memory by cp.async in chunks of 16 tokens, one
-//    chunk ahead of the compute; outputs leave per chunk in coalesced rows.
+// One CTA per (b, h).  Every matrix row is held by SPLIT = d_k / 32 adjacent
+// lanes, 32 columns each, so the per-row products run inside the lanes and
+// one xor shuffle joins the halves.  The covariance recursion does not read
+// S, so it runs on its own warps, one 16-token chunk ahead of the state:
+//  - Covariance warps (d_k SPLIT / 32 of them): half h of row i holds
+//    Pr[c'] = P[i][(i + SPLIT c' + h) mod d_k], the row rotated by i, so the
+//    diagonal that W touches is always register 0 of half 0.
+//    u_i = sum_c P-[i][i + c] k[i + c] reads k rotated from shared memory,
+//    where k is stored twice in a row so that the reads of a lane are fixed
+//    offsets from one address (distinct lanes, distinct banks).  k.u and q.u
+//    are reduced across the lanes and warps, g = u / s and g.q = q.u / s go
+//    to shared memory for the state warps, and P is updated with u read
+//    rotated the same way.  P stays exactly symmetric: entry (i, j) and
+//    (j, i) are formed from the same operands in the same order.
+//  - State warps: half h of row j holds S[j][32 h + c'].  S k and S q are
+//    in-lane dot products with k and q read as broadcasts; the update
+//    S_j <- a S_j + e_j g likewise.
+//  - Inputs come into shared memory by cp.async in chunks of 16 tokens, three
+//    stages deep; outputs leave per chunk in coalesced rows.
 #include "kdn_common.cuh"
 
 namespace kdn {
 namespace {
 
-constexpr int kXWarps = 8, kXThreads = kXWarps * 32, kTC = 16;
+constexpr int kTC = 16;  // tokens per chunk
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
@@ -48,79 +55,79 @@ __device__ __forceinline__ void cp_async_wait_newest_pending() {
   asm volatile("cp.async.wait_group 1;" ::: "memory");
 }
 
-// One recursive-halving step at lane offset O over n values: a lane with bit
-// O set keeps the upper half, its partner the lower half; each adds what the
-// partner sends.
-template <int N, int O>
-__device__ __forceinline__ void halve(float* x, int lane) {
-  const bool up = (lane & O) != 0;
-#pragma unroll
-  for (int i = 0; i < N / 2; ++i) {
-    const float send = up ? x[i] : x[i + N / 2];
-    const float keep = up ? x[i + N / 2] : x[i];
-    x[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+// barrier of the covariance warps only (named barrier 1)
+template <int NT>
+__device__ __forceinline__ void pbar() {
+  if constexpr (NT == 32) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
   }
 }
 
-// Sums item i of x[N] over the 32 lanes; afterwards every lane l holds the
-// total of item l / (32 / N).  N in {8, 16, 32}.
-template <int N>
-__device__ __forceinline__ float transpose_sum(float (&x)[N], int lane) {
-  static_assert(N == 8 || N == 16 || N == 32, "items per lane");
-  halve<N, 16>(x, lane);
-  halve<N / 2, 8>(x, lane);
-  halve<N / 4, 4>(x, lane);
-  if constexpr (N >= 16) halve<N / 8, 2>(x, lane);
-  if constexpr (N >= 32) halve<N / 16, 1>(x, lane);
-  float y = x[0];
-  if constexpr (N <= 16) y += __shfl_xor_sync(0xffffffffu, y, 1);
-  if constexpr (N <= 8) y += __shfl_xor_sync(0xffffffffu, y, 2);
-  return y;
-}
-
-// Shared-memory plan of one CTA (bytes): two input stages, the partial sums
-// of u (two buffers, by token parity) and the output rows of one chunk.
-template <int DK, int RPW, bool DIAG, typename InT>
+// Shared-memory plan of one CTA (bytes).
+template <int DK, int SW, bool DIAG, typename InT>
 struct XPlan {
-  static constexpr int DVP = RPW * kXWarps;                 // d_v rounded up
-  static constexpr int KQ = kTC * 2 * DK * (int)sizeof(InT);  // [t][k | q]
+  static constexpr int SPLIT = DK / 32;                       // lanes per row
+  static constexpr int PW = DK * SPLIT / 32;                  // covariance warps
+  static constexpr int DVP = SW * 32 / SPLIT;                 // d_v rounded up
+  static constexpr int KQ = kTC * 2 * DK * (int)sizeof(InT);  // [t][k | q] as read
   static constexpr int VB = kTC * DVP * (int)sizeof(InT);     // [t][v]
   static constexpr int WN = DIAG ? DK : 1;
   static constexpr int F32 = kTC * (2 + WN) * 4;              // a[t], r[t], w[t][WN]
   static constexpr int STAGE = (KQ + VB + F32 + 15) / 16 * 16;
-  static constexpr int OFF_RED = 2 * STAGE;
-  static constexpr int OFF_OUT = OFF_RED + 2 * kXWarps * DK * 4;
-  static constexpr int TOTAL = OFF_OUT + kTC * DVP * 4;
+  static constexpr int OFF_KQF = 3 * STAGE;                   // [2][kTC][k | q] fp32
+  static constexpr int OFF_G = OFF_KQF + 2 * kTC * 2 * DK * 4;  // [2][kTC][DK] gains
+  static constexpr int OFF_KD = OFF_G + 2 * kTC * DK * 4;       // [kTC][2 DK] k, k again
+  static constexpr int OFF_U = OFF_KD + kTC * 2 * DK * 4;       // [2][2 DK] u, u again, by parity
+  static constexpr int OFF_GQ = OFF_U + 2 * 2 * DK * 4;         // [2][kTC] g.q
+  static constexpr int OFF_RED = OFF_GQ + 2 * kTC * 4;          // [2][PW][2] k.u, q.u
+  static constexpr int OFF_OUT = (OFF_RED + 2 * PW * 2 * 4 + 15) / 16 * 16;  // [2][kTC][DVP]
+  static constexpr int TOTAL = OFF_OUT + 2 * kTC * DVP * 4;
 };
 
-template <int DK, int RPW, bool DIAG, typename InT>
-__global__ void __launch_bounds__(kXThreads)
+template <int DK, int SW, bool DIAG, typename InT>
+__global__ void __launch_bounds__((DK * DK / 1024 + SW) * 32)
 exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
                     const InT* __restrict__ V, const float* __restrict__ A,
                     const float* __restrict__ Wn, const float* __restrict__ R, const float* S0,
                     const float* P0, float* __restrict__ O, float* S_out, float* P_out, int T,
                     int H, int dv) {
-  using X = XPlan<DK, RPW, DIAG, InT>;
-  constexpr int CPL = DK / 32;   // columns per lane
-  static_assert(CPL == 1 || CPL == 2, "d_k 32 or 64");
-  constexpr int PR = DK / kXWarps;  // rows of P per warp
-  constexpr int N = 2 * RPW;     // row sums per warp and token: S k, then S q
-  constexpr int G = 32 / N;      // lanes that share one row sum
+  using X = XPlan<DK, SW, DIAG, InT>;
+  constexpr int PW = X::PW, SPLIT = X::SPLIT, NTH = (PW + SW) * 32, M = DK - 1;
   extern __shared__ __align__(16) uint8_t xsm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool pwarp = warp < PW;
+  const int rt = pwarp ? tid : tid - PW * 32;
+  const int row = rt / SPLIT, hf = rt % SPLIT;  // row of P or S, and which half of it
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
-  float* red = reinterpret_cast<float*>(xsm + X::OFF_RED);  // [2][8][DK]
-  float* obuf = reinterpret_cast<float*>(xsm + X::OFF_OUT);  // [kTC][DVP]
+  float* kqf = reinterpret_cast<float*>(xsm + X::OFF_KQF);
+  float* gring = reinterpret_cast<float*>(xsm + X::OFF_G);
+  float* ubuf = reinterpret_cast<float*>(xsm + X::OFF_U);
+  float* kdup = reinterpret_cast<float*>(xsm + X::OFF_KD);
+  float* gqring = reinterpret_cast<float*>(xsm + X::OFF_GQ);
+  float* red = reinterpret_cast<float*>(xsm + X::OFF_RED);
+  float* obuf = reinterpret_cast<float*>(xsm + X::OFF_OUT);
 
-  // stage the inputs of tokens [16 c, 16 c + 16) into buffer c & 1
+  struct Stage {
+    const InT* kq;
+    const InT* v;
+    const float* f;
+  };
+  auto stage = [&](int c) {
+    const uint8_t* st = xsm + (c % 3) * X::STAGE;
+    return Stage{reinterpret_cast<const InT*>(st), reinterpret_cast<const InT*>(st + X::KQ),
+                 reinterpret_cast<const float*>(st + X::KQ + X::VB)};
+  };
+  // stage the inputs of tokens [16 c, 16 c + 16) into buffer c % 3
   auto issue = [&](int c) {
-    uint8_t* st = xsm + (c & 1) * X::STAGE;
+    uint8_t* st = xsm + (c % 3) * X::STAGE;
     InT* skq = reinterpret_cast<InT*>(st);
     InT* sv = reinterpret_cast<InT*>(st + X::KQ);
     float* sf = reinterpret_cast<float*>(st + X::KQ + X::VB);
     const int t0 = c * kTC, nt = min(kTC, T - t0);
     constexpr int PK = DK * (int)sizeof(InT) / 16;  // 16-byte pieces of one k row
-    for (int i = tid; i < nt * 2 * PK; i += kXThreads) {
+    for (int i = tid; i < nt * 2 * PK; i += NTH) {
       const int t = i / (2 * PK), p = i % (2 * PK), half = p / PK, pp = p % PK;
       const size_t tok = ((size_t)b * T + t0 + t) * H + h;
       const InT* src = (half ? Q : K) + tok * DK;
@@ -128,22 +135,22 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
                  reinterpret_cast<const uint8_t*>(src) + pp * 16);
     }
     const int pv = dv * (int)sizeof(InT) / 16;
-    for (int i = tid; i < nt * pv; i += kXThreads) {
+    for (int i = tid; i < nt * pv; i += NTH) {
       const int t = i / pv, pp = i % pv;
       const size_t tok = ((size_t)b * T + t0 + t) * H + h;
       cp_async16(sv + t * X::DVP + pp * (16 / (int)sizeof(InT)),
                  reinterpret_cast<const uint8_t*>(V + tok * dv) + pp * 16);
     }
     if constexpr (DIAG) {
-      constexpr int PW = DK * 4 / 16;
-      for (int i = tid; i < nt * PW; i += kXThreads) {
-        const int t = i / PW, pp = i % PW;
+      constexpr int PWN = DK * 4 / 16;
+      for (int i = tid; i < nt * PWN; i += NTH) {
+        const int t = i / PWN, pp = i % PWN;
         const size_t tok = ((size_t)b * T + t0 + t) * H + h;
         cp_async16(sf + 2 * kTC + t * DK + pp * 4, Wn + tok * DK + pp * 4);
       }
     }
-    if (tid < 3 * nt) {
-      const int which = tid / nt, t = tid % nt;
+    for (int i = tid; i < 3 * nt; i += NTH) {
+      const int which = i / nt, t = i % nt;
       const size_t tok = ((size_t)b * T + t0 + t) * H + h;
       if (which == 0) cp_async4(sf + t, A + tok);
       else if (which == 1) cp_async4(sf + kTC + t, R + tok);
@@ -153,172 +160,204 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
 
   // ---- state into registers.  S_out may alias S0 and P_out P0: every read
   // of the initial state comes before the barrier that precedes the stores.
-  float S[RPW][CPL], P[PR][CPL];
+  // covariance warps: Pr[c'] = P[row][(row + SPLIT c' + hf) mod DK];
+  // state warps: S[row][32 hf + c']
+  float X_[32];
   const size_t s_base = (size_t)bh * dv * DK, p_base = (size_t)bh * DK * DK;
+  if (pwarp) {
 #pragma unroll
-  for (int i = 0; i < RPW; ++i) {
-    const int j = warp + kXWarps * i;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c)
-      S[i][c] = (S0 && j < dv) ? S0[s_base + (size_t)j * DK + lane * CPL + c] : 0.f;
-  }
-#pragma unroll
-  for (int m = 0; m < PR; ++m) {
-    const int i = warp + kXWarps * m;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int j = lane * CPL + c;
+    for (int c = 0; c < 32; ++c) {
+      const int j = (row + SPLIT * c + hf) & M;
       // the symmetric part of P0: the same value at (i, j) and (j, i)
-      P[m][c] = P0 ? 0.5f * (P0[p_base + (size_t)i * DK + j] + P0[p_base + (size_t)j * DK + i])
-                   : (i == j ? 1.f : 0.f);
+      X_[c] = P0 ? 0.5f * (P0[p_base + (size_t)row * DK + j] + P0[p_base + (size_t)j * DK + row])
+                 : (c == 0 && hf == 0 ? 1.f : 0.f);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (S0 && row < dv)
+        x = *reinterpret_cast<const float4*>(S0 + s_base + (size_t)row * DK + 32 * hf + c);
+      X_[c] = x.x;
+      X_[c + 1] = x.y;
+      X_[c + 2] = x.z;
+      X_[c + 3] = x.w;
     }
   }
 
-  const int nchunks = (T + kTC - 1) / kTC;
-  if (nchunks > 0) issue(0);
-  cp_async_commit();
-  for (int ch = 0; ch < nchunks; ++ch) {
-    if (ch + 1 < nchunks) issue(ch + 1);  // its buffer was released by the barrier below
-    cp_async_commit();
-    cp_async_wait_newest_pending();       // chunk ch has landed (this thread's copies)
-    __syncthreads();                      // ... and everyone's
-    const uint8_t* st = xsm + (ch & 1) * X::STAGE;
-    const InT* skq = reinterpret_cast<const InT*>(st);
-    const InT* sv = reinterpret_cast<const InT*>(st + X::KQ);
-    const float* sf = reinterpret_cast<const float*>(st + X::KQ + X::VB);
-    const int t0 = ch * kTC, nt = min(kTC, T - t0);
+  // The covariance warps turn chunk cc's inputs into its gains and g.q, and
+  // leave k and q of the chunk in fp32 for the state warps.
+  auto gains = [&](int cc) {
+    const Stage st = stage(cc);
+    const int nt = min(kTC, T - cc * kTC);
+    float* kf = kqf + (cc & 1) * kTC * 2 * DK;
+    float* gout = gring + (cc & 1) * kTC * DK;
+    // k and q of the chunk in fp32 for the state warps, and k written twice
+    // in a row for the rotated reads here (no index wraps around)
+    for (int i = rt; i < nt * 2 * DK; i += PW * 32) {
+      const float x = to_f32(st.kq[i]);
+      kf[i] = x;
+      if ((i & (2 * DK - 1)) < DK) {
+        const int t = i / (2 * DK), j = i & M;
+        kdup[t * 2 * DK + j] = x;
+        kdup[t * 2 * DK + DK + j] = x;
+      }
+    }
+    pbar<PW * 32>();
     for (int t = 0; t < nt; ++t) {
-      const InT* kq = skq + t * 2 * DK;
-      float k[CPL], q[CPL], krow[PR];
+      const float* kt = kf + t * 2 * DK;  // k, then q
+      const float ki = kt[row], qi = kt[DK + row];
+      const float* krot = kdup + t * 2 * DK + row + hf;  // krot[SPLIT c] = k[(row + SPLIT c + hf) mod DK]
+      const float aa = st.f[t] * st.f[t], r = st.f[kTC + t];
+      const float wd = hf == 0 ? (DIAG ? st.f[2 * kTC + t * DK + row] : st.f[2 * kTC + t]) : 0.f;
+      float* ub = ubuf + (t & 1) * 2 * DK;
+      const float* urot = ub + row + hf;  // urot[SPLIT c] = u[(row + SPLIT c + hf) mod DK]
+      // P- = a^2 P + W (W on the diagonal: register 0 of half 0) and
+      // u_i = (P- k)_i; P- is formed again, identically, in the update
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        k[c] = to_f32(kq[lane * CPL + c]);
-        q[c] = to_f32(kq[DK + lane * CPL + c]);
+      for (int c = 0; c < 32; ++c)
+        acc[c & 3] = __fmaf_rn(__fmaf_rn(aa, X_[c], c == 0 ? wd : 0.f), krot[SPLIT * c],
+                               acc[c & 3]);
+      float u = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      if constexpr (SPLIT == 2) u += __shfl_xor_sync(0xffffffffu, u, 1);
+      if (hf == 0) {
+        ub[row] = u;
+        ub[DK + row] = u;
       }
+      // k.u and q.u, each row counted once (half 0)
+      const float ku = warp_sum(hf == 0 ? ki * u : 0.f), qu = warp_sum(hf == 0 ? qi * u : 0.f);
+      float* rd = red + (t & 1) * PW * 2;
+      if (lane == 0) {
+        rd[2 * warp] = ku;
+        rd[2 * warp + 1] = qu;
+      }
+      pbar<PW * 32>();  // u and the partial sums visible
+      float kus = 0.f, qus = 0.f;
 #pragma unroll
-      for (int m = 0; m < PR; ++m) krow[m] = to_f32(kq[warp + kXWarps * m]);
-      const float a = sf[t], r = sf[kTC + t], aa = a * a;
+      for (int w = 0; w < PW; ++w) {
+        kus += rd[2 * w];
+        qus += rd[2 * w + 1];
+      }
+      const float inv_s = __frcp_rn(kus + r);
+      if (hf == 0) gout[t * DK + row] = u * inv_s;
+      if (tid == 0) gqring[(cc & 1) * kTC + t] = qus * inv_s;
+      // P = P- - u u^T / s
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        X_[c] = __fmaf_rn(-__fmul_rn(u, urot[SPLIT * c]), inv_s,
+                          __fmaf_rn(aa, X_[c], c == 0 ? wd : 0.f));
+      // (u and the partial sums are double-buffered by token parity: the
+      // barrier of the next token orders this token's reads before their reuse)
+    }
+  };
 
-      // P- = a^2 P + W, and this warp's share of u = P- k (column sums)
-      float Pm[PR][CPL], part[CPL];
+  // The state warps run chunk cc's tokens through S with its gains.
+  auto states = [&](int cc) {
+    const Stage st = stage(cc);
+    const int nt = min(kTC, T - cc * kTC);
+    const float* kf = kqf + (cc & 1) * kTC * 2 * DK;
+    const float* gin = gring + (cc & 1) * kTC * DK;
+    float* ob = obuf + (cc & 1) * kTC * X::DVP;
+    for (int t = 0; t < nt; ++t) {
+      const float4* k4 = reinterpret_cast<const float4*>(kf + t * 2 * DK + 32 * hf);
+      const float4* q4 = reinterpret_cast<const float4*>(kf + t * 2 * DK + DK + 32 * hf);
+      float sk[2] = {0.f, 0.f}, sq[2] = {0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) part[c] = 0.f;
-#pragma unroll
-      for (int m = 0; m < PR; ++m) {
-        const int i = warp + kXWarps * m;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          const int j = lane * CPL + c;
-          const float wij = i == j ? (DIAG ? sf[2 * kTC + t * DK + i] : sf[2 * kTC + t]) : 0.f;
-          Pm[m][c] = __fmaf_rn(aa, P[m][c], wij);
-          part[c] = __fmaf_rn(Pm[m][c], krow[m], part[c]);
-        }
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 kk = k4[c4], qq = q4[c4];
+        const int p = c4 & 1;
+        sk[p] = __fmaf_rn(X_[4 * c4], kk.x, sk[p]);
+        sk[p] = __fmaf_rn(X_[4 * c4 + 1], kk.y, sk[p]);
+        sk[p] = __fmaf_rn(X_[4 * c4 + 2], kk.z, sk[p]);
+        sk[p] = __fmaf_rn(X_[4 * c4 + 3], kk.w, sk[p]);
+        sq[p] = __fmaf_rn(X_[4 * c4], qq.x, sq[p]);
+        sq[p] = __fmaf_rn(X_[4 * c4 + 1], qq.y, sq[p]);
+        sq[p] = __fmaf_rn(X_[4 * c4 + 2], qq.z, sq[p]);
+        sq[p] = __fmaf_rn(X_[4 * c4 + 3], qq.w, sq[p]);
       }
-      float* rd = red + (t & 1) * kXWarps * DK;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) rd[warp * DK + lane * CPL + c] = part[c];
-      __syncthreads();
-      float u[CPL];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        float x = 0.f;
-#pragma unroll
-        for (int w = 0; w < kXWarps; ++w) x += rd[w * DK + lane * CPL + c];
-        u[c] = x;
+      float skt = sk[0] + sk[1], sqt = sq[0] + sq[1];
+      if constexpr (SPLIT == 2) {
+        skt += __shfl_xor_sync(0xffffffffu, skt, 1);
+        sqt += __shfl_xor_sync(0xffffffffu, sqt, 1);
       }
-      float ku = 0.f;
+      const float a = st.f[t], gq = gqring[(cc & 1) * kTC + t];
+      const float vj = row < dv ? to_f32(st.v[t * X::DVP + row]) : 0.f;
+      const float e = vj - a * skt;
+      if (hf == 0) ob[t * X::DVP + row] = __fmaf_rn(e, gq, a * sqt);
+      const float4* g4 = reinterpret_cast<const float4*>(gin + t * DK + 32 * hf);
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) ku = __fmaf_rn(k[c], u[c], ku);
-      const float s = warp_sum(ku) + r;
-      const float inv_s = 1.f / s;
-      float g[CPL], gq = 0.f;
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        g[c] = u[c] * inv_s;
-        gq = __fmaf_rn(g[c], q[c], gq);
-      }
-      gq = warp_sum(gq);
-
-      // P = P- - u u^T / s; u_i of this warp's rows comes from the lane that owns column i
-#pragma unroll
-      for (int m = 0; m < PR; ++m) {
-        const int i = warp + kXWarps * m;
-        const float own = CPL == 1 ? u[0] : ((i & 1) ? u[CPL - 1] : u[0]);  // CPL <= 2
-        const float ui = __shfl_sync(0xffffffffu, own, i / CPL);
-#pragma unroll
-        for (int c = 0; c < CPL; ++c)
-          P[m][c] = __fmaf_rn(-__fmul_rn(ui, u[c]), inv_s, Pm[m][c]);
-      }
-
-      // e = v - a S k and o = a S q + e (g.q) for this warp's rows
-      float x[N];
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        float sk = 0.f, sq = 0.f;
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          sk = __fmaf_rn(S[i][c], k[c], sk);
-          sq = __fmaf_rn(S[i][c], q[c], sq);
-        }
-        x[i] = sk;
-        x[RPW + i] = sq;
-      }
-      const float tot = transpose_sum<N>(x, lane);
-      const int item = lane / G;
-      float e = 0.f;
-      if (item < RPW) {
-        const int j = warp + kXWarps * item;
-        e = (j < dv ? to_f32(sv[t * X::DVP + j]) : 0.f) - a * tot;
-      }
-      // lanes of item RPW + i take e_i from the first lane of item i
-      const float ei = __shfl_sync(0xffffffffu, e, (item - RPW) * G & 31);
-      if (item >= RPW && lane % G == 0) {
-        const int j = warp + kXWarps * (item - RPW);
-        obuf[t * X::DVP + j] = __fmaf_rn(ei, gq, a * tot);
-      }
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const float e_i = __shfl_sync(0xffffffffu, e, i * G);
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) S[i][c] = __fmaf_rn(e_i, g[c], a * S[i][c]);
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 gg = g4[c4];
+        X_[4 * c4] = __fmaf_rn(e, gg.x, a * X_[4 * c4]);
+        X_[4 * c4 + 1] = __fmaf_rn(e, gg.y, a * X_[4 * c4 + 1]);
+        X_[4 * c4 + 2] = __fmaf_rn(e, gg.z, a * X_[4 * c4 + 2]);
+        X_[4 * c4 + 3] = __fmaf_rn(e, gg.w, a * X_[4 * c4 + 3]);
       }
     }
-    __syncthreads();  // obuf complete; stage ch & 1 free for chunk ch + 2
-    for (int i = tid; i < nt * dv; i += kXThreads) {
+  };
+
+  // output rows of chunk cc, staged in obuf, go out coalesced
+  auto flush = [&](int cc) {
+    const int t0 = cc * kTC, nt = min(kTC, T - t0);
+    const float* ob = obuf + (cc & 1) * kTC * X::DVP;
+    for (int i = tid; i < nt * dv; i += NTH) {
       const int t = i / dv, j = i % dv;
-      O[(((size_t)b * T + t0 + t) * H + h) * dv + j] = obuf[t * X::DVP + j];
+      O[(((size_t)b * T + t0 + t) * H + h) * dv + j] = ob[t * X::DVP + j];
+    }
+  };
+
+  // Phase c: the covariance warps compute the gains of chunk c + 1 while the
+  // state warps run chunk c.  Inputs are three stages deep: chunk c + 2 is
+  // copied during phase c into the stage chunk c - 1 used.
+  const int nchunks = (T + kTC - 1) / kTC;
+  issue(0);
+  cp_async_commit();
+  if (nchunks > 1) issue(1);
+  cp_async_commit();
+  cp_async_wait_newest_pending();  // chunk 0 landed (this thread's copies)
+  __syncthreads();                 // ... and everyone's
+  if (pwarp) gains(0);
+  for (int c = 0; c < nchunks; ++c) {
+    __syncthreads();  // phase c - 1 done: gains of chunk c written, chunk c - 1 read
+    if (c > 0) flush(c - 1);
+    if (c + 2 < nchunks) issue(c + 2);
+    cp_async_commit();
+    cp_async_wait_newest_pending();  // chunk c + 1 landed (this thread's copies)
+    __syncthreads();                 // ... and everyone's
+    if (pwarp) {
+      if (c + 1 < nchunks) gains(c + 1);
+    } else {
+      states(c);
     }
   }
-  __syncthreads();  // every read of S0 / P0 is done before the stores
+  __syncthreads();  // the last chunk's outputs; every read of S0 / P0 is done
+  if (nchunks > 0) flush(nchunks - 1);
 
   // ---- state out
+  if (pwarp) {
 #pragma unroll
-  for (int i = 0; i < RPW; ++i) {
-    const int j = warp + kXWarps * i;
-    if (j < dv) {
+    for (int c = 0; c < 32; ++c)
+      P_out[p_base + (size_t)row * DK + ((row + SPLIT * c + hf) & M)] = X_[c];
+  } else if (row < dv) {
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) S_out[s_base + (size_t)j * DK + lane * CPL + c] = S[i][c];
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < PR; ++m) {
-    const int i = warp + kXWarps * m;
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) P_out[p_base + (size_t)i * DK + lane * CPL + c] = P[m][c];
+    for (int c = 0; c < 32; c += 4)
+      *reinterpret_cast<float4*>(S_out + s_base + (size_t)row * DK + 32 * hf + c) =
+          make_float4(X_[c], X_[c + 1], X_[c + 2], X_[c + 3]);
   }
 }
 
-template <int DK, int RPW, bool DIAG, typename InT>
+template <int DK, int SW, bool DIAG, typename InT>
 kdn_status launch_x(const void* q, const void* k, const void* v, const float* a, const float* w,
                     const float* r, const float* S0, const float* P0, float* o, float* S_out,
                     float* P_out, int B, int T, int H, int dv, cudaStream_t s) {
-  using X = XPlan<DK, RPW, DIAG, InT>;
-  auto kern = exact_kalman_kernel<DK, RPW, DIAG, InT>;
+  using X = XPlan<DK, SW, DIAG, InT>;
+  auto kern = exact_kalman_kernel<DK, SW, DIAG, InT>;
   if (X::TOTAL > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, X::TOTAL) !=
           cudaSuccess)
     return KDN_ERR_CUDA;
-  kern<<<(unsigned)(B * H), kXThreads, X::TOTAL, s>>>(
+  kern<<<(unsigned)(B * H), (X::PW + SW) * 32, X::TOTAL, s>>>(
       static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w, r,
       S0, P0, o, S_out, P_out, T, H, dv);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
@@ -328,11 +367,19 @@ template <int DK, bool DIAG, typename InT>
 kdn_status launch_dv(const void* q, const void* k, const void* v, const float* a, const float* w,
                      const float* r, const float* S0, const float* P0, float* o, float* S_out,
                      float* P_out, int B, int T, int H, int dv, cudaStream_t s) {
-  if (dv <= 32)
+  // state warps: d_v rows of DK / 32 lanes each, rounded up to 1, 2, 4 or 8 warps
+  const int need = (dv * (DK / 32) + 31) / 32;
+  if (need <= 1)
+    return launch_x<DK, 1, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
+  if (need <= 2)
+    return launch_x<DK, 2, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
+  if constexpr (DK == 32) {
     return launch_x<DK, 4, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
-  if (dv <= 64)
+  } else {
+    if (need <= 4)
+      return launch_x<DK, 4, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
     return launch_x<DK, 8, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
-  return launch_x<DK, 16, DIAG, InT>(q, k, v, a, w, r, S0, P0, o, S_out, P_out, B, T, H, dv, s);
+  }
 }
 
 template <bool DIAG, typename InT>

@@ -459,6 +459,18 @@ def exact_bytes(B, T, H, dk, dv, in_bytes=2):
             B * H * (dv * dk + dk * dk) * 4)
 
 
+def exact_flops(B, T, H, dk, dv):
+    """Algorithmic FLOPs of the dense filter (an FMA counts 2): per token and
+    head, P- = a^2 P + W (2 dk^2), u = P- k (2 dk^2), P = P- - u u^T / s
+    (3 dk^2); S k and S q (4 dv dk), S = a S + e g^T (3 dv dk)."""
+    return B * T * H * (7 * dk * dk + 7 * dv * dk)
+
+
+# FP32 peak of the CUDA cores (no tensor cores): 148 SMs x 128 FP32 lanes x
+# 2 FLOPs per FMA x 1.965 GHz (the B200's maximum SM clock)
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 def exact_case(kdn, synth, dev, B=None, T=None):
     """The dense filter: (launch fn, tokens, algorithmic bytes, description)."""
     import torch
@@ -551,9 +563,13 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     f, units, alg, desc = exact_case(kdn, synth, dev)
     n = 3
     ms = time_launches(f, n, 3, stream) / n
+    fl = exact_flops(desc['B'], desc['T'], desc['H'], desc['dk'], desc['dv'])
     out['exact_d64'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
                         'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
-                        'algorithmic_bytes': alg, **desc}
+                        'algorithmic_bytes': alg,
+                        'alu': {'achieved_tflops': fl / ms / 1e9, 'peak_tflops': FP32_PEAK_TFLOPS,
+                                'frac': fl / ms / 1e9 / FP32_PEAK_TFLOPS, 'flops': fl},
+                        **desc}
     return out
 
 

@@ -14,8 +14,9 @@ Also measured on the same run and reported under "secondary": the Diagonal
 KDN forward at the same shape, the standalone variance scan (4096 x 65536),
 the long-context diagonal forward (B1 T65536), the decode step (batch 256) and
 the isotropic forward over 32768 tokens packed from sequences of mixed length
-(kdn_forward_varlen), and the dense (full-covariance) filter at d_k = d_v = 64
-(kdn_exact_forward).
+(kdn_forward_varlen), the dense (full-covariance) filter at d_k = d_v = 64
+(kdn_exact_forward) and the information-form diagonal filter (kdn_kla_forward)
+on the Diagonal KDN's inputs.
 
 --impl reference times the fp64 CPU oracle (the correctness reference) on a
 bounded sample of the same workload on the host cores.
@@ -256,7 +257,7 @@ def main():
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
-    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact'],
+    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact', 'kla'],
                     help='run only this kernel (for profiler captures) and print its timing')
     ap.add_argument('--B', type=int, default=None, help='batch override for --only')
     ap.add_argument('--T', type=int, default=None, help='length override for --only')
@@ -411,6 +412,13 @@ def run_only(args):
         f, units, alg, _ = varlen_case(kdn, synth, dev)
     elif args.only == 'exact':
         f, units, alg, _ = exact_case(kdn, synth, dev, args.B, args.T)
+    elif args.only == 'kla':
+        c = synth.WORKLOADS['diag_1p3b']
+        B, T, H, d = args.B or c['B'], args.T or c['T'], c['H'], c['dk']
+        x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'diag', c['seed'],
+                                                         c['dtype']).items()}
+        f = lambda: kdn.kdn_kla_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'])
+        units, alg = B * T, layer_bytes('diag', B, T, H, d, d)
     else:
         c = synth.WORKLOADS['diag_long']
         B = args.B or c['decode_batch']
@@ -559,6 +567,25 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     out['iso_varlen'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
                          'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                          'algorithmic_bytes': alg, **desc}
+    # information-form diagonal filter (KLA) on the Diagonal KDN's inputs
+    c = synth.WORKLOADS['diag_1p3b']
+    B, T, H, d = c['B'], c['T'], c['H'], c['dk']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'diag', c['seed'],
+                                                     c['dtype']).items()}
+    o = torch.empty((B, T, H, d), dtype=torch.float32, device=dev)
+    S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    lam = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    f = lambda: kdn.kdn_kla_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], o=o,
+                                    S_out=S, lam_out=lam)
+    n = 5
+    ms = time_launches(f, n, 3, stream) / n
+    alg = layer_bytes('diag', B, T, H, d, d)
+    fl = B * T * H * 5 * d * d  # S f + v u^T (3 per element), S q (2)
+    out['kla_1p3b'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
+                       'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg,
+                       'alu': {'achieved_tflops': fl / ms / 1e9, 'peak_tflops': FP32_PEAK_TFLOPS,
+                               'frac': fl / ms / 1e9 / FP32_PEAK_TFLOPS, 'flops': fl}}
+    del x, o, S, lam
     # dense (full-covariance) filter, B8 T4096 H16 d64
     f, units, alg, desc = exact_case(kdn, synth, dev)
     n = 3

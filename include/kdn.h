@@ -330,6 +330,37 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k,
                              void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_kla_forward -- the diagonal Kalman filter in information form ("Kalman
+ * Linear Attention: Parallel Bayesian Filtering ...", 方法论 §1-§3): a
+ * precision per key dimension, updated by a Mobius map of the previous one,
+ * and an information mean that is an affine recursion given the precisions,
+ * read out with the query.  It runs on the Diagonal KDN's inputs (decay a,
+ * process noise w per key dimension, value precision 1 / r) with every
+ * element of the memory filtered on its own, so per token and dimension i:
+ *   lambda-_i = 1 / (a^2 / lambda_i + w_i),  lambda_i = lambda-_i + k_i^2 / r
+ *   S <- S diag(f) + v u^T,  f = a lambda- / lambda,  u = (k / r) / lambda
+ *   o = S q
+ * (forget gate f and write gate u: ratios of precisions).
+ *
+ * q, k     [B, T, H, dk] in_dtype device;  v [B, T, H, dv] in_dtype device
+ * a, r     [B, T, H] fp32 device;  w [B, T, H, dk] fp32 device
+ * S0       [B, H, dv, dk] fp32 device posterior mean, or NULL for zeros
+ * lam0     [B, H, dk] fp32 device precision, or NULL for ones
+ * o        [B, T, H, dv] fp32 device output
+ * S_out    [B, H, dv, dk];  lam_out [B, H, dk] fp32 device outputs; they may
+ *          alias S0 and lam0
+ * Supported: dk in {32, 64, 128}; 8 <= dv <= 128 with dv a multiple of 8;
+ * every pointer 16-byte aligned.  One CTA per (b, h); no workspace and no
+ * on-device waits.  Errors: KDN_ERR_INVALID_ARG (NULL, shape, alignment,
+ * dtype), KDN_ERR_UNSUPPORTED (sizes), KDN_ERR_CUDA (launch).
+ * ---------------------------------------------------------------------- */
+kdn_status kdn_kla_forward(const void* q, const void* k, const void* v,
+                           kdn_dtype in_dtype, const float* a, const float* w,
+                           const float* r, const float* S0, const float* lam0,
+                           float* o, float* S_out, float* lam_out, int B, int T,
+                           int H, int dk, int dv, void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_read_workspace_status -- synchronise `stream`, then report the device
  * error word a previous call left in `workspace`: KDN_OK, KDN_ERR_TIMEOUT
  * if a bounded on-device wait gave up, or KDN_ERR_INVALID_ARG if packed-

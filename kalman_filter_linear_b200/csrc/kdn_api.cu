@@ -36,6 +36,11 @@ kdn_status exact_kalman_launch(bool diag, kdn_dtype dt, const void* q, const voi
                                const void* v, const float* a, const float* w, const float* r,
                                const float* S0, const float* P0, float* o, float* S_out,
                                float* P_out, int B, int T, int H, int dk, int dv, cudaStream_t s);
+bool kla_supported(int dk, int dv);
+kdn_status kla_launch(kdn_dtype dt, const void* q, const void* k, const void* v, const float* a,
+                      const float* w, const float* r, const float* S0, const float* L0, float* o,
+                      float* S_out, float* L_out, int B, int T, int H, int dk, int dv,
+                      cudaStream_t s);
 }  // namespace kdn
 
 namespace {
@@ -275,6 +280,21 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k, 
   if (!kdn::exact_kalman_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
   return kdn::exact_kalman_launch(variant == KDN_DIAG, in_dtype, q, k, v, a, w, r, S0, P0, o,
                                   S_out, P_out, B, T, H, dk, dv, as_stream(stream));
+}
+
+kdn_status kdn_kla_forward(const void* q, const void* k, const void* v, kdn_dtype in_dtype,
+                           const float* a, const float* w, const float* r, const float* S0,
+                           const float* lam0, float* o, float* S_out, float* lam_out, int B,
+                           int T, int H, int dk, int dv, void* stream) {
+  if (!q || !k || !v || !a || !w || !r || !o || !S_out || !lam_out) return KDN_ERR_INVALID_ARG;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(a) || !al16(w) || !al16(r) || !al16(o) ||
+      !al16(S_out) || !al16(lam_out) || !al16_or_null(S0) || !al16_or_null(lam0))
+    return KDN_ERR_INVALID_ARG;
+  if (!kdn::kla_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
+  return kdn::kla_launch(in_dtype, q, k, v, a, w, r, S0, lam0, o, S_out, lam_out, B, T, H, dk,
+                         dv, as_stream(stream));
 }
 
 size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,

@@ -75,6 +75,8 @@ def lib():
         [_f32, _vp]
     L.kdn_exact_forward.restype = _i32
     L.kdn_exact_forward.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
+    L.kdn_kla_forward.restype = _i32
+    L.kdn_kla_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
     L.kdn_read_workspace_status.restype = _i32
     L.kdn_read_workspace_status.argtypes = [_vp, _sz, _vp]
     L.kdn_testing_mobius_scan_unpublished_tile.restype = _i32
@@ -403,6 +405,37 @@ def kdn_exact_forward(variant, q, k, v, a, w, r, S0=None, P0=None, o=None, S_out
                                  B, T, H, dk, dv, _stream())
     _check(st, 'kdn_exact_forward')
     return o, S_out, P_out
+
+
+def kdn_kla_forward(q, k, v, a, w, r, S0=None, lam0=None, o=None, S_out=None, lam_out=None):
+    """The information-form diagonal filter (KLA): q, k [B,T,H,dk], v [B,T,H,dv],
+    a, r [B,T,H], w [B,T,H,dk].  Returns (o [B,T,H,dv], S_T [B,H,dv,dk],
+    lam_T [B,H,dk]) -- lam is the precision."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _in_dtype(q)
+    _req(q, 'q', dt)
+    _req(k, 'k', dt, (B, T, H, dk))
+    _req(v, 'v', dt, (B, T, H, dv))
+    f = torch.float32
+    _req(a, 'a', f, (B, T, H))
+    _req(r, 'r', f, (B, T, H))
+    _req(w, 'w', f, (B, T, H, dk))
+    _opt(S0, 'S0', f, (B, H, dv, dk))
+    _opt(lam0, 'lam0', f, (B, H, dk))
+    dev = q.device
+    o = _req(o, 'o', f, (B, T, H, dv)) if o is not None else \
+        torch.empty((B, T, H, dv), dtype=f, device=dev)
+    S_out = _req(S_out, 'S_out', f, (B, H, dv, dk)) if S_out is not None else \
+        torch.empty((B, H, dv, dk), dtype=f, device=dev)
+    lam_out = _req(lam_out, 'lam_out', f, (B, H, dk)) if lam_out is not None else \
+        torch.empty((B, H, dk), dtype=f, device=dev)
+    st = lib().kdn_kla_forward(_ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w), _ptr(r),
+                               _ptr(S0), _ptr(lam0), _ptr(o), _ptr(S_out), _ptr(lam_out), B, T, H,
+                               dk, dv, _stream())
+    _check(st, 'kdn_kla_forward')
+    return o, S_out, lam_out
 
 
 def kdn_read_workspace_status(workspace):

@@ -134,3 +134,17 @@ def test_exact_forward_rejects_bad_arguments(L):
     assert x(dk=16) == kdn.KDN_ERR_UNSUPPORTED
     assert x(dv=12) == kdn.KDN_ERR_UNSUPPORTED    # d_v a multiple of 8
     assert x(dv=136) == kdn.KDN_ERR_UNSUPPORTED
+
+
+def test_kla_forward_rejects_bad_arguments(L):
+    base = dict(q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_BF16, a=FAKE, w=FAKE, r=FAKE, S0=None,
+                lam0=None, o=FAKE, S=FAKE, lam=FAKE, B=1, T=8, H=1, dk=128, dv=128, stream=None)
+    x = lambda **kw: L.kdn_kla_forward(*dict(base, **kw).values())
+    assert x(v=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(lam=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dt=9) == kdn.KDN_ERR_INVALID_ARG
+    assert x(T=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(lam0=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dk=96) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(dv=4) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(dv=130) == kdn.KDN_ERR_UNSUPPORTED

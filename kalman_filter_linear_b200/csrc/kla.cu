@@ -19,11 +19,13 @@
 //  - Precision warps (d_k / 32 of them): thread i runs dimension i's
 //    recursion over the chunk, with no barrier, and leaves f, u and q (fp32)
 //    in shared memory.
-//  - State warps: each row j of S is held by d_k / 32 lanes, 32 columns each,
-//    as 8 groups of 4 columns interleaved across the row's lanes (group
-//    LPR c + h on lane h), so that the lanes of a row read consecutive 16-byte
-//    words of f, u and q.  Per token: S <- S f + v u, then o_j = S_j . q,
-//    joined across the row's lanes by xor shuffles.
+//  - State warps: warp w holds rows [8 w, 8 w + 8) of S; lane l holds
+//    columns [l CPL, (l + 1) CPL), CPL = d_k / 32.  A lane therefore reads
+//    only its own columns' f, u and q per token (one load each, consecutive
+//    across the warp) and its rows' v in one 16-byte word (bf16), and
+//    o_j = S_j . q, 8 row sums per warp, is joined
+//    across the lanes by recursive halving (each exchange step halves the
+//    values a lane keeps).
 //  - Inputs come in by cp.async in 16-token chunks, three stages deep;
 //    outputs leave per chunk in coalesced rows.
 #include "kdn_common.cuh"
@@ -44,11 +46,34 @@ __device__ __forceinline__ void la_cp4(void* dst, const void* src) {
 __device__ __forceinline__ void la_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void la_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
+// Sums item i of x[8] over the 32 lanes by recursive halving: at lane offsets
+// 16, 8 and 4 a lane keeps half of its values and adds its partner's copy of
+// that half; two xor steps then finish.  Lane l ends with the total of item
+// l / 4.
+template <int N, int O>
+__device__ __forceinline__ void la_halve(float* x, int lane) {
+  const bool up = (lane & O) != 0;
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float send = up ? x[i] : x[i + N / 2];
+    const float keep = up ? x[i + N / 2] : x[i];
+    x[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+  }
+}
+__device__ __forceinline__ float la_transpose_sum8(float (&x)[8], int lane) {
+  la_halve<8, 16>(x, lane);
+  la_halve<4, 8>(x, lane);
+  la_halve<2, 4>(x, lane);
+  float y = x[0];
+  y += __shfl_xor_sync(0xffffffffu, y, 2);
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  return y;
+}
+
 template <int DK, int SW, typename InT>
 struct LPlan {
-  static constexpr int LPR = DK / 32;                         // lanes per row of S
   static constexpr int PW = DK / 32;                          // precision warps
-  static constexpr int DVP = SW * 32 / LPR;                   // d_v rounded up
+  static constexpr int DVP = SW * 8;                          // d_v rounded up: 8 rows a warp
   static constexpr int KQ = kLC * 2 * DK * (int)sizeof(InT);  // [t][k | q]
   static constexpr int VB = kLC * DVP * (int)sizeof(InT);     // [t][v]
   static constexpr int F32 = kLC * (2 + DK) * 4;              // a[t], r[t], w[t][DK]
@@ -65,12 +90,11 @@ kla_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __re
            const float* __restrict__ R, const float* S0, const float* L0,
            float* __restrict__ O, float* S_out, float* L_out, int T, int H, int dv) {
   using X = LPlan<DK, SW, InT>;
-  constexpr int PW = X::PW, LPR = X::LPR, NTH = (PW + SW) * 32;
+  constexpr int PW = X::PW, CPL = DK / 32, NTH = (PW + SW) * 32;
   extern __shared__ __align__(16) uint8_t lsm[];
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool pwarp = warp < PW;
-  const int st_t = tid - PW * 32;
-  const int row = st_t / LPR, hl = st_t % LPR;  // state lanes: row of S and its lane
+  const int sw = warp - PW;  // state warp: rows 8 sw + i
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
   float* gates = reinterpret_cast<float*>(lsm + X::OFF_G);
   float* obuf = reinterpret_cast<float*>(lsm + X::OFF_OUT);
@@ -119,23 +143,20 @@ kla_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __re
   };
 
   // ---- state: the precision lanes carry the variance p_i = 1 / lambda_i;
-  // the state lanes hold their 32 columns of row j.  S_out / L_out may alias
+  // the state lanes hold their CPL columns of 8 rows.  S_out / L_out may alias
   // S0 / L0: every read comes before the barrier that precedes the stores.
   float p = 1.f;
-  float Sr[32];
+  float Sr[8][CPL];
   const size_t s_base = (size_t)bh * dv * DK;
   if (pwarp) {
     p = L0 ? 1.f / L0[(size_t)bh * DK + tid] : 1.f;
   } else {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (S0 && row < dv)
-        x = *reinterpret_cast<const float4*>(S0 + s_base + (size_t)row * DK + 4 * (LPR * c + hl));
-      Sr[4 * c] = x.x;
-      Sr[4 * c + 1] = x.y;
-      Sr[4 * c + 2] = x.z;
-      Sr[4 * c + 3] = x.w;
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * sw + i;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c)
+        Sr[i][c] = (S0 && j < dv) ? S0[s_base + (size_t)j * DK + lane * CPL + c] : 0.f;
     }
   }
 
@@ -163,28 +184,45 @@ kla_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __re
     const float* g = gates + (cc & 1) * kLC * 3 * DK;
     float* ob = obuf + (cc & 1) * kLC * X::DVP;
     for (int t = 0; t < nt; ++t) {
-      const float4* f4 = reinterpret_cast<const float4*>(g + (t * 3 + 0) * DK);
-      const float4* u4 = reinterpret_cast<const float4*>(g + (t * 3 + 1) * DK);
-      const float4* q4 = reinterpret_cast<const float4*>(g + (t * 3 + 2) * DK);
-      const float vj = row < dv ? to_f32(st.v[t * X::DVP + row]) : 0.f;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float f[CPL], u[CPL], q[CPL];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const int gi = LPR * c + hl;
-        const float4 ff = f4[gi], uu = u4[gi], qq = q4[gi];
-        Sr[4 * c] = __fmaf_rn(vj, uu.x, Sr[4 * c] * ff.x);
-        Sr[4 * c + 1] = __fmaf_rn(vj, uu.y, Sr[4 * c + 1] * ff.y);
-        Sr[4 * c + 2] = __fmaf_rn(vj, uu.z, Sr[4 * c + 2] * ff.z);
-        Sr[4 * c + 3] = __fmaf_rn(vj, uu.w, Sr[4 * c + 3] * ff.w);
-        acc[0] = __fmaf_rn(Sr[4 * c], qq.x, acc[0]);
-        acc[1] = __fmaf_rn(Sr[4 * c + 1], qq.y, acc[1]);
-        acc[2] = __fmaf_rn(Sr[4 * c + 2], qq.z, acc[2]);
-        acc[3] = __fmaf_rn(Sr[4 * c + 3], qq.w, acc[3]);
+      for (int c = 0; c < CPL; ++c) {
+        f[c] = g[(t * 3 + 0) * DK + lane * CPL + c];
+        u[c] = g[(t * 3 + 1) * DK + lane * CPL + c];
+        q[c] = g[(t * 3 + 2) * DK + lane * CPL + c];
       }
-      float o = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      // v of this warp's 8 rows (rows at or past d_v were never staged: zero)
+      float vr[8];
+      const InT* vp = st.v + t * X::DVP + 8 * sw;
+      if constexpr (sizeof(InT) == 2) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(vp);
+        const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int m = 1; m < LPR; m <<= 1) o += __shfl_xor_sync(0xffffffffu, o, m);
-      if (hl == 0) ob[t * X::DVP + row] = o;
+        for (int e = 0; e < 4; ++e) {
+          vr[2 * e] = __uint_as_float(wd[e] << 16);
+          vr[2 * e + 1] = __uint_as_float(wd[e] & 0xffff0000u);
+        }
+      } else {
+        const float4 v0 = *reinterpret_cast<const float4*>(vp);
+        const float4 v1 = *reinterpret_cast<const float4*>(vp + 4);
+        vr[0] = v0.x; vr[1] = v0.y; vr[2] = v0.z; vr[3] = v0.w;
+        vr[4] = v1.x; vr[5] = v1.y; vr[6] = v1.z; vr[7] = v1.w;
+      }
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float vj = 8 * sw + i < dv ? vr[i] : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          Sr[i][c] = __fmaf_rn(vj, u[c], Sr[i][c] * f[c]);
+          acc = __fmaf_rn(Sr[i][c], q[c], acc);
+        }
+        x[i] = acc;
+      }
+      // lane l ends with the row sum of row 8 sw + l / 4
+      const float o = la_transpose_sum8(x, lane);
+      if ((lane & 3) == 0) ob[t * X::DVP + 8 * sw + (lane >> 2)] = o;
     }
   };
 
@@ -225,11 +263,15 @@ kla_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __re
 
   if (pwarp) {
     L_out[(size_t)bh * DK + tid] = 1.f / p;
-  } else if (row < dv) {
+  } else {
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<float4*>(S_out + s_base + (size_t)row * DK + 4 * (LPR * c + hl)) =
-          make_float4(Sr[4 * c], Sr[4 * c + 1], Sr[4 * c + 2], Sr[4 * c + 3]);
+    for (int i = 0; i < 8; ++i) {
+      const int j = 8 * sw + i;
+      if (j < dv) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) S_out[s_base + (size_t)j * DK + lane * CPL + c] = Sr[i][c];
+      }
+    }
   }
 }
 
@@ -249,22 +291,17 @@ kdn_status launch_l(const void* q, const void* k, const void* v, const float* a,
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
-// state warps: d_v rows of DK / 32 lanes each, rounded up to 1, 2, 4, 8 or 16 warps
+// state warps: 8 rows of S each, d_v / 8 rounded up to 1, 2, 4, 8 or 16 warps
 template <int DK, typename InT>
 kdn_status launch_ldv(const void* q, const void* k, const void* v, const float* a, const float* w,
                       const float* r, const float* S0, const float* L0, float* o, float* S_out,
                       float* L_out, int B, int T, int H, int dv, cudaStream_t s) {
-  const int need = (dv * (DK / 32) + 31) / 32;
+  const int need = (dv + 7) / 8;
   if (need <= 1) return launch_l<DK, 1, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
   if (need <= 2) return launch_l<DK, 2, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
   if (need <= 4) return launch_l<DK, 4, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
-  if constexpr (DK >= 64) {
-    if (need <= 8) return launch_l<DK, 8, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
-  }
-  if constexpr (DK == 128) {
-    return launch_l<DK, 16, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
-  }
-  return KDN_ERR_UNSUPPORTED;
+  if (need <= 8) return launch_l<DK, 8, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
+  return launch_l<DK, 16, InT>(q, k, v, a, w, r, S0, L0, o, S_out, L_out, B, T, H, dv, s);
 }
 
 template <typename InT>

@@ -26,6 +26,8 @@
 //    o_j = S_j . q, 8 row sums per warp, is joined
 //    across the lanes by recursive halving (each exchange step halves the
 //    values a lane keeps).
+//    The update and the row sums run on column pairs with the packed FP32
+//    instructions (two FMAs per instruction).
 //  - Inputs come in by cp.async in 16-token chunks, three stages deep;
 //    outputs leave per chunk in coalesced rows.
 #include "kdn_common.cuh"
@@ -212,13 +214,24 @@ kla_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __re
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float vj = 8 * sw + i < dv ? vr[i] : 0.f;
-        float acc = 0.f;
+        if constexpr (CPL == 1) {
+          Sr[i][0] = __fmaf_rn(vj, u[0], Sr[i][0] * f[0]);
+          x[i] = Sr[i][0] * q[0];
+        } else {
+          // column pairs on the packed FP32 pipe: S <- (S f) + v u, acc += S q
+          float2 acc = make_float2(0.f, 0.f);
+          const float2 v2 = make_float2(vj, vj);
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-          Sr[i][c] = __fmaf_rn(vj, u[c], Sr[i][c] * f[c]);
-          acc = __fmaf_rn(Sr[i][c], q[c], acc);
+          for (int c = 0; c < CPL; c += 2) {
+            float2 sp = make_float2(Sr[i][c], Sr[i][c + 1]);
+            sp = __ffma2_rn(v2, make_float2(u[c], u[c + 1]),
+                            __fmul2_rn(sp, make_float2(f[c], f[c + 1])));
+            acc = __ffma2_rn(sp, make_float2(q[c], q[c + 1]), acc);
+            Sr[i][c] = sp.x;
+            Sr[i][c + 1] = sp.y;
+          }
+          x[i] = acc.x + acc.y;
         }
-        x[i] = acc;
       }
       // lane l ends with the row sum of row 8 sw + l / 4
       const float o = la_transpose_sum8(x, lane);

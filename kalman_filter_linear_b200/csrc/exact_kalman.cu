@@ -31,6 +31,8 @@
 //  - State warps: half h of row j holds S[j][32 h + c'].  S k and S q are
 //    in-lane dot products with k and q read as broadcasts; the update
 //    S_j <- a S_j + e_j g likewise.
+//  - Both roles run their per-element arithmetic on column pairs with the
+//    packed FP32 instructions (two FMAs per instruction).
 //  - Inputs come into shared memory by cp.async in chunks of 16 tokens, three
 //    stages deep; outputs leave per chunk in coalesced rows.
 #include "kdn_common.cuh"
@@ -214,12 +216,18 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       const float* urot = ub + row + hf;  // urot[SPLIT c] = u[(row + SPLIT c + hf) mod DK]
       // P- = a^2 P + W (W on the diagonal: register 0 of half 0) and
       // u_i = (P- k)_i; P- is formed again, identically, in the update
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      // (column pairs on the packed FP32 pipe; each element rounds as a scalar
+      // operation would, so (i, j) and (j, i) still agree bit for bit)
+      const float2 aa2 = make_float2(aa, aa);
+      float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        acc[c & 3] = __fmaf_rn(__fmaf_rn(aa, X_[c], c == 0 ? wd : 0.f), krot[SPLIT * c],
-                               acc[c & 3]);
-      float u = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      for (int c = 0; c < 32; c += 2) {
+        const float2 pm = __ffma2_rn(aa2, make_float2(X_[c], X_[c + 1]),
+                                     make_float2(c == 0 ? wd : 0.f, 0.f));
+        acc[(c >> 1) & 1] = __ffma2_rn(pm, make_float2(krot[SPLIT * c], krot[SPLIT * (c + 1)]),
+                                       acc[(c >> 1) & 1]);
+      }
+      float u = (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);
       if constexpr (SPLIT == 2) u += __shfl_xor_sync(0xffffffffu, u, 1);
       if (hf == 0) {
         ub[row] = u;
@@ -243,10 +251,16 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       if (hf == 0) gout[t * DK + row] = u * inv_s;
       if (tid == 0) gqring[(cc & 1) * kTC + t] = qus * inv_s;
       // P = P- - u u^T / s
+      const float2 nu = make_float2(-u, -u), is2 = make_float2(inv_s, inv_s);
 #pragma unroll
-      for (int c = 0; c < 32; ++c)
-        X_[c] = __fmaf_rn(-__fmul_rn(u, urot[SPLIT * c]), inv_s,
-                          __fmaf_rn(aa, X_[c], c == 0 ? wd : 0.f));
+      for (int c = 0; c < 32; c += 2) {
+        const float2 pm = __ffma2_rn(aa2, make_float2(X_[c], X_[c + 1]),
+                                     make_float2(c == 0 ? wd : 0.f, 0.f));
+        const float2 uu = __fmul2_rn(nu, make_float2(urot[SPLIT * c], urot[SPLIT * (c + 1)]));
+        const float2 x = __ffma2_rn(uu, is2, pm);
+        X_[c] = x.x;
+        X_[c + 1] = x.y;
+      }
       // (u and the partial sums are double-buffered by token parity: the
       // barrier of the next token orders this token's reads before their reuse)
     }
@@ -262,21 +276,20 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
     for (int t = 0; t < nt; ++t) {
       const float4* k4 = reinterpret_cast<const float4*>(kf + t * 2 * DK + 32 * hf);
       const float4* q4 = reinterpret_cast<const float4*>(kf + t * 2 * DK + DK + 32 * hf);
-      float sk[2] = {0.f, 0.f}, sq[2] = {0.f, 0.f};
+      float2 sk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float2 sq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
         const float4 kk = k4[c4], qq = q4[c4];
-        const int p = c4 & 1;
-        sk[p] = __fmaf_rn(X_[4 * c4], kk.x, sk[p]);
-        sk[p] = __fmaf_rn(X_[4 * c4 + 1], kk.y, sk[p]);
-        sk[p] = __fmaf_rn(X_[4 * c4 + 2], kk.z, sk[p]);
-        sk[p] = __fmaf_rn(X_[4 * c4 + 3], kk.w, sk[p]);
-        sq[p] = __fmaf_rn(X_[4 * c4], qq.x, sq[p]);
-        sq[p] = __fmaf_rn(X_[4 * c4 + 1], qq.y, sq[p]);
-        sq[p] = __fmaf_rn(X_[4 * c4 + 2], qq.z, sq[p]);
-        sq[p] = __fmaf_rn(X_[4 * c4 + 3], qq.w, sq[p]);
+        const float2 x0 = make_float2(X_[4 * c4], X_[4 * c4 + 1]);
+        const float2 x1 = make_float2(X_[4 * c4 + 2], X_[4 * c4 + 3]);
+        sk[0] = __ffma2_rn(x0, make_float2(kk.x, kk.y), sk[0]);
+        sk[1] = __ffma2_rn(x1, make_float2(kk.z, kk.w), sk[1]);
+        sq[0] = __ffma2_rn(x0, make_float2(qq.x, qq.y), sq[0]);
+        sq[1] = __ffma2_rn(x1, make_float2(qq.z, qq.w), sq[1]);
       }
-      float skt = sk[0] + sk[1], sqt = sq[0] + sq[1];
+      float skt = (sk[0].x + sk[1].x) + (sk[0].y + sk[1].y);
+      float sqt = (sq[0].x + sq[1].x) + (sq[0].y + sq[1].y);
       if constexpr (SPLIT == 2) {
         skt += __shfl_xor_sync(0xffffffffu, skt, 1);
         sqt += __shfl_xor_sync(0xffffffffu, sqt, 1);
@@ -286,13 +299,18 @@ exact_kalman_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       const float e = vj - a * skt;
       if (hf == 0) ob[t * X::DVP + row] = __fmaf_rn(e, gq, a * sqt);
       const float4* g4 = reinterpret_cast<const float4*>(gin + t * DK + 32 * hf);
+      const float2 e2 = make_float2(e, e), a2 = make_float2(a, a);
 #pragma unroll
       for (int c4 = 0; c4 < 8; ++c4) {
         const float4 gg = g4[c4];
-        X_[4 * c4] = __fmaf_rn(e, gg.x, a * X_[4 * c4]);
-        X_[4 * c4 + 1] = __fmaf_rn(e, gg.y, a * X_[4 * c4 + 1]);
-        X_[4 * c4 + 2] = __fmaf_rn(e, gg.z, a * X_[4 * c4 + 2]);
-        X_[4 * c4 + 3] = __fmaf_rn(e, gg.w, a * X_[4 * c4 + 3]);
+        const float2 x0 = __ffma2_rn(e2, make_float2(gg.x, gg.y),
+                                     __fmul2_rn(a2, make_float2(X_[4 * c4], X_[4 * c4 + 1])));
+        const float2 x1 = __ffma2_rn(e2, make_float2(gg.z, gg.w),
+                                     __fmul2_rn(a2, make_float2(X_[4 * c4 + 2], X_[4 * c4 + 3])));
+        X_[4 * c4] = x0.x;
+        X_[4 * c4 + 1] = x0.y;
+        X_[4 * c4 + 2] = x1.x;
+        X_[4 * c4 + 3] = x1.y;
       }
     }
   };

@@ -1020,8 +1020,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __device__ __forceinline__ void split_pack2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
   hi = *reinterpret_cast<const uint32_t*>(&hb);
-  const __nv_bfloat162 lb = __floats2bfloat162_rn(x0 - __uint_as_float(hi << 16),
-                                                  x1 - __uint_as_float(hi & 0xffff0000u));
+  // x - hi for both halves in one packed FP32 add (rounds as two scalar ones)
+  const float2 d = __fadd2_rn(make_float2(x0, x1), make_float2(-__uint_as_float(hi << 16),
+                                                               -__uint_as_float(hi & 0xffff0000u)));
+  const __nv_bfloat162 lb = __floats2bfloat162_rn(d.x, d.y);
   lo = *reinterpret_cast<const uint32_t*>(&lb);
 }
 
@@ -1690,10 +1692,16 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float4 g4 = gm4[i4];
           const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < 4; e += 2) {
             const int i = 4 * i4 + e;
-            const uint16_t vb = *reinterpret_cast<const uint16_t*>(vrow + i * 128 + voff[i & 7]);
-            z[i] = fmaf(-gv[e], z[i], __uint_as_float((uint32_t)vb << 16));
+            const uint16_t vb0 = *reinterpret_cast<const uint16_t*>(vrow + i * 128 + voff[i & 7]);
+            const uint16_t vb1 =
+                *reinterpret_cast<const uint16_t*>(vrow + (i + 1) * 128 + voff[(i + 1) & 7]);
+            const float2 zz = __ffma2_rn(make_float2(-gv[e], -gv[e + 1]), make_float2(z[i], z[i + 1]),
+                                         make_float2(__uint_as_float((uint32_t)vb0 << 16),
+                                                     __uint_as_float((uint32_t)vb1 << 16)));
+            z[i] = zz.x;
+            z[i + 1] = zz.y;
           }
         }
 #pragma unroll
@@ -1738,10 +1746,14 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 g4 = gm4[i4];
-          qr[4 * i4] = __float_as_uint(g4.x * qs[4 * i4]);
-          qr[4 * i4 + 1] = __float_as_uint(g4.y * qs[4 * i4 + 1]);
-          qr[4 * i4 + 2] = __float_as_uint(g4.z * qs[4 * i4 + 2]);
-          qr[4 * i4 + 3] = __float_as_uint(g4.w * qs[4 * i4 + 3]);
+          const float2 p0 = __fmul2_rn(make_float2(g4.x, g4.y),
+                                       make_float2(qs[4 * i4], qs[4 * i4 + 1]));
+          const float2 p1 = __fmul2_rn(make_float2(g4.z, g4.w),
+                                       make_float2(qs[4 * i4 + 2], qs[4 * i4 + 3]));
+          qr[4 * i4] = __float_as_uint(p0.x);
+          qr[4 * i4 + 1] = __float_as_uint(p0.y);
+          qr[4 * i4 + 2] = __float_as_uint(p1.x);
+          qr[4 * i4 + 3] = __float_as_uint(p1.y);
         }
         tmem_st32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qr);
         const float gC = sc_gC[sl];
@@ -1752,7 +1764,11 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           tmem_ld32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, x);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(gC * x[i]);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 d = __fmul2_rn(make_float2(gC, gC), make_float2(x[i], x[i + 1]));
+            r[i] = __float_as_uint(d.x);
+            r[i + 1] = __float_as_uint(d.y);
+          }
           tmem_st32(tmem + tm_lane + P::COL_ST + 64 * ch + 32 * h32, r);
         }
       }
@@ -1770,8 +1786,11 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 c4 = cf4[i4];
-          split_pack2(c4.x * u[4 * i4], c4.y * u[4 * i4 + 1], hi[2 * i4], lo[2 * i4]);
-          split_pack2(c4.z * u[4 * i4 + 2], c4.w * u[4 * i4 + 3], hi[2 * i4 + 1], lo[2 * i4 + 1]);
+          const float2 b0 = __fmul2_rn(make_float2(c4.x, c4.y), make_float2(u[4 * i4], u[4 * i4 + 1]));
+          const float2 b1 =
+              __fmul2_rn(make_float2(c4.z, c4.w), make_float2(u[4 * i4 + 2], u[4 * i4 + 3]));
+          split_pack2(b0.x, b0.y, hi[2 * i4], lo[2 * i4]);
+          split_pack2(b1.x, b1.y, hi[2 * i4 + 1], lo[2 * i4 + 1]);
         }
         tmem_st16u(tmem + tm_lane + P::COL_W + 16 * ch, hi);  // Z has been read
         tmem_st16u(tmem + tm_lane + P::COL_W + 32 + 16 * ch, lo);

@@ -1948,9 +1948,15 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           const float lj[4] = {lgj.x, lgj.y, lgj.z, lgj.w};
           const float bv[4] = {bj.x, bj.y, bj.z, bj.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float val = ex2_approx(lg_t - lj[e]) * bv[e] * d1[4 * i4 + e];
-            preg[4 * i4 + e] = (j0 + e < lim) ? val : 0.f;
+          for (int e = 0; e < 4; e += 2) {
+            // (gamma_t / gamma_j) beta_j D1, a pair per packed FP32 operation
+            const float2 dl = __fadd2_rn(make_float2(lg_t, lg_t), make_float2(-lj[e], -lj[e + 1]));
+            const float2 val = __fmul2_rn(
+                __fmul2_rn(make_float2(ex2_approx(dl.x), ex2_approx(dl.y)),
+                           make_float2(bv[e], bv[e + 1])),
+                make_float2(d1[4 * i4 + e], d1[4 * i4 + e + 1]));
+            preg[4 * i4 + e] = (j0 + e < lim) ? val.x : 0.f;
+            preg[4 * i4 + e + 1] = (j0 + e + 1 < lim) ? val.y : 0.f;
           }
         }
       }

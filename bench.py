@@ -586,6 +586,26 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
                        'alu': {'achieved_tflops': fl / ms / 1e9, 'peak_tflops': FP32_PEAK_TFLOPS,
                                'frac': fl / ms / 1e9 / FP32_PEAK_TFLOPS, 'flops': fl}}
     del x, o, S, lam
+    # backward pass (token-recurrent), B8 T4096 H16 d64, isotropic
+    c = synth.WORKLOADS['exact_d64']
+    B, T, H, d = c['B'], c['T'], c['H'], c['dk']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'iso', c['seed'],
+                                                     c['dtype']).items()}
+    dO = torch.randn((B, T, H, d), device=dev)
+    wsb = torch.empty(kdn.kdn_backward_workspace_size(kdn.KDN_ISO, B, T, H, d, d),
+                      dtype=torch.uint8, device=dev)
+    f = lambda: kdn.kdn_backward('iso', x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,
+                                 workspace=wsb)
+    n = 2
+    ms = time_launches(f, n, 2, stream) / n
+    # inputs read twice (the forward again, then the backward), the saved
+    # states written and read once, gradients written
+    alg = (2 * B * T * H * (3 * d * 2 + 12) + B * T * H * d * 4 +
+           2 * B * H * T * (d * d + 1) * 4 + B * T * H * (3 * d + 3) * 4)
+    out['backward_d64'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms,
+                           'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                           'algorithmic_bytes': alg, 'B': B, 'T': T, 'H': H, 'd': d}
+    del x, dO, wsb
     # dense (full-covariance) filter, B8 T4096 H16 d64
     f, units, alg, desc = exact_case(kdn, synth, dev)
     n = 3

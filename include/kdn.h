@@ -330,6 +330,41 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k,
                              void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_backward -- the backward pass of kdn_iso_forward / kdn_diag_forward
+ * (variant): the gradients of a loss L with respect to every input, given
+ * dL/do, dL/dS_T and dL/dp_T ("Kalman Delta Networks: 不确定性感知的联想记忆",
+ * 实验: the layers are trained in language models).  It runs the forward
+ * again on the token-recurrent kernel, saving the state before every token
+ * in the workspace, then the adjoint recursion from the last token to the
+ * first (dS, dp carried backwards).
+ *
+ * q, k, v, a, w, r, S0, p0, info_scale, in_dtype: as the forward call
+ * dO       [B, T, H, dv] fp32 device: dL/do
+ * dS_T     [B, H, dv, dk], dp_T [B, H] (iso) or [B, H, dk] (diag) fp32
+ *          device, or NULL for zero
+ * dq, dk   [B, T, H, dk];  dv [B, T, H, dv];  da, dr [B, T, H];
+ * dw       [B, T, H] (iso) or [B, T, H, dk] (diag);  dS0 [B, H, dv, dk];
+ * dp0      [B, H] (iso) or [B, H, dk] (diag): fp32 device outputs
+ * workspace   device scratch of >= kdn_backward_workspace_size(...) bytes,
+ *          256-byte aligned: B H T (dv dk + 1 or dk) floats of saved state,
+ *          plus the forward's outputs
+ * Supported: dk in {32, 64}; 1 <= dv <= 128; every pointer 16-byte aligned.
+ * Errors: KDN_ERR_INVALID_ARG, KDN_ERR_UNSUPPORTED, KDN_ERR_WORKSPACE,
+ * KDN_ERR_CUDA, all before anything is enqueued except KDN_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+size_t kdn_backward_workspace_size(kdn_variant variant, int B, int T, int H,
+                                   int dk, int dv);
+kdn_status kdn_backward(kdn_variant variant, const void* q, const void* k,
+                        const void* v, kdn_dtype in_dtype, const float* a,
+                        const float* w, const float* r, const float* S0,
+                        const float* p0, const float* dO, const float* dS_T,
+                        const float* dp_T, float* dq, float* dk, float* dv,
+                        float* da, float* dw, float* dr, float* dS0,
+                        float* dp0, int B, int T, int H, int dk_dim,
+                        int dv_dim, float info_scale, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_kla_forward -- the diagonal Kalman filter in information form ("Kalman
  * Linear Attention: Parallel Bayesian Filtering ...", 方法论 §1-§3): a
  * precision per key dimension, updated by a Mobius map of the previous one,

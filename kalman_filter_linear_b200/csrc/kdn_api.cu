@@ -22,7 +22,8 @@ kdn_status recurrent_launch(bool diag, kdn_dtype dt, const void* q, const void* 
                             const float* a, const float* w, const float* r, const float* S0,
                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
                             int H, int dk, int dv, float kappa, cudaStream_t s,
-                            const int* cu_seqlens = nullptr, uint32_t* err = nullptr);
+                            const int* cu_seqlens = nullptr, uint32_t* err = nullptr,
+                            float* Ssave = nullptr, float* Psave = nullptr);
 bool chunk_engine_supported(kdn_dtype dt, int dk, int dv);
 size_t chunk_engine_workspace_size(bool diag, int B, int H);
 kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const void* v,
@@ -36,6 +37,13 @@ kdn_status exact_kalman_launch(bool diag, kdn_dtype dt, const void* q, const voi
                                const void* v, const float* a, const float* w, const float* r,
                                const float* S0, const float* P0, float* o, float* S_out,
                                float* P_out, int B, int T, int H, int dk, int dv, cudaStream_t s);
+bool backward_supported(int dk, int dv);
+kdn_status backward_launch(bool diag, kdn_dtype dt, const void* q, const void* k, const void* v,
+                           const float* a, const float* w, const float* r, const float* dO,
+                           const float* dS_T, const float* dp_T, const float* Ssave,
+                           const float* Psave, float* dq, float* dk, float* dv_, float* da,
+                           float* dw, float* dr, float* dS0, float* dp0, int B, int T, int H,
+                           int dkk, int dv, float kappa, cudaStream_t s);
 bool kla_supported(int dk, int dv);
 kdn_status kla_launch(kdn_dtype dt, const void* q, const void* k, const void* v, const float* a,
                       const float* w, const float* r, const float* S0, const float* L0, float* o,
@@ -280,6 +288,72 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k, 
   if (!kdn::exact_kalman_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
   return kdn::exact_kalman_launch(variant == KDN_DIAG, in_dtype, q, k, v, a, w, r, S0, P0, o,
                                   S_out, P_out, B, T, H, dk, dv, as_stream(stream));
+}
+
+namespace {
+// backward workspace: saved states, saved variances, then the forward's
+// outputs (o, S_T, p_T), each region 256-byte aligned
+struct BwdLayout {
+  size_t states, vars, o, s, p, bytes;
+};
+inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+BwdLayout bwd_layout(bool diag, int B, int T, int H, int dk, int dv) {
+  BwdLayout L{};
+  const size_t bh = (size_t)B * H, np = diag ? (size_t)dk : 1;
+  L.states = 0;
+  L.vars = al256(bh * T * dv * dk * 4);
+  L.o = L.vars + al256(bh * T * np * 4);
+  L.s = L.o + al256((size_t)B * T * H * dv * 4);
+  L.p = L.s + al256(bh * dv * dk * 4);
+  L.bytes = L.p + al256(bh * np * 4);
+  return L;
+}
+}  // namespace
+
+size_t kdn_backward_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv) {
+  if ((variant != KDN_ISO && variant != KDN_DIAG) || !shape_ok(B, T, H, dk, dv) ||
+      !kdn::backward_supported(dk, dv))
+    return 0;
+  return bwd_layout(variant == KDN_DIAG, B, T, H, dk, dv).bytes;
+}
+
+kdn_status kdn_backward(kdn_variant variant, const void* q, const void* k, const void* v,
+                        kdn_dtype in_dtype, const float* a, const float* w, const float* r,
+                        const float* S0, const float* p0, const float* dO, const float* dS_T,
+                        const float* dp_T, float* dq, float* dk_, float* dv_, float* da,
+                        float* dw, float* dr, float* dS0, float* dp0, int B, int T, int H, int dk,
+                        int dv, float info_scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  if (!q || !k || !v || !a || !w || !r || !dO || !dq || !dk_ || !dv_ || !da || !dw || !dr ||
+      !dS0 || !dp0)
+    return KDN_ERR_INVALID_ARG;
+  if (variant != KDN_ISO && variant != KDN_DIAG) return KDN_ERR_INVALID_ARG;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  if (!(info_scale == info_scale) || info_scale > 3.0e38f) return KDN_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(a) || !al16(w) || !al16(r) || !al16(dO) ||
+      !al16(dq) || !al16(dk_) || !al16(dv_) || !al16(da) || !al16(dw) || !al16(dr) ||
+      !al16(dS0) || !al16(dp0) || !al16_or_null(S0) || !al16_or_null(p0) ||
+      !al16_or_null(dS_T) || !al16_or_null(dp_T))
+    return KDN_ERR_INVALID_ARG;
+  if (!kdn::backward_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
+  const bool diag = variant == KDN_DIAG;
+  const BwdLayout L = bwd_layout(diag, B, T, H, dk, dv);
+  if (!workspace || workspace_bytes < L.bytes) return KDN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDN_ERR_INVALID_ARG;
+  char* ws = static_cast<char*>(workspace);
+  float* Ssave = reinterpret_cast<float*>(ws + L.states);
+  float* Psave = reinterpret_cast<float*>(ws + L.vars);
+  const float kappa = diag ? 1.f : (info_scale > 0.f ? info_scale : 1.f / (float)dk);
+  // the forward again, saving the state before every token
+  kdn_status st = kdn::recurrent_launch(
+      diag, in_dtype, q, k, v, a, w, r, S0, p0, reinterpret_cast<float*>(ws + L.o),
+      reinterpret_cast<float*>(ws + L.s), reinterpret_cast<float*>(ws + L.p), B, T, H, dk, dv,
+      kappa, as_stream(stream), nullptr, nullptr, Ssave, Psave);
+  if (st != KDN_OK) return st;
+  return kdn::backward_launch(diag, in_dtype, q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq,
+                              dk_, dv_, da, dw, dr, dS0, dp0, B, T, H, dk, dv, kappa,
+                              as_stream(stream));
 }
 
 kdn_status kdn_kla_forward(const void* q, const void* k, const void* v, kdn_dtype in_dtype,

@@ -62,13 +62,16 @@ __device__ __forceinline__ void load_state(const float* p, int lane, float (&x)[
 
 // Layout of the per-token tensors: q/k/v at ((b*T + t)*H + h)*d; a/w/r at
 // (b*T + t)*H + h (diag w: ((b*T + t)*H + h)*dk).  The decode step is T = 1.
-template <bool DIAG, int CPL, typename InT>
+// SAVE: the state (S, p) before every token is also written to Ssave /
+// Psave ([B H][T][dv][dk] and [B H][T][1 or dk]) for the backward pass.
+template <bool DIAG, int CPL, typename InT, bool SAVE>
 __global__ void __launch_bounds__(kWarps * 32)
 recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __restrict__ V,
                  const float* __restrict__ A, const float* __restrict__ Wn,
                  const float* __restrict__ R, const float* S0, const float* P0,
                  float* __restrict__ O, float* S_out, float* P_out, int T, int H, int dv,
-                 float kappa, const int* __restrict__ cu_seqlens, uint32_t* err) {
+                 float kappa, const int* __restrict__ cu_seqlens, uint32_t* err,
+                 float* __restrict__ Ssave, float* __restrict__ Psave) {
   constexpr int DK = CPL * 32;
   const int bh = blockIdx.x;
   const int h = bh % H;
@@ -112,6 +115,25 @@ recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT
 
   for (int t = 0; t < Tn; ++t) {
     const size_t tok = (row0 + t) * H + h;
+    if constexpr (SAVE) {
+      const size_t sb = ((size_t)bh * T + t) * dv * DK;
+#pragma unroll
+      for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+        const int j = warp + kWarps * i;
+        if (j < dv) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) Ssave[sb + (size_t)j * DK + lane * CPL + c] = S[i][c];
+        }
+      }
+      if constexpr (DIAG) {
+        if (warp == 0) {
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) Psave[((size_t)bh * T + t) * DK + lane * CPL + c] = p[c];
+        }
+      } else {
+        if (threadIdx.x == 0) Psave[(size_t)bh * T + t] = p[0];
+      }
+    }
     float k[CPL], q[CPL];
     load_vec<CPL>(K + tok * DK, lane, k);
     load_vec<CPL>(Q + tok * DK, lane, q);
@@ -220,10 +242,16 @@ template <bool DIAG, int CPL, typename InT>
 kdn_status launch_t(const void* q, const void* k, const void* v, const float* a, const float* w,
                     const float* r, const float* S0, const float* p0, float* o, float* S_out,
                     float* p_out, int B, int T, int H, int dv, float kappa, cudaStream_t s,
-                    const int* cu, uint32_t* err) {
-  recurrent_kernel<DIAG, CPL, InT><<<B * H, kWarps * 32, 0, s>>>(
-      static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w, r,
-      S0, p0, o, S_out, p_out, T, H, dv, kappa, cu, err);
+                    const int* cu, uint32_t* err, float* Ssave, float* Psave) {
+  if (Ssave) {
+    recurrent_kernel<DIAG, CPL, InT, true><<<B * H, kWarps * 32, 0, s>>>(
+        static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w,
+        r, S0, p0, o, S_out, p_out, T, H, dv, kappa, cu, err, Ssave, Psave);
+  } else {
+    recurrent_kernel<DIAG, CPL, InT, false><<<B * H, kWarps * 32, 0, s>>>(
+        static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w,
+        r, S0, p0, o, S_out, p_out, T, H, dv, kappa, cu, err, nullptr, nullptr);
+  }
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
@@ -231,11 +259,11 @@ template <bool DIAG, typename InT>
 kdn_status launch_dk(const void* q, const void* k, const void* v, const float* a, const float* w,
                      const float* r, const float* S0, const float* p0, float* o, float* S_out,
                      float* p_out, int B, int T, int H, int dk, int dv, float kappa,
-                     cudaStream_t s, const int* cu, uint32_t* err) {
+                     cudaStream_t s, const int* cu, uint32_t* err, float* Ssave, float* Psave) {
   switch (dk) {
-    case 32: return launch_t<DIAG, 1, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
-    case 64: return launch_t<DIAG, 2, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
-    case 128: return launch_t<DIAG, 4, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err);
+    case 32: return launch_t<DIAG, 1, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err, Ssave, Psave);
+    case 64: return launch_t<DIAG, 2, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err, Ssave, Psave);
+    case 128: return launch_t<DIAG, 4, InT>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, s, cu, err, Ssave, Psave);
     default: return KDN_ERR_UNSUPPORTED;
   }
 }
@@ -248,15 +276,15 @@ kdn_status recurrent_launch(bool diag, kdn_dtype dt, const void* q, const void* 
                             const float* a, const float* w, const float* r, const float* S0,
                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
                             int H, int dk, int dv, float kappa, cudaStream_t s,
-                            const int* cu_seqlens, uint32_t* err) {
+                            const int* cu_seqlens, uint32_t* err, float* Ssave, float* Psave) {
   if (diag) {
     return dt == KDN_BF16
-               ? launch_dk<true, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err)
-               : launch_dk<true, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err);
+               ? launch_dk<true, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err, Ssave, Psave)
+               : launch_dk<true, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err, Ssave, Psave);
   }
   return dt == KDN_BF16
-             ? launch_dk<false, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err)
-             : launch_dk<false, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err);
+             ? launch_dk<false, __nv_bfloat16>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err, Ssave, Psave)
+             : launch_dk<false, float>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dk, dv, kappa, s, cu_seqlens, err, Ssave, Psave);
 }
 
 }  // namespace kdn

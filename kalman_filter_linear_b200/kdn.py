@@ -75,6 +75,11 @@ def lib():
         [_f32, _vp]
     L.kdn_exact_forward.restype = _i32
     L.kdn_exact_forward.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
+    L.kdn_backward_workspace_size.restype = _sz
+    L.kdn_backward_workspace_size.argtypes = [_i32] * 6
+    L.kdn_backward.restype = _i32
+    L.kdn_backward.argtypes = [_i32, _vp, _vp, _vp, _i32] + [_vp] * 16 + [_i32] * 5 + \
+        [_f32, _vp, _sz, _vp]
     L.kdn_kla_forward.restype = _i32
     L.kdn_kla_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
     L.kdn_read_workspace_status.restype = _i32
@@ -405,6 +410,54 @@ def kdn_exact_forward(variant, q, k, v, a, w, r, S0=None, P0=None, o=None, S_out
                                  B, T, H, dk, dv, _stream())
     _check(st, 'kdn_exact_forward')
     return o, S_out, P_out
+
+
+def kdn_backward_workspace_size(variant, B, T, H, dk, dv):
+    return int(lib().kdn_backward_workspace_size(variant, B, T, H, dk, dv))
+
+
+def kdn_backward(variant, q, k, v, a, w, r, dO, S0=None, p0=None, dS_T=None, dp_T=None,
+                 info_scale=0.0, workspace=None):
+    """Backward of the layer forward: returns a dict of the gradients
+    q, k, v, a, w, r, S0, p0 (fp32, shaped like the inputs) of the loss whose
+    gradients with respect to o, S_T and p_T are dO, dS_T, dp_T."""
+    var = KDN_DIAG if variant in ('diag', KDN_DIAG) else KDN_ISO
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = q.dtype
+    _in_dtype(q)
+    _req(q, 'q', dt)
+    _req(k, 'k', dt, (B, T, H, dk))
+    _req(v, 'v', dt, (B, T, H, dv))
+    f = torch.float32
+    _req(a, 'a', f, (B, T, H))
+    _req(r, 'r', f, (B, T, H))
+    wshape = (B, T, H) if var == KDN_ISO else (B, T, H, dk)
+    pshape = (B, H) if var == KDN_ISO else (B, H, dk)
+    _req(w, 'w', f, wshape)
+    _req(dO, 'dO', f, (B, T, H, dv))
+    _opt(S0, 'S0', f, (B, H, dv, dk))
+    _opt(p0, 'p0', f, pshape)
+    _opt(dS_T, 'dS_T', f, (B, H, dv, dk))
+    _opt(dp_T, 'dp_T', f, pshape)
+    dev = q.device
+    g = dict(q=torch.empty((B, T, H, dk), dtype=f, device=dev),
+             k=torch.empty((B, T, H, dk), dtype=f, device=dev),
+             v=torch.empty((B, T, H, dv), dtype=f, device=dev),
+             a=torch.empty((B, T, H), dtype=f, device=dev),
+             w=torch.empty(wshape, dtype=f, device=dev),
+             r=torch.empty((B, T, H), dtype=f, device=dev),
+             S0=torch.empty((B, H, dv, dk), dtype=f, device=dev),
+             p0=torch.empty(pshape, dtype=f, device=dev))
+    need = kdn_backward_workspace_size(var, B, T, H, dk, dv)
+    workspace = _workspace(need, dev, workspace)
+    st = lib().kdn_backward(var, _ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w),
+                            _ptr(r), _ptr(S0), _ptr(p0), _ptr(dO), _ptr(dS_T), _ptr(dp_T),
+                            _ptr(g['q']), _ptr(g['k']), _ptr(g['v']), _ptr(g['a']), _ptr(g['w']),
+                            _ptr(g['r']), _ptr(g['S0']), _ptr(g['p0']), B, T, H, dk, dv,
+                            float(info_scale), _ptr(workspace), workspace.numel(), _stream())
+    _check(st, 'kdn_backward')
+    return g
 
 
 def kdn_kla_forward(q, k, v, a, w, r, S0=None, lam0=None, o=None, S_out=None, lam_out=None):

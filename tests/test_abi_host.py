@@ -148,3 +148,21 @@ def test_kla_forward_rejects_bad_arguments(L):
     assert x(dk=96) == kdn.KDN_ERR_UNSUPPORTED
     assert x(dv=4) == kdn.KDN_ERR_UNSUPPORTED
     assert x(dv=130) == kdn.KDN_ERR_UNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments(L):
+    base = dict(var=kdn.KDN_ISO, q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_F32, a=FAKE, w=FAKE, r=FAKE,
+                S0=None, p0=None, dO=FAKE, dS_T=None, dp_T=None, dq=FAKE, dk=FAKE, dv=FAKE,
+                da=FAKE, dw=FAKE, dr=FAKE, dS0=FAKE, dp0=FAKE, B=1, T=8, H=1, dkk=64, dvv=64,
+                kappa=0.0, ws=ctypes.c_void_p(0x20000), wsb=1 << 40, stream=None)
+    x = lambda **kw: L.kdn_backward(*dict(base, **kw).values())
+    assert x(dO=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dp0=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(var=5) == kdn.KDN_ERR_INVALID_ARG
+    assert x(T=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dS_T=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dkk=128) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(dvv=129) == kdn.KDN_ERR_INVALID_ARG or x(dvv=129) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(ws=None) == kdn.KDN_ERR_WORKSPACE
+    assert x(wsb=16) == kdn.KDN_ERR_WORKSPACE
+    assert L.kdn_backward_workspace_size(kdn.KDN_DIAG, 2, 10, 3, 32, 16) >= 2 * 3 * 10 * 16 * 32 * 4

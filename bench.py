@@ -257,7 +257,8 @@ def main():
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
-    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact', 'kla'],
+    ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact', 'kla',
+                                       'bwd'],
                     help='run only this kernel (for profiler captures) and print its timing')
     ap.add_argument('--B', type=int, default=None, help='batch override for --only')
     ap.add_argument('--T', type=int, default=None, help='length override for --only')
@@ -412,6 +413,17 @@ def run_only(args):
         f, units, alg, _ = varlen_case(kdn, synth, dev)
     elif args.only == 'exact':
         f, units, alg, _ = exact_case(kdn, synth, dev, args.B, args.T)
+    elif args.only == 'bwd':
+        c = synth.WORKLOADS['exact_d64']
+        B, T, H, d = args.B or c['B'], args.T or c['T'], c['H'], c['dk']
+        x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'iso', c['seed'],
+                                                         c['dtype']).items()}
+        dO = torch.randn((B, T, H, d), device=dev)
+        wsb = torch.empty(kdn.kdn_backward_workspace_size(kdn.KDN_ISO, B, T, H, d, d),
+                          dtype=torch.uint8, device=dev)
+        f = lambda: kdn.kdn_backward('iso', x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,
+                                     workspace=wsb)
+        units, alg = B * T, backward_bytes(B, T, H, d)
     elif args.only == 'kla':
         c = synth.WORKLOADS['diag_1p3b']
         B, T, H, d = args.B or c['B'], args.T or c['T'], c['H'], c['dk']
@@ -458,6 +470,15 @@ def varlen_case(kdn, synth, dev):
     desc = {'sequences': N, 'tokens': total, 'max_len': max(lengths),
             'min_len': min(lengths), 'H': H, 'd': d}
     return f, total, alg, desc
+
+
+def backward_bytes(B, T, H, d, in_bytes=2):
+    """Algorithmic HBM bytes of one backward call (isotropic, d_k = d_v = d):
+    inputs read twice (the forward again, then the backward), dO read, the
+    forward's o written, the saved states and variances written and read
+    once, the gradients of q, k, v, a, w, r written."""
+    return (2 * B * T * H * (3 * d * in_bytes + 12) + 2 * B * T * H * d * 4 +
+            2 * B * H * T * (d * d + 1) * 4 + B * T * H * (3 * d + 3) * 4)
 
 
 def exact_bytes(B, T, H, dk, dv, in_bytes=2):
@@ -598,10 +619,7 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
                                  workspace=wsb)
     n = 2
     ms = time_launches(f, n, 2, stream) / n
-    # inputs read twice (the forward again, then the backward), the saved
-    # states written and read once, gradients written
-    alg = (2 * B * T * H * (3 * d * 2 + 12) + B * T * H * d * 4 +
-           2 * B * H * T * (d * d + 1) * 4 + B * T * H * (3 * d + 3) * 4)
+    alg = backward_bytes(B, T, H, d)
     out['backward_d64'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms,
                            'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                            'algorithmic_bytes': alg, 'B': B, 'T': T, 'H': H, 'd': d}

@@ -371,10 +371,15 @@ kdn_status launch_x(const void* q, const void* k, const void* v, const float* a,
                     float* P_out, int B, int T, int H, int dv, cudaStream_t s) {
   using X = XPlan<DK, SW, DIAG, InT>;
   auto kern = exact_kalman_kernel<DK, SW, DIAG, InT>;
-  if (X::TOTAL > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, X::TOTAL) !=
-          cudaSuccess)
-    return KDN_ERR_CUDA;
+  // the shared-memory opt-in is a property of the function: set it once per
+  // instantiation (a race between first calls sets the same value twice)
+  static bool smem_set = false;
+  if (X::TOTAL > 48 * 1024 && !smem_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, X::TOTAL) !=
+        cudaSuccess)
+      return KDN_ERR_CUDA;
+    smem_set = true;
+  }
   kern<<<(unsigned)(B * H), (X::PW + SW) * 32, X::TOTAL, s>>>(
       static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w, r,
       S0, P0, o, S_out, P_out, T, H, dv);

@@ -418,7 +418,8 @@ def run_only(args):
         B, T, H, d = args.B or c['B'], args.T or c['T'], c['H'], c['dk']
         x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'iso', c['seed'],
                                                          c['dtype']).items()}
-        dO = torch.randn((B, T, H, d), device=dev)
+        dO = torch.randn((B, T, H, d),
+                         generator=torch.Generator().manual_seed(c['seed'] + 100)).to(dev)
         wsb = torch.empty(kdn.kdn_backward_workspace_size(kdn.KDN_ISO, B, T, H, d, d),
                           dtype=torch.uint8, device=dev)
         f = lambda: kdn.kdn_backward('iso', x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,
@@ -612,7 +613,8 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     B, T, H, d = c['B'], c['T'], c['H'], c['dk']
     x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'iso', c['seed'],
                                                      c['dtype']).items()}
-    dO = torch.randn((B, T, H, d), device=dev)
+    dO = torch.randn((B, T, H, d),
+                     generator=torch.Generator().manual_seed(c['seed'] + 100)).to(dev)
     wsb = torch.empty(kdn.kdn_backward_workspace_size(kdn.KDN_ISO, B, T, H, d, d),
                       dtype=torch.uint8, device=dev)
     f = lambda: kdn.kdn_backward('iso', x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,

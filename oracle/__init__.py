@@ -31,8 +31,9 @@ itself -- ``tests/test_oracle_pins.py`` (brute-force Gaussian conditioning,
 numerical KL minimisation, closed forms, Mobius algebra, the gated delta rule,
 invariants), ``tests/test_kla_pins.py`` (scalar-chain conditioning, the
 Diagonal KDN special cases, the precision fixed point) and
-``tests/test_grad_pins.py`` (finite differences of the forward). The one "parity unpinned" item is agreement with the KDN paper's
-own equations, which no page prints: the reading of the process noise
+``tests/test_grad_pins.py`` (finite differences of the forward).  The one
+"parity unpinned" item is agreement with the KDN paper's own equations, which
+no page prints: the reading of the process noise
 (p_prior = a^2 p + w) and of the isotropic information scale (kappa = 1/d_k)
 are the plainest readings the pages support, not the paper's verified text.
 """

@@ -49,3 +49,23 @@ def test_backward_defaults():
                                 f64(dO))
     for name in ref:
         assert rel_maxabs(got[name], ref[name]) <= GRAD_TOL, name
+
+
+def test_backward_full_size_sampled_heads():
+    """The benchmark shape (B8 T4096 H16, d_k = d_v = 64, bf16, isotropic):
+    sampled heads against the oracle over all 4096 tokens."""
+    c = synth.WORKLOADS['exact_d64']
+    B, T, H, d = c['B'], c['T'], c['H'], c['dk']
+    x = synth.layer_inputs(B, T, H, d, d, 'iso', seed=c['seed'], dtype=c['dtype'])
+    dO = torch.randn(B, T, H, d, generator=torch.Generator().manual_seed(c['seed'] + 100))
+    xd = {k: v.cuda() for k, v in x.items()}
+    got = kdn.kdn_backward('iso', xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'],
+                           dO.cuda())
+    torch.cuda.synchronize()
+    for b, h in [(0, 0), (7, 15)]:
+        sl = {n: f64(x[n][b:b + 1, :, h:h + 1]) for n in ('q', 'k', 'v', 'a', 'w', 'r')}
+        ref = kdn_grad.kdn_backward('iso', sl['q'], sl['k'], sl['v'], sl['a'], sl['w'], sl['r'],
+                                    f64(dO[b:b + 1, :, h:h + 1]))
+        for name in ('q', 'k', 'v', 'a', 'w', 'r'):
+            assert rel_maxabs(got[name][b, :, h], ref[name][0, :, 0]) <= GRAD_TOL, (name, b, h)
+        assert rel_maxabs(got['S0'][b, h], ref['S0'][0, 0]) <= GRAD_TOL

@@ -166,3 +166,44 @@ def test_backward_rejects_bad_arguments(L):
     assert x(ws=None) == kdn.KDN_ERR_WORKSPACE
     assert x(wsb=16) == kdn.KDN_ERR_WORKSPACE
     assert L.kdn_backward_workspace_size(kdn.KDN_DIAG, 2, 10, 3, 32, 16) >= 2 * 3 * 10 * 16 * 32 * 4
+
+
+def test_varlen_rejects_bad_arguments(L):
+    ws = ctypes.c_void_p(0x20000)
+    base = dict(var=kdn.KDN_ISO, q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_BF16, a=FAKE, w=FAKE, r=FAKE,
+                cu=FAKE, S0=None, p0=None, o=FAKE, S=FAKE, p=FAKE, N=4, total=100, H=2, dk=128,
+                dv=128, kappa=0.0, chunk=0, ws=ws, wsb=1 << 30, stream=None)
+    x = lambda **kw: L.kdn_forward_varlen(*dict(base, **kw).values())
+    assert x(cu=None) == kdn.KDN_ERR_INVALID_ARG         # offsets are required
+    assert x(total=-1) == kdn.KDN_ERR_INVALID_ARG
+    assert x(var=3) == kdn.KDN_ERR_INVALID_ARG
+    assert x(N=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(o=MIS) == kdn.KDN_ERR_INVALID_ARG
+    assert x(ws=None) == kdn.KDN_ERR_WORKSPACE
+    assert x(wsb=64) == kdn.KDN_ERR_WORKSPACE              # at least the 256-byte error word
+    assert x(chunk=kdn.KDN_CHUNK_64, dv=64, dk=128) == kdn.KDN_ERR_UNSUPPORTED
+    assert L.kdn_forward_varlen_workspace_size(kdn.KDN_ISO, 4, 2, 128, 128, 0) >= 256
+    assert L.kdn_forward_varlen_workspace_size(kdn.KDN_ISO, 0, 2, 128, 128, 0) == 0
+
+
+def test_host_forward_rejects_bad_arguments(L):
+    ws = ctypes.c_void_p(0x20000)
+    base = dict(var=kdn.KDN_ISO, q=FAKE, k=FAKE, v=FAKE, dt=kdn.KDN_BF16, a=FAKE, w=FAKE, r=FAKE,
+                S0=None, p0=None, o=FAKE, S=FAKE, p=FAKE, B=2, T=64, H=2, dk=128, dv=128,
+                kappa=0.0, chunk=0, slice_b=1, ws=ws, wsb=1 << 40, stream=None)
+    x = lambda **kw: L.kdn_forward_host(*dict(base, **kw).values())
+    assert x(var=2) == kdn.KDN_ERR_INVALID_ARG
+    assert x(p=None) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dt=5) == kdn.KDN_ERR_INVALID_ARG
+    assert x(T=0) == kdn.KDN_ERR_INVALID_ARG
+    assert x(dk=96) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(ws=None) == kdn.KDN_ERR_WORKSPACE
+    assert x(wsb=1024) == kdn.KDN_ERR_WORKSPACE
+    assert x(ws=ctypes.c_void_p(0x20010)) == kdn.KDN_ERR_INVALID_ARG  # not 256-byte aligned
+    need = L.kdn_forward_host_workspace_size(kdn.KDN_ISO, 2, 64, 2, 128, 128, kdn.KDN_BF16, 0, 1)
+    assert need > 256
+
+
+def test_read_status_rejects_a_missing_workspace(L):
+    assert L.kdn_read_workspace_status(None, 256, None) == kdn.KDN_ERR_INVALID_ARG
+    assert L.kdn_read_workspace_status(FAKE, 2, None) == kdn.KDN_ERR_INVALID_ARG

@@ -340,8 +340,10 @@ def main():
     ms_e2e = time_launches(e2e_step, e2e_steps, 2, stream) / e2e_steps
     e2e_value = whole_job_rate(B * T, world, max_over_ranks(ms_e2e, dist, dev))
 
+    # secondary lines at N = 1 only: at N > 1 the other ranks would wait at the
+    # closing barrier (under the process group's timeout) while rank 0 measures
     secondary = {}
-    if not args.no_secondary and rank == 0:
+    if not args.no_secondary and rank == 0 and world == 1:
         secondary = measure_secondary(kdn, synth, dev, stream, hbm_peak)
 
     cpu = None

@@ -203,7 +203,9 @@ def run_reference(args, rank):
     cfg = synth.WORKLOADS[WORKLOAD]
     B, T, H, d = cfg['B'], cfg['T'], cfg['H'], cfg['dk']
     x = synth.layer_inputs(B, T, H, d, d, 'iso', cfg['seed'], cfg['dtype'])
-    tok = 16  # tokens of all B*H heads per step: a bounded sample of the workload
+    # tokens of all B*H heads per step, a bounded sample of the workload: 16 at
+    # up to 50 steps, fewer for more steps, so the whole run stays near 15 s
+    tok = max(1, min(16, (16 * 50) // max(args.steps, 1)))
     xs = {k: x[k][:, :tok].double().numpy() for k in 'qkvawr'}
     for _ in range(args.warmup):
         kdn_ref.iso_forward(*(xs[n] for n in 'qkvawr'))
@@ -252,7 +254,7 @@ def cpu_baseline(seconds=12.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument('--gpus', type=int, default=1)
-    ap.add_argument('--steps', type=int, default=50)
+    ap.add_argument('--steps', type=int, default=2000)
     ap.add_argument('--warmup', type=int, default=5)
     ap.add_argument('--impl', default='kdn', choices=['kdn', 'reference'])
     ap.add_argument('--no-secondary', action='store_true')

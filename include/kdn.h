@@ -62,7 +62,8 @@ enum {
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* kdn_status_string(kdn_status status);
 
-/* Library version, major*10000 + minor*100 + patch. */
+/* Library version, major*10000 + minor*100 + patch (0.2.0: adds the packed,
+ * host-buffer, backward, dense-filter and KLA entry points). */
 int kdn_version(void);
 
 /* ------------------------------------------------------------------------

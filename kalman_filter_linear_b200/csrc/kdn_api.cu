@@ -195,7 +195,7 @@ const char* kdn_status_string(kdn_status status) {
   return "unknown kdn_status";
 }
 
-int kdn_version(void) { return 100; }
+int kdn_version(void) { return 200; }
 
 size_t kdn_mobius_scan_workspace_size(int64_t N, int64_t T) {
   return kdn::mobius_scan_workspace_size(N, T);

@@ -113,15 +113,20 @@ kdn_status kdn_mobius_scan(const float* a, const float* w, const float* r,
  * code.  Every GPU that loads the library holds it until the process exits.
  * Limit: N * ceil(T / 2048) <= KDN_SCAN_NOALLOC_MAX_TILES (e.g. 4096 lanes
  * up to T = 114688); larger calls return KDN_ERR_WORKSPACE without enqueuing
- * anything.  The call allocates nothing: the first call on a device looks up
- * the array's device address with that device current (documented set-up;
- * make this first call before any stream capture), and every call clears the
- * part of the array that must start at zero on `stream` before its kernel.
- * All calls share the one array: calls whose work overlaps on the GPU (for
- * example on two streams without ordering between them) race and give wrong
- * results, so order them.  A look-back wait that gives up is recorded only in
- * that internal array and is not reported by this entry point.  Otherwise the
- * arguments, results and errors are those of kdn_mobius_scan.
+ * anything.  The call allocates nothing.  Every call looks up the array's
+ * device address in the caller's current device and context (the lookup
+ * allocates nothing), so the address stays right across context switches
+ * and device resets.  The first call in a context also loads the library's
+ * device code there: make that first call before any stream capture.  Every
+ * call clears the part of the array that must start at zero on `stream`
+ * before its kernel.  All calls share the one array: calls whose work
+ * overlaps on the GPU (for example on two streams without ordering between
+ * them) race and give wrong results, so order them.  A look-back wait that
+ * gives up (after 1 s, which only a stalled GPU reaches) is recorded only in
+ * that internal array and is not reported by this entry point; callers that
+ * must detect it use kdn_mobius_scan with a workspace and
+ * kdn_read_workspace_status.  Otherwise the arguments, results and errors
+ * are those of kdn_mobius_scan.
  * ---------------------------------------------------------------------- */
 #define KDN_SCAN_NOALLOC_MAX_TILES 229376
 kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w,

@@ -31,13 +31,26 @@ def sources():
 
 
 def build(verbose=False, extra=()):
+    """Compile every source to an object in parallel, then link the library."""
+    from concurrent.futures import ThreadPoolExecutor
     srcs = sources()
-    cmd = [nvcc(), '-shared', '-Xcompiler', '-fPIC', '-O3', '-lineinfo', '-std=c++17', *ARCH,
-           '-I', os.path.join(ROOT, 'include'), '--expt-relaxed-constexpr',
-           '-Xptxas', '-warn-spills', *extra, '-o', LIB + '.tmp', *srcs, '-lcudart']
-    if verbose:
-        print(' '.join(cmd))
-    subprocess.run(cmd, check=True)
+    objdir = os.path.join(ROOT, '_build')
+    os.makedirs(objdir, exist_ok=True)
+    flags = ['-Xcompiler', '-fPIC', '-O3', '-lineinfo', '-std=c++17', *ARCH,
+             '-I', os.path.join(ROOT, 'include'), '--expt-relaxed-constexpr',
+             '-Xptxas', '-warn-spills', *extra]
+
+    def compile_one(src):
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + '.o')
+        cmd = [nvcc(), '-c', *flags, '-o', obj, src]
+        if verbose:
+            print(' '.join(cmd), flush=True)
+        subprocess.run(cmd, check=True)
+        return obj
+
+    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, srcs))
+    subprocess.run([nvcc(), '-shared', *ARCH, '-o', LIB + '.tmp', *objs, '-lcudart'], check=True)
     os.replace(LIB + '.tmp', LIB)
     return LIB
 

@@ -365,7 +365,12 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
     // timeout and stops
     const bool late = !mbar_wait(&s_full, (uint32_t)(it & 1));
     if (__syncthreads_or(late)) {
-      if (tid == 0) atomicOr(ws.error, DEV_TIMEOUT);
+      if (tid == 0) {
+        atomicOr(ws.error, DEV_TIMEOUT);
+        // the copy may still land in this CTA's buffer: give it one more
+        // bounded wait before the CTA exits and its shared memory is reused
+        (void)mbar_wait(&s_full, (uint32_t)(it & 1));
+      }
       break;
     }
     int64_t j, seq;
@@ -406,9 +411,10 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
     // (the next iteration's first barrier keeps the shared tile state until
     // every thread is done with it)
   }
-  // Nothing is in flight at exit: a copy is started only for a tile below
-  // ntiles, which the next iteration waits for (or gives up on, after which
-  // the CTA stops).
+  // A copy is started only for a tile below ntiles, and the next iteration
+  // waits for it, so on the normal path nothing is in flight at exit.  After
+  // a timeout the CTA waits for the late copy once more (bounded); if that
+  // wait gives up too, the copy can still be in flight when the CTA exits.
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -431,6 +437,39 @@ inline ScanLayout scan_layout(int64_t N, int64_t T) {
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// CTAs of the persistent kernel that fit on the current device at once (its
+// SM count times the CTAs per SM), found once per device with that device
+// current; 0 on a CUDA error.  Devices may differ, so the value is kept per
+// device ordinal, and the first calls from several host threads agree
+// through the lock.
+constexpr int kCapDevices = 64;
+std::atomic<int> g_grid_cap[kCapDevices];
+std::mutex g_grid_cap_mu;
+
+int persistent_grid_cap() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < kCapDevices) {
+    const int cap = g_grid_cap[dev].load(std::memory_order_acquire);
+    if (cap > 0) return cap;
+  }
+  std::lock_guard<std::mutex> lock(g_grid_cap_mu);
+  if (dev < kCapDevices) {
+    const int cap = g_grid_cap[dev].load(std::memory_order_acquire);
+    if (cap > 0) return cap;
+  }
+  int sms = 0, per_sm = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaFuncSetAttribute(mobius_scan_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kBufBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mobius_scan_persistent, kThreads,
+                                                    kBufBytes) != cudaSuccess ||
+      per_sm < 1 || sms < 1)
+    return 0;
+  if (dev < kCapDevices) g_grid_cap[dev].store(sms * per_sm, std::memory_order_release);
+  return sms * per_sm;
+}
 
 }  // namespace
 
@@ -467,19 +506,8 @@ kdn_status mobius_scan_launch(const float* a, const float* w, const float* r, co
   if (cudaMemsetAsync(workspace, 0, L.clear_bytes, stream) != cudaSuccess) return KDN_ERR_CUDA;
   const int vec_ok = (T % 4 == 0) ? 1 : 0;
   if (vec_ok) {
-    static int grid_cap = 0;  // CTAs that fit on the device at once
-    if (grid_cap == 0) {
-      int dev = 0, sms = 0, per_sm = 0;
-      if (cudaGetDevice(&dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-          cudaFuncSetAttribute(mobius_scan_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               kBufBytes) != cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, mobius_scan_persistent, kThreads,
-                                                        kBufBytes) != cudaSuccess ||
-          per_sm < 1)
-        return KDN_ERR_CUDA;
-      grid_cap = sms * per_sm;
-    }
+    const int grid_cap = persistent_grid_cap();
+    if (grid_cap < 1) return KDN_ERR_CUDA;
     const int64_t grid = std::min<int64_t>(L.ntiles, grid_cap);
     mobius_scan_persistent<<<(unsigned)grid, kThreads, kBufBytes, stream>>>(
         a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out, N, T, L.ntiles, ws,
@@ -518,24 +546,18 @@ constexpr size_t kNoAllocBytes =
 
 static __device__ __align__(256) uint8_t g_noalloc_scan_scratch[kNoAllocBytes];
 
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_noalloc_addr[kMaxDevices];
-std::mutex g_noalloc_mu;
-
-// Device address of the scratch array on the current device, looked up once
-// per device with that device current.  In host code the array's name is a
-// host-side stand-in, not a device address, so it is never passed to a kernel.
-void* noalloc_scratch_on_current_device() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
-  if (p) return p;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  p = g_noalloc_addr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+// Device address of the scratch array in the caller's current context.  In
+// host code the array's name is a host-side stand-in, not a device address,
+// so it is never passed to a kernel.  The address is looked up on every call
+// with the caller's device and context current: the lookup allocates
+// nothing, and it stays right when the caller switches contexts on a device
+// or resets the device between calls (a cached address would then point into
+// a context that no longer exists).  The first lookup in a context loads the
+// library's device code there, which is why that first call belongs before
+// any stream capture.
+void* noalloc_scratch_in_current_context() {
   void* addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, g_noalloc_scan_scratch) != cudaSuccess || !addr) return nullptr;
-  g_noalloc_addr[dev].store(addr, std::memory_order_release);
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scan_scratch) != cudaSuccess) return nullptr;
   return addr;
 }
 
@@ -550,7 +572,7 @@ extern "C" kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w, co
   if (N <= 0 || T <= 0 || N * T >= (int64_t(1) << 40)) return KDN_ERR_INVALID_ARG;
   const int64_t tiles = N * ((T + kdn::kTile - 1) / kdn::kTile);
   if (tiles > kdn::kNoAllocMaxTiles) return KDN_ERR_WORKSPACE;
-  void* scratch = kdn::noalloc_scratch_on_current_device();
+  void* scratch = kdn::noalloc_scratch_in_current_context();
   if (!scratch) return KDN_ERR_CUDA;
   return kdn::mobius_scan_launch(a, w, r, n, lambda0, info_scale, lambda_out, prior_out, gain_out,
                                  N, T, scratch, kdn::kNoAllocBytes,

@@ -86,6 +86,35 @@ def layer_inputs(B, T, H, dk, dv, variant='iso', seed=0, dtype='bf16'):
     return dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), a=a, w=w, r=r)
 
 
+def layer_inputs_extreme(B, T, H, dk, dv, variant='iso', seed=0, dtype='bf16'):
+    """Layer inputs at the edges of the coefficient range, as CPU tensors,
+    shaped as ``layer_inputs``.
+
+    Per token and head: a is 1e-3 (a third of the tokens), exactly 1 (a
+    third) or sigmoid(N(2, 0.5)); w = softplus(N(-2, 0.5)) with every fifth
+    token's w exactly 0 (the whole vector, diagonal variant); r = 10^U(-3, 3);
+    k is a unit direction times a norm 10^U(-0.5, 0.3) (so ||k||^2 spans about
+    0.1 to 4); q is a unit direction; v ~ N(0, 1).  Draw order: q, k, the key
+    norms, v, the decay kind, the decay, w, r.
+    """
+    g = _gen(seed)
+    dt = _DT[dtype] if isinstance(dtype, str) else dtype
+    q = _unit(_normal(g, (B, T, H, dk)))
+    k = _unit(_normal(g, (B, T, H, dk)))
+    knorm = torch.pow(10.0, torch.rand((B, T, H, 1), generator=g) * 0.8 - 0.5)
+    k = k * knorm
+    v = _normal(g, (B, T, H, dv))
+    kind = torch.randint(0, 3, (B, T, H), generator=g)
+    a = torch.sigmoid(_normal(g, (B, T, H), 2.0, 0.5))
+    a = torch.where(kind == 0, torch.full_like(a, 1e-3), a)
+    a = torch.where(kind == 1, torch.ones_like(a), a)
+    wshape = (B, T, H) if variant == 'iso' else (B, T, H, dk)
+    w = torch.nn.functional.softplus(_normal(g, wshape, -2.0, 0.5))
+    w[:, ::5] = 0.0
+    r = torch.pow(10.0, torch.rand((B, T, H), generator=g) * 6.0 - 3.0)
+    return dict(q=q.to(dt), k=k.to(dt), v=v.to(dt), a=a, w=w, r=r)
+
+
 def scan_inputs(N, T, seed=1):
     """Inputs of the standalone variance scan: a, w, r, n each [N, T] fp32.
 

@@ -143,3 +143,49 @@ def test_chunked_bounded_wait_reports_timeout_and_context_survives(variant):
     o_r, S_r, p_r = _ref(variant, x)
     assert rel_maxabs(o, o_r) <= OUT_TOL
     assert rel_maxabs(S, S_r) <= STATE_TOL
+
+
+def _per_head_err(o, o_ref, S, S_ref):
+    """Per (b, h): max-abs error over the reference's RMS, for o [B,T,H,dv]
+    and S [B,H,dv,dk]; computed on the device."""
+    eo = (o - o_ref).abs().amax(dim=(1, 3)) / o_ref.pow(2).mean(dim=(1, 3)).sqrt()
+    eS = (S - S_ref).abs().amax(dim=(2, 3)) / S_ref.pow(2).mean(dim=(2, 3)).sqrt()
+    return eo, eS
+
+
+@pytest.mark.parametrize("name", ["iso_1p3b", "diag_1p3b", "diag_long"])
+def test_engine_full_width_matches_recurrent_kernel(name):
+    """Every head and every token of the benchmark launches: the chunked
+    engine against the token-recurrent kernel (itself checked against the
+    oracle), each head within the layer tolerances."""
+    c = synth.WORKLOADS[name]
+    x = to_dev(synth.layer_inputs(c['B'], c['T'], c['H'], c['dk'], c['dv'], c['variant'],
+                                  c['seed'], c['dtype']))
+    o1, S1, p1 = _run(c['variant'], x, chunk=kdn.KDN_CHUNK_AUTO)
+    o2, S2, p2 = _run(c['variant'], x, chunk=kdn.KDN_CHUNK_RECURRENT)
+    eo, eS = _per_head_err(o1, o2, S1, S2)
+    assert float(eo.max()) <= OUT_TOL, float(eo.max())
+    assert float(eS.max()) <= STATE_TOL, float(eS.max())
+    ep = float(((p1 - p2).abs() / p2.abs()).max())
+    assert ep <= 1e-4, ep
+
+
+@pytest.mark.parametrize("variant", ["iso", "diag"])
+@pytest.mark.parametrize("T,dv", [(63, 128), (129, 128), (63, 64), (129, 64)])
+def test_engine_extreme_coefficients(variant, T, dv):
+    """Decays of 1e-3 and exactly 1, zero process noise, observation noise
+    over six decades and key norms away from 1 (the log-space decay prefix,
+    the gains and the variance carry at their edges), against the oracle."""
+    B, H, dk = 1, 2, 128
+    x = to_dev(synth.layer_inputs_extreme(B, T, H, dk, dv, variant, seed=T + dv + 7,
+                                          dtype='bf16'))
+    g = torch.Generator().manual_seed(T + 1)
+    S0 = (0.05 * torch.randn(B, H, dv, dk, generator=g)).cuda()
+    p0 = (torch.rand((B, H) if variant == 'iso' else (B, H, dk), generator=g) + 0.2).cuda()
+    o, S, p = _run(variant, x, S0, p0, chunk=kdn.KDN_CHUNK_AUTO)
+    o_r, S_r, p_r = _ref(variant, x, S0, p0)
+    assert torch.isfinite(o).all() and torch.isfinite(S).all()
+    eo, eS = rel_maxabs(o, o_r), rel_maxabs(S, S_r)
+    assert eo <= OUT_TOL, eo
+    assert eS <= STATE_TOL, eS
+    np.testing.assert_allclose(f64(p), p_r, rtol=1e-5)

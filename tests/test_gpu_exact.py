@@ -49,10 +49,14 @@ def _oracle(variant, x, S0, P0, heads):
 
 @pytest.mark.parametrize("variant", ["iso", "diag"])
 @pytest.mark.parametrize("dk,dv,dtype", [(64, 64, 'bf16'), (32, 128, 'f32'), (64, 40, 'f32'),
-                                         (32, 24, 'bf16')])
+                                         (32, 24, 'bf16'), (64, 8, 'f32'), (64, 24, 'bf16'),
+                                         (32, 48, 'f32'), (64, 128, 'bf16')])
 def test_exact_matches_dense_oracle(variant, dk, dv, dtype):
     """Random SPD P0 and a non-zero S0; T = 150 spans nine 16-token stages
-    and a ragged one."""
+    and a ragged one.  The shapes take every state-warp count the kernel has:
+    one (d_v rows of d_k / 32 lanes fit in a warp: (32, 24), (64, 8)), two
+    ((64, 24), (32, 48)), four ((64, 64), (32, 128), (64, 40)) and eight
+    ((64, 128))."""
     B, T, H = 2, 150, 2
     x = synth.layer_inputs(B, T, H, dk, dv, variant, seed=31 + dk + dv, dtype=dtype)
     g = torch.Generator().manual_seed(5)

@@ -27,10 +27,13 @@ def _run(x, S0=None, lam0=None):
 
 
 @pytest.mark.parametrize("dk,dv,dtype", [(128, 128, 'bf16'), (64, 64, 'f32'), (32, 40, 'bf16'),
-                                         (128, 56, 'f32'), (64, 128, 'bf16')])
+                                         (128, 56, 'f32'), (64, 128, 'bf16'), (128, 8, 'f32'),
+                                         (64, 16, 'bf16'), (32, 32, 'f32'), (128, 24, 'bf16')])
 def test_kla_matches_oracle(dk, dv, dtype):
     """Non-zero S0 and random precisions; T = 150 spans nine 16-token chunks
-    and a ragged one."""
+    and a ragged one.  The shapes take every state-warp count the kernel has
+    (8 rows of S a warp): one (d_v 8), two (16), four (24, 32), eight (40 to
+    64) and sixteen (128)."""
     B, T, H = 2, 150, 2
     x = synth.layer_inputs(B, T, H, dk, dv, 'diag', seed=61 + dk + dv, dtype=dtype)
     g = torch.Generator().manual_seed(62)

@@ -3,8 +3,9 @@ memory at the call (their host owns all device memory through its own pool,
 or hands them only input and output buffers).  Its scratch is a fixed array
 inside the library, so the test checks, through the C ABI, that two calls in
 a row (the second reusing what the first left in that array) both match the
-workspace-taking kdn_mobius_scan, and that a size beyond the array's limit is
-refused.  This file is collected last on purpose.
+workspace-taking kdn_mobius_scan, that the first case also matches the fp64
+oracle directly, and that a size beyond the array's limit is refused.  This
+file is collected last on purpose.
 """
 import ctypes
 
@@ -12,7 +13,8 @@ import pytest
 import torch
 
 from kalman_filter_linear_b200 import kdn, synth
-from gpu_util import SCAN_RTOL, max_rel
+from oracle import kdn_ref
+from gpu_util import SCAN_RTOL, max_rel, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -45,6 +47,13 @@ def test_noalloc_scan_matches_workspace_scan_twice_in_a_row():
         if aux:
             assert max_rel(g[1], ref[1].double().cpu().numpy()) <= SCAN_RTOL
             assert max_rel(g[2], ref[2].double().cpu().numpy()) <= SCAN_RTOL
+    # the first case against the oracle itself (variances, priors, gains)
+    x, l0, (N, T, kappa, _), g = inputs[0], lam0s[0], cases[0], got[0]
+    a, w, r, n = (f64(x[k]) for k in 'awrn')
+    prior, post = kdn_ref.variance_scan(a, w, r, kappa * n, f64(l0))
+    assert max_rel(g[0], post) <= SCAN_RTOL
+    assert max_rel(g[1], prior) <= SCAN_RTOL
+    assert max_rel(g[2], prior / (prior * n + r)) <= SCAN_RTOL
 
 
 def test_noalloc_scan_rejects_sizes_beyond_its_scratch():

@@ -160,6 +160,22 @@ kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w,
  *             256-byte aligned (NULL allowed when that size is 0).  The
  *             chunked path keeps its device error word and a copy of p0
  *             there; kdn_read_workspace_status() reads the error word.
+ *             The size depends on B, T, H and the current device: few heads
+ *             over a long sequence take the segmented forward below, whose
+ *             scratch (per segment: a state transition, a state and the
+ *             start variances) is much larger, so query the size with the
+ *             device that will run the call current.
+ * Segmented forward: with dk = dv = 128 on the chunked path, when B H is at
+ * most a quarter of the SM count and T is a multiple of 4096 (the segment
+ * count S, a power of two >= 4 with B H S <= SMs and 1024 S dividing T, is
+ * chosen by the library), the sequence is cut into S segments run as extra
+ * heads of the engine: the variance at each segment start from the composed
+ * Mobius maps, each segment's state transition from a run with V = 0 and
+ * S0 = I and its zero-start state from a run with S0 = 0, the segment
+ * starts chained, and a last run from the true starts.  The memory
+ * recursion is affine in the state, so the result is the same up to
+ * rounding; it takes three engine passes over T / S tokens each instead of
+ * one over T.
  * Supported: T >= 1; dk in {32, 64, 128}; 1 <= dv <= 128.  KDN_CHUNK_64
  * additionally needs in_dtype == KDN_BF16, dk == 128 and dv in {64, 128}.
  * All pointers 16-byte aligned.  o must not alias the inputs.

@@ -2237,16 +2237,20 @@ kdn_status launch(const void* q, const void* k, const void* v, const float* a, c
 }
 
 // (cu_seqlens: B packed sequences in [1, T, H, d] tensors, T = total tokens)
+// (v_zero_rows > 0: v is a zeroed [1, v_zero_rows, H, 128] buffer, so every V
+// copy reads zeros, inside it or past its bounds, where TMA fills zeros)
 template <bool DIAG>
 kdn_status launch_ws(const void* q, const void* k, const void* v, const float* a,
                      const float* w, const float* r, const float* S0, const float* p0, float* o,
                      float* S_out, float* p_out, int B, int T, int H, float kappa, void* ws,
-                     cudaStream_t s, int debug_skip_v, const int* cu_seqlens) {
+                     cudaStream_t s, int debug_skip_v, const int* cu_seqlens,
+                     int v_zero_rows = 0) {
   const int Bm = cu_seqlens ? 1 : B;  // batch extent of the tensor maps
   using P = WsPlan<DIAG>;
   CUtensorMap mq, mk, mv, mo, mw;
   if (!make_map(&mq, q, Bm, T, H, kDK, 64) || !make_map(&mk, k, Bm, T, H, kDK, 64) ||
-      !make_map(&mv, v, Bm, T, H, 128, 64))
+      !(v_zero_rows > 0 ? make_map(&mv, v, 1, v_zero_rows, H, 128, 64)
+                        : make_map(&mv, v, Bm, T, H, 128, 64)))
     return KDN_ERR_CUDA;
   // isotropic: the output tile map; diagonal: the output is written without a
   // map, and w [B, T, H, 128] is read in boxes of 16 tokens
@@ -2312,6 +2316,20 @@ kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const vo
   if (debug_skip_v >= 0 || cu_seqlens) return KDN_ERR_UNSUPPORTED;
   return diag ? launch<true, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s)
               : launch<false, 64>(q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv, kappa, ws, s);
+}
+
+// The d_v = 128 engine with V taken as zero: v_zero is a zeroed [1, 64, H,
+// 128] bf16 buffer (16-byte aligned).  Used for the state-transition runs of
+// the segmented long-sequence forward.
+kdn_status chunk_engine_launch_zero_v(bool diag, const void* q, const void* k, const void* v_zero,
+                                      const float* a, const float* w, const float* r,
+                                      const float* S0, const float* p0, float* o, float* S_out,
+                                      float* p_out, int B, int T, int H, float kappa, void* ws,
+                                      cudaStream_t s) {
+  return diag ? launch_ws<true>(q, k, v_zero, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa, ws,
+                                s, -1, nullptr, 64)
+              : launch_ws<false>(q, k, v_zero, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa,
+                                 ws, s, -1, nullptr, 64);
 }
 
 }  // namespace kdn

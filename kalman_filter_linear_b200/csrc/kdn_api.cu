@@ -26,6 +26,12 @@ kdn_status recurrent_launch(bool diag, kdn_dtype dt, const void* q, const void* 
                             float* Ssave = nullptr, float* Psave = nullptr);
 bool chunk_engine_supported(kdn_dtype dt, int dk, int dv);
 size_t chunk_engine_workspace_size(bool diag, int B, int H);
+int segment_count(int B, int T, int H);
+size_t segmented_workspace_size(bool diag, int B, int T, int H, int nseg);
+kdn_status segmented_forward(bool diag, const void* q, const void* k, const void* v,
+                             const float* a, const float* w, const float* r, const float* S0,
+                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
+                             int H, float kappa, int nseg, void* ws, cudaStream_t st);
 kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const void* v,
                                const float* a, const float* w, const float* r, const float* S0,
                                const float* p0, float* o, float* S_out, float* p_out, int B,
@@ -118,9 +124,16 @@ kdn_status forward_common(bool diag, const void* q, const void* k, const void* v
     return kdn::recurrent_launch(diag, in_dtype, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T,
                                  H, dk, dv, kappa, as_stream(stream), cu_seqlens, err);
   }
-  const size_t need = kdn::chunk_engine_workspace_size(diag, B, H);
+  // few heads over a long sequence: the segmented forward (whole segments as
+  // extra heads of the same engine)
+  const int nseg = (dv == 128 && !cu_seqlens && debug_skip_v < 0) ? kdn::segment_count(B, T, H) : 1;
+  const size_t need = nseg > 1 ? kdn::segmented_workspace_size(diag, B, T, H, nseg)
+                               : kdn::chunk_engine_workspace_size(diag, B, H);
   if (need && (!workspace || workspace_bytes < need)) return KDN_ERR_WORKSPACE;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDN_ERR_INVALID_ARG;
+  if (nseg > 1)
+    return kdn::segmented_forward(diag, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, kappa,
+                                  nseg, workspace, as_stream(stream));
   return kdn::chunk_engine_launch(diag, q, k, v, a, w, r, S0, p0, o, S_out, p_out, B, T, H, dv,
                                   kappa, workspace, as_stream(stream), debug_skip_v, cu_seqlens);
 }
@@ -211,11 +224,12 @@ kdn_status kdn_mobius_scan(const float* a, const float* w, const float* r, const
 
 size_t kdn_forward_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,
                                   int chunk) {
-  (void)T;
-  if (!dims_supported(dk, dv) || B < 1 || H < 1) return 0;
-  return select_path(chunk, KDN_BF16, dk, dv) == 1
-             ? kdn::chunk_engine_workspace_size(variant == KDN_DIAG, B, H)
-             : 0;
+  if (!dims_supported(dk, dv) || B < 1 || H < 1 || T < 0) return 0;
+  if (select_path(chunk, KDN_BF16, dk, dv) != 1) return 0;
+  const bool diag = variant == KDN_DIAG;
+  const int nseg = dv == 128 && T > 0 ? kdn::segment_count(B, T, H) : 1;
+  return nseg > 1 ? kdn::segmented_workspace_size(diag, B, T, H, nseg)
+                  : kdn::chunk_engine_workspace_size(diag, B, H);
 }
 
 kdn_status kdn_iso_forward(const void* q, const void* k, const void* v, kdn_dtype in_dtype,

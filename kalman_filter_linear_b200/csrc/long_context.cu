@@ -1,0 +1,368 @@
+// Segmented forward for long sequences over few heads.
+//
+// The chunked engine runs one CTA per (batch entry, head) and walks that
+// head's chunks in order, so a call with few heads and a long sequence (for
+// example B1 T65536 H16: 16 CTAs, 1024 chunks each) leaves most SMs idle.
+// The memory recursion is affine in the state ("Kalman Delta Networks:
+// Uncertainty-aware Associative Memory", abstract: a gain-weighted delta-rule
+// write per token): over a stretch of tokens whose variances are known,
+//     S_end = S_start F + E,
+// with F (d_k x d_k) the state transition of the stretch and E (d_v x d_k)
+// the state the stretch reaches from S_start = 0.  The variance recursion is
+// a Mobius map per token and composes by matrix products ("Kalman Linear
+// Attention ...", 方法论 §2; the same abstract), so the variance at the start
+// of each stretch follows from the composed maps of the stretches before it.
+//
+// The sequence is cut into S segments of L = T / S tokens, viewed as S extra
+// batch entries of the same [B, T, H, d] tensors ([B S, L, H, d] is the same
+// memory).  Then:
+//   1. every lane composes the Mobius maps of blocks of 1024 tokens in
+//      parallel, and one pass per lane applies the block products in order,
+//      recording the variance at each segment start;
+//   2. the engine runs all segments from S_start = 0 (giving E) and, with V
+//      read as zero, from S_start = I (giving F: with d_v = d_k the final
+//      state is I F);
+//   3. a pass per (batch entry, head, block of 16 state rows) chains the
+//      segments: S_start(s + 1) = S_start(s) F(s) + E(s);
+//   4. the engine runs all segments from their true S_start, writing o and
+//      each segment's final state, of which the last segment's is S_T.
+// Steps 2 and 4 have S times the heads of the call, at 1/S of its length.
+#include <algorithm>
+
+#include "kdn_common.cuh"
+
+namespace kdn {
+
+kdn_status chunk_engine_launch(bool diag, const void* q, const void* k, const void* v,
+                               const float* a, const float* w, const float* r, const float* S0,
+                               const float* p0, float* o, float* S_out, float* p_out, int B,
+                               int T, int H, int dv, float kappa, void* ws, cudaStream_t s,
+                               int debug_skip_v, const int* cu_seqlens);
+kdn_status chunk_engine_launch_zero_v(bool diag, const void* q, const void* k, const void* v_zero,
+                                      const float* a, const float* w, const float* r,
+                                      const float* S0, const float* p0, float* o, float* S_out,
+                                      float* p_out, int B, int T, int H, float kappa, void* ws,
+                                      cudaStream_t s);
+
+namespace {
+
+constexpr int kD = 128;          // d_k = d_v of the engine
+constexpr int kBlock = 1024;     // tokens per composed Mobius block
+constexpr int kMinSegments = 4;  // three engine passes over 1/S of the tokens each
+
+struct M2 {
+  float a, b, c, d;  // [[a, b], [c, d]]
+};
+// x * y (x the later map)
+__device__ __forceinline__ M2 mul(const M2& x, const M2& y) {
+  return {fmaf(x.a, y.a, x.b * y.c), fmaf(x.a, y.b, x.b * y.d), fmaf(x.c, y.a, x.d * y.c),
+          fmaf(x.c, y.b, x.d * y.d)};
+}
+// scale by a power of two that brings the largest entry to [1, 2): exact
+__device__ __forceinline__ M2 renorm(const M2& x) {
+  const float m = fmaxf(fmaxf(x.a, x.b), fmaxf(x.c, x.d));
+  const int e = (int)((__float_as_uint(m) >> 23) & 0xffu) - 127;
+  if (e > -120 && e < 120) {
+    const float sc = __uint_as_float((uint32_t)(127 - e) << 23);
+    return {x.a * sc, x.b * sc, x.c * sc, x.d * sc};
+  }
+  return x;
+}
+// the variance step p -> r (a^2 p + w) / (c (a^2 p + w) + r) as a matrix
+__device__ __forceinline__ M2 step_map(float a, float w, float r, float c) {
+  const float a2 = a * a;
+  return {r * a2, r * w, c * a2, fmaf(c, w, r)};
+}
+
+// Diagonal variant: lane (b, h, i), block j of kBlock tokens.  Threads of a
+// warp take consecutive i, so every token's w and k reads are coalesced.
+__global__ void __launch_bounds__(256)
+block_maps_diag_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ A,
+                       const float* __restrict__ W, const float* __restrict__ R, int B, int T,
+                       int H, int nblk, float4* __restrict__ prod) {
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t lanes = (int64_t)B * H * kD;
+  if (gid >= lanes * nblk) return;
+  const int j = (int)(gid / lanes);
+  const int64_t lane = gid % lanes;
+  const int i = (int)(lane % kD);
+  const int h = (int)((lane / kD) % H);
+  const int b = (int)(lane / ((int64_t)kD * H));
+  const int t0 = j * kBlock, t1 = min(T, t0 + kBlock);
+  M2 P = {1.f, 0.f, 0.f, 1.f};
+#pragma unroll 4
+  for (int t = t0; t < t1; ++t) {
+    const size_t tok = ((size_t)b * T + t) * H + h;
+    const float kv = __bfloat162float(K[tok * kD + i]);
+    P = mul(step_map(__ldg(A + tok), __ldg(W + tok * kD + i), __ldg(R + tok), kv * kv), P);
+    if ((t & 7) == 7) P = renorm(P);
+  }
+  P = renorm(P);
+  prod[lane * nblk + j] = make_float4(P.a, P.b, P.c, P.d);
+}
+
+// Isotropic variant: lane (b, h), block j; one warp per (lane, block), lane
+// l composing tokens [t0 + 32 l, t0 + 32 l + 32) (c = kappa ||k||^2), then
+// the 32 partial products combined in token order.
+__global__ void __launch_bounds__(256)
+block_maps_iso_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ A,
+                      const float* __restrict__ W, const float* __restrict__ R, int B, int T,
+                      int H, int nblk, float kappa, float4* __restrict__ prod) {
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int l = threadIdx.x & 31;
+  const int64_t lanes = (int64_t)B * H;
+  if (wid >= lanes * nblk) return;  // (whole warps leave together)
+  const int j = (int)(wid / lanes);
+  const int64_t lane = wid % lanes;
+  const int h = (int)(lane % H), b = (int)(lane / H);
+  const int t0 = j * kBlock + 32 * l, t1 = min(T, t0 + 32);
+  M2 P = {1.f, 0.f, 0.f, 1.f};
+  for (int t = t0; t < t1; ++t) {
+    const size_t tok = ((size_t)b * T + t) * H + h;
+    const uint4* kr = reinterpret_cast<const uint4*>(K + tok * kD);
+    float n = 0.f;
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {
+      const uint4 u = __ldg(kr + c);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(wv[e] << 16), x1 = __uint_as_float(wv[e] & 0xffff0000u);
+        n = fmaf(x0, x0, fmaf(x1, x1, n));
+      }
+    }
+    P = mul(step_map(__ldg(A + tok), __ldg(W + tok), __ldg(R + tok), kappa * n), P);
+    if ((t & 7) == 7) P = renorm(P);
+  }
+  P = renorm(P);
+  // ordered product over the warp: lane l's tokens come after lane l - 1's
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    M2 o;
+    o.a = __shfl_down_sync(0xffffffffu, P.a, d);
+    o.b = __shfl_down_sync(0xffffffffu, P.b, d);
+    o.c = __shfl_down_sync(0xffffffffu, P.c, d);
+    o.d = __shfl_down_sync(0xffffffffu, P.d, d);
+    // lane l holds the product of lanes [l, l + d); combine with [l + d, l + 2 d)
+    if ((l & (2 * d - 1)) == 0) P = renorm(mul(o, P));
+  }
+  if (l == 0) prod[lane * nblk + j] = make_float4(P.a, P.b, P.c, P.d);
+}
+
+// Per lane: apply the block products in order from p0, recording the variance
+// at the start of every segment (segments are bps blocks long) in the layout
+// of the segment view's p0: [(b S + s), H, dim].
+__global__ void __launch_bounds__(256)
+segment_starts_kernel(const float4* __restrict__ prod, const float* __restrict__ p0, int B,
+                      int H, int dim, int nseg, int bps, float* __restrict__ p_start) {
+  const int64_t lane = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t lanes = (int64_t)B * H * dim;
+  if (lane >= lanes) return;
+  const int64_t b = lane / ((int64_t)H * dim), hd = lane % ((int64_t)H * dim);
+  float p = p0 ? p0[lane] : 1.f;
+  const int nblk = nseg * bps;
+  for (int j = 0; j < nblk; ++j) {
+    if (j % bps == 0) p_start[((b * nseg) + j / bps) * H * dim + hd] = p;
+    const float4 m = prod[lane * nblk + j];
+    p = __fdividef(fmaf(m.x, p, m.y), fmaf(m.z, p, m.w));
+  }
+}
+
+// Identity states for the transition runs: [n][kD][kD].
+__global__ void identity_kernel(float* __restrict__ S, int64_t n) {
+  const int64_t total = n * kD * kD;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = i % (kD * kD);
+    S[i] = (e / kD == e % kD) ? 1.f : 0.f;
+  }
+}
+
+// Segment starts: S_start(0) = S0 (or 0), S_start(s + 1) = S_start(s) F(s) +
+// E(s).  One CTA per (batch entry, head, block of 16 rows of S); rows of S
+// do not mix, so the blocks are independent.  State layouts: [(b S + s), H,
+// kD, kD] for F, E and S_start; S0 [B, H, kD, kD].
+constexpr int kRows = 16;
+__global__ void __launch_bounds__(256)
+chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
+                      const float* __restrict__ E, int B, int H, int nseg,
+                      float* __restrict__ S_start) {
+  __shared__ float cur[kRows][kD];
+  const int rb = blockIdx.x % (kD / kRows);
+  const int h = (blockIdx.x / (kD / kRows)) % H;
+  const int b = blockIdx.x / ((kD / kRows) * H);
+  const int tid = threadIdx.x;
+  const int r = tid >> 4, c0 = (tid & 15) * 8;  // row r, columns c0 .. c0 + 7
+  const int row = rb * kRows + r;
+  const auto at = [&](int s) { return ((((size_t)b * nseg + s) * H + h) * kD) * kD; };
+  {
+    float* dst = S_start + at(0) + (size_t)row * kD + c0;
+    const float* src = S0 ? S0 + ((((size_t)b * H + h) * kD) + row) * kD + c0 : nullptr;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = src ? src[e] : 0.f;
+      cur[r][c0 + e] = x;
+      dst[e] = x;
+    }
+  }
+  __syncthreads();
+  for (int s = 0; s + 1 < nseg; ++s) {
+    const float* Fs = F + at(s);
+    const float* Es = E + at(s) + (size_t)row * kD + c0;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = Es[e];
+    for (int j = 0; j < kD; ++j) {
+      const float x = cur[r][j];
+      const float4 f0 = *reinterpret_cast<const float4*>(Fs + (size_t)j * kD + c0);
+      const float4 f1 = *reinterpret_cast<const float4*>(Fs + (size_t)j * kD + c0 + 4);
+      acc[0] = fmaf(x, f0.x, acc[0]);
+      acc[1] = fmaf(x, f0.y, acc[1]);
+      acc[2] = fmaf(x, f0.z, acc[2]);
+      acc[3] = fmaf(x, f0.w, acc[3]);
+      acc[4] = fmaf(x, f1.x, acc[4]);
+      acc[5] = fmaf(x, f1.y, acc[5]);
+      acc[6] = fmaf(x, f1.z, acc[6]);
+      acc[7] = fmaf(x, f1.w, acc[7]);
+    }
+    __syncthreads();  // every thread has read cur
+    float* dst = S_start + at(s + 1) + (size_t)row * kD + c0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      cur[r][c0 + e] = acc[e];
+      dst[e] = acc[e];
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void or_error_words(uint32_t* dst, const uint32_t* a, const uint32_t* b,
+                               const uint32_t* c) {
+  atomicOr(dst, *a | *b | *c);
+}
+
+inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct SegLayout {
+  size_t err_e, err_f, err_g, prod, p_start, p_scratch, ident, E, F, S_start, zero_v, total;
+};
+
+// Workspace: the call's error word (bytes 0-3, first 256-byte block), one
+// error word per engine pass, then the segment data.
+SegLayout seg_layout(bool diag, int B, int T, int H, int nseg) {
+  SegLayout L{};
+  size_t off = 256;
+  auto take = [&](size_t n) {
+    const size_t at = off;
+    off = up256(off + n);
+    return at;
+  };
+  const int dim = diag ? kD : 1;
+  const size_t states = (size_t)B * nseg * H * kD * kD * 4;
+  const size_t vars = (size_t)B * nseg * H * dim * 4;
+  L.err_e = take(256);
+  L.err_f = take(256);
+  L.err_g = take(256);
+  L.prod = take((size_t)B * H * dim * (T / kBlock) * 16);
+  L.p_start = take(vars);
+  L.p_scratch = take(vars);
+  L.ident = take(states);
+  L.E = take(states);
+  L.F = take(states);
+  L.S_start = take(states);
+  L.zero_v = take((size_t)64 * H * kD * 2);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+// Number of segments for a call of the d_v = 128 engine on the current
+// device: the largest power of two S >= 4 with B H S CTAs fitting on the SMs
+// at once and T a multiple of 1024 S (whole composed blocks per segment),
+// or 1 (no segmentation).
+int segment_count(int B, int T, int H) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 1;
+  const int64_t heads = (int64_t)B * H;
+  int S = 1;
+  while ((int64_t)heads * S * 2 <= sms && T % (kBlock * S * 2) == 0) S *= 2;
+  return S >= kMinSegments ? S : 1;
+}
+
+size_t segmented_workspace_size(bool diag, int B, int T, int H, int nseg) {
+  return seg_layout(diag, B, T, H, nseg).total;
+}
+
+kdn_status segmented_forward(bool diag, const void* q, const void* k, const void* v,
+                             const float* a, const float* w, const float* r, const float* S0,
+                             const float* p0, float* o, float* S_out, float* p_out, int B, int T,
+                             int H, float kappa, int nseg, void* ws, cudaStream_t st) {
+  const SegLayout L = seg_layout(diag, B, T, H, nseg);
+  char* base = static_cast<char*>(ws);
+  const int dim = diag ? kD : 1;
+  const int Bs = B * nseg, Ls = T / nseg;
+  const int nblk = T / kBlock, bps = nblk / nseg;
+  float4* prod = reinterpret_cast<float4*>(base + L.prod);
+  float* p_start = reinterpret_cast<float*>(base + L.p_start);
+  float* p_scratch = reinterpret_cast<float*>(base + L.p_scratch);
+  float* ident = reinterpret_cast<float*>(base + L.ident);
+  float* E = reinterpret_cast<float*>(base + L.E);
+  float* F = reinterpret_cast<float*>(base + L.F);
+  float* S_start = reinterpret_cast<float*>(base + L.S_start);
+  if (cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return KDN_ERR_CUDA;
+  if (cudaMemsetAsync(base + L.zero_v, 0, (size_t)64 * H * kD * 2, st) != cudaSuccess)
+    return KDN_ERR_CUDA;
+
+  // 1. variances at the segment starts
+  const int64_t lanes = (int64_t)B * H * dim;
+  if (diag) {
+    const int64_t n = lanes * nblk;
+    block_maps_diag_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), a, w, r, B, T, H, nblk, prod);
+  } else {
+    const int64_t nthr = lanes * nblk * 32;
+    block_maps_iso_kernel<<<(unsigned)((nthr + 255) / 256), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(k), a, w, r, B, T, H, nblk, kappa, prod);
+  }
+  segment_starts_kernel<<<(unsigned)((lanes + 255) / 256), 256, 0, st>>>(prod, p0, B, H, dim,
+                                                                         nseg, bps, p_start);
+  identity_kernel<<<592, 256, 0, st>>>(ident, (int64_t)Bs * H);
+  if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
+
+  // 2. every segment from S_start = 0 (E), and with V read as zero from
+  // S_start = I (F).  Their outputs land in o; pass 4 overwrites them.
+  kdn_status stt = chunk_engine_launch(diag, q, k, v, a, w, r, nullptr, p_start, o, E, p_scratch,
+                                       Bs, Ls, H, kD, kappa, base + L.err_e, st, -1, nullptr);
+  if (stt != KDN_OK) return stt;
+  stt = chunk_engine_launch_zero_v(diag, q, k, base + L.zero_v, a, w, r, ident, p_start, o, F,
+                                   p_scratch, Bs, Ls, H, kappa, base + L.err_f, st);
+  if (stt != KDN_OK) return stt;
+
+  // 3. the true state at every segment start
+  chain_segments_kernel<<<(unsigned)(B * H * (kD / kRows)), 256, 0, st>>>(S0, F, E, B, H, nseg,
+                                                                          S_start);
+  if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
+
+  // 4. every segment from its true start: o, and each segment's final state
+  // and variance (into E and p_scratch), of which the last segment's are the
+  // call's
+  stt = chunk_engine_launch(diag, q, k, v, a, w, r, S_start, p_start, o, E, p_scratch, Bs, Ls, H,
+                            kD, kappa, base + L.err_g, st, -1, nullptr);
+  if (stt != KDN_OK) return stt;
+  const size_t sbytes = (size_t)H * kD * kD * 4, pbytes = (size_t)H * dim * 4;
+  if (cudaMemcpy2DAsync(S_out, sbytes, E + (size_t)(nseg - 1) * H * kD * kD, sbytes * nseg,
+                        sbytes, B, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+      cudaMemcpy2DAsync(p_out, pbytes, p_scratch + (size_t)(nseg - 1) * H * dim, pbytes * nseg,
+                        pbytes, B, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return KDN_ERR_CUDA;
+  or_error_words<<<1, 1, 0, st>>>(static_cast<uint32_t*>(ws),
+                                  reinterpret_cast<const uint32_t*>(base + L.err_e),
+                                  reinterpret_cast<const uint32_t*>(base + L.err_f),
+                                  reinterpret_cast<const uint32_t*>(base + L.err_g));
+  return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
+}
+
+}  // namespace kdn

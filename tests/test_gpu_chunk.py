@@ -189,3 +189,39 @@ def test_engine_extreme_coefficients(variant, T, dv):
     assert eo <= OUT_TOL, eo
     assert eS <= STATE_TOL, eS
     np.testing.assert_allclose(f64(p), p_r, rtol=1e-5)
+
+
+@pytest.mark.parametrize("variant", ["iso", "diag"])
+@pytest.mark.parametrize("extreme", [False, True])
+def test_segmented_long_sequence_matches_oracle(variant, extreme):
+    """Few heads over a long sequence (B1 H2 T8192) take the segmented
+    forward: eight segments of 1024 tokens run as extra heads, from the
+    variances their composed Mobius maps give and the states the chained
+    segment transitions give.  Against the oracle over the whole sequence,
+    with a non-zero initial state and variance."""
+    B, T, H, d = 1, 8192, 2, 128
+    gen = synth.layer_inputs_extreme if extreme else synth.layer_inputs
+    x = to_dev(gen(B, T, H, d, d, variant, seed=81 + extreme, dtype='bf16'))
+    g = torch.Generator().manual_seed(82)
+    S0 = (0.05 * torch.randn(B, H, d, d, generator=g)).cuda()
+    p0 = (torch.rand((B, H) if variant == 'iso' else (B, H, d), generator=g) + 0.2).cuda()
+    var = kdn.KDN_ISO if variant == 'iso' else kdn.KDN_DIAG
+    ws = torch.empty(kdn.kdn_forward_workspace_size(var, B, T, H, d, d), dtype=torch.uint8,
+                     device='cuda')
+    # the segmented forward needs more than the engine's own 256-byte workspace
+    assert ws.numel() > kdn.kdn_forward_workspace_size(var, B, 300, H, d, d)
+    o, S, p = _run(variant, x, S0, p0, chunk=kdn.KDN_CHUNK_AUTO, workspace=ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_OK
+    o_r, S_r, p_r = _ref(variant, x, S0, p0)
+    eo, eS = rel_maxabs(o, o_r), rel_maxabs(S, S_r)
+    assert eo <= OUT_TOL, eo
+    assert eS <= STATE_TOL, eS
+    np.testing.assert_allclose(f64(p), p_r, rtol=1e-5)
+    # the same call split at the middle with the state handed over agrees
+    h = T // 2
+    xa = {k: v[:, :h].contiguous() for k, v in x.items()}
+    xb = {k: v[:, h:].contiguous() for k, v in x.items()}
+    _, Sa, pa = _run(variant, xa, S0, p0, chunk=kdn.KDN_CHUNK_AUTO)
+    ob, Sb, pb = _run(variant, xb, Sa, pa, chunk=kdn.KDN_CHUNK_AUTO)
+    assert rel_maxabs(ob, o_r[:, h:]) <= OUT_TOL
+    assert rel_maxabs(Sb, S_r) <= STATE_TOL

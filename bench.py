@@ -361,7 +361,7 @@ def main():
     ap.add_argument('--no-secondary', action='store_true')
     ap.add_argument('--no-cpu-baseline', action='store_true')
     ap.add_argument('--only', choices=['iso', 'diag', 'scan', 'decode', 'varlen', 'exact', 'kla',
-                                       'bwd'],
+                                       'bwd', 'bwd128'],
                     help='run only this kernel (for profiler captures) and print its timing')
     ap.add_argument('--B', type=int, default=None, help='batch override for --only')
     ap.add_argument('--T', type=int, default=None, help='length override for --only')
@@ -530,6 +530,8 @@ def run_only(args):
         f = lambda: kdn.kdn_backward('iso', x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,
                                      workspace=wsb)
         units, alg = B * T, backward_bytes(B, T, H, d)
+    elif args.only == 'bwd128':
+        f, units, alg, _ = backward128_case(kdn, synth, dev, args.B, args.T)
     elif args.only == 'kla':
         c = synth.WORKLOADS['diag_1p3b']
         B, T, H, d = args.B or c['B'], args.T or c['T'], c['H'], c['dk']
@@ -578,13 +580,35 @@ def varlen_case(kdn, synth, dev):
     return f, total, alg, desc
 
 
-def backward_bytes(B, T, H, d, in_bytes=2):
-    """Algorithmic HBM bytes of one backward call (isotropic, d_k = d_v = d):
-    inputs read twice (the forward again, then the backward), dO read, the
-    forward's o written, the saved states and variances written and read
-    once, the gradients of q, k, v, a, w, r written."""
-    return (2 * B * T * H * (3 * d * in_bytes + 12) + 2 * B * T * H * d * 4 +
-            2 * B * H * T * (d * d + 1) * 4 + B * T * H * (3 * d + 3) * 4)
+def backward_bytes(B, T, H, d, variant='iso', in_bytes=2, ck=16):
+    """Algorithmic HBM bytes of one backward call at d_k = d_v = d: inputs
+    read twice (the forward again, then the backward), dO read, the forward's
+    o written, the state checkpoints (every ck-th token) and the variance of
+    every token written and read once, the gradients written.  The rebuilt
+    states of each 16-token block stay in a per-CTA scratch that L2 holds."""
+    dim = d if variant == 'diag' else 1
+    inp = B * T * H * (3 * d * in_bytes + (2 + dim) * 4)
+    ck_states = B * H * (-(-T // ck)) * d * d * 4
+    grads = B * T * H * (3 * d + 2 + dim) * 4
+    return (2 * inp + 2 * B * T * H * d * 4 + 2 * ck_states + 2 * B * H * T * dim * 4 + grads)
+
+
+def backward128_case(kdn, synth, dev, B=None, T=None, variant='iso'):
+    """The backward pass at the 1.3B-layer shape (d_k = d_v = 128): (launch
+    fn, tokens, algorithmic bytes, description)."""
+    import torch
+    c = synth.WORKLOADS['iso_1p3b' if variant == 'iso' else 'diag_1p3b']
+    B, T, H, d = B or c['B'], T or c['T'], c['H'], c['dk']
+    x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, variant, c['seed'],
+                                                     c['dtype']).items()}
+    dO = torch.randn((B, T, H, d), generator=torch.Generator().manual_seed(c['seed'] + 100)).to(dev)
+    var = kdn.KDN_ISO if variant == 'iso' else kdn.KDN_DIAG
+    wsb = torch.empty(kdn.kdn_backward_workspace_size(var, B, T, H, d, d), dtype=torch.uint8,
+                      device=dev)
+    f = lambda: kdn.kdn_backward(variant, x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], dO,
+                                 workspace=wsb)
+    return f, B * T, backward_bytes(B, T, H, d, variant), {'B': B, 'T': T, 'H': H, 'd': d,
+                                                             'variant': variant}
 
 
 def exact_bytes(B, T, H, dk, dv, in_bytes=2):
@@ -731,6 +755,15 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
                            'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                            'algorithmic_bytes': alg, 'B': B, 'T': T, 'H': H, 'd': d}
     del x, dO, wsb
+    # backward pass at the 1.3B-layer shape, B8 T4096 H16 d128, isotropic
+    f, units, alg, desc = backward128_case(kdn, synth, dev)
+    n = 2
+    ms = time_launches(f, n, 2, stream) / n
+    out['backward_d128'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
+                            'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
+                            'algorithmic_bytes': alg, **desc}
+    del f
+    torch.cuda.empty_cache()
     # dense (full-covariance) filter, B8 T4096 H16 d64
     f, units, alg, desc = exact_case(kdn, synth, dev)
     n = 3

@@ -60,7 +60,7 @@ def is_stale():
         return True
     t = os.path.getmtime(LIB)
     deps = sources() + glob.glob(os.path.join(PKG, 'csrc', '*.cuh')) + \
-        glob.glob(os.path.join(ROOT, 'include', '*.h'))
+        glob.glob(os.path.join(PKG, 'csrc', '*.h')) + glob.glob(os.path.join(ROOT, 'include', '*.h'))
     return any(os.path.getmtime(d) > t for d in deps)
 
 

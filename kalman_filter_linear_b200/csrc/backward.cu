@@ -13,41 +13,59 @@
 // then the terms of the gain g and of the variance recursion p, which give
 // dk, da, dw, dr and carry dp to the token before (dp <- a^2 dp-).
 //
-// Layout as the recurrent forward kernel: one CTA of 8 warps per (b, h);
-// warp w holds rows w, w + 8, ... of S and dS, lane l holds columns
-// [l CPL, (l + 1) CPL).  Row sums (S k, dS g) are butterfly reductions inside
-// a warp; the column sums over all rows (S'^T do, dS^T e, S^T de) and the
-// scalar <dS, S> meet in shared memory, one block barrier per token.  The
-// gain and variance terms are per column and are computed by every warp
-// identically, so no further exchange is needed.
+// Layout as the recurrent forward kernel: one CTA per (b, h) of NW warps
+// (8, or 16 at d_k = 128 so that S and dS of a warp's rows fit in its
+// registers); warp w holds rows w, w + NW, ... of S and dS, lane l holds
+// columns [l CPL, (l + 1) CPL).  Row sums (S k, dS g) are butterfly
+// reductions inside a warp; the column sums over all rows (S'^T do, dS^T e,
+// S^T de) and the scalar <dS, S> meet in shared memory, one block barrier per
+// token.  The gain and variance terms are per column and are computed by
+// every warp identically, so no further exchange is needed.
+//
+// States: the forward keeps S only before every 16th token (a checkpoint)
+// and p before every token.  The backward walks blocks of 16 tokens from
+// the last to the first; for each it rebuilds the block's states from its
+// checkpoint with the forward's own arithmetic into a per-CTA scratch of 16
+// states (small enough to stay in L2 for all CTAs of a launch), then runs
+// the adjoint over them.  Each thread reads back only what it wrote itself.
 #include "kdn_common.cuh"
+#include "bwd_checkpoint.h"
 
 namespace kdn {
 namespace {
 
-constexpr int kBW = 8, kBRows = 16;  // warps; rows of S per warp (d_v <= 128)
+template <int CPL>
+struct BwdShape {
+  static constexpr int NW = CPL == 4 ? 16 : 8;  // warps
+  static constexpr int NR = 128 / NW;            // rows of S per warp (d_v <= 128)
+  static constexpr int DK = CPL * 32;
+  static constexpr int RED = 3 * DK + 1;
+  static constexpr size_t SMEM = 2u * NW * RED * sizeof(float);
+};
 
 template <bool DIAG, int CPL, typename InT>
-__global__ void __launch_bounds__(kBW * 32)
+__global__ void __launch_bounds__(BwdShape<CPL>::NW * 32)
 kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
                const InT* __restrict__ V, const float* __restrict__ A,
                const float* __restrict__ Wn, const float* __restrict__ R,
                const float* __restrict__ dO, const float* __restrict__ dS_T,
-               const float* __restrict__ dp_T, const float* __restrict__ Ssave,
-               const float* __restrict__ Psave, float* __restrict__ dQ, float* __restrict__ dK,
-               float* __restrict__ dV, float* __restrict__ dA, float* __restrict__ dW,
-               float* __restrict__ dR, float* __restrict__ dS0, float* __restrict__ dP0, int T,
-               int H, int dv, float kappa) {
-  constexpr int DK = CPL * 32, NP = DIAG ? CPL : 1, RED = 3 * DK + 1;
-  __shared__ float red[2][kBW][RED];
+               const float* __restrict__ dp_T, const float* __restrict__ Sck,
+               const float* __restrict__ Psave, float* __restrict__ scratch,
+               float* __restrict__ dQ, float* __restrict__ dK, float* __restrict__ dV,
+               float* __restrict__ dA, float* __restrict__ dW, float* __restrict__ dR,
+               float* __restrict__ dS0, float* __restrict__ dP0, int T, int H, int dv,
+               float kappa) {
+  using X = BwdShape<CPL>;
+  constexpr int NW = X::NW, NR = X::NR, DK = X::DK, RED = X::RED, NP = DIAG ? CPL : 1;
+  extern __shared__ float red_dyn[];  // [2][NW][RED]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int bh = blockIdx.x, b = bh / H, h = bh % H;
 
-  float dS[kBRows][CPL], dp[NP];
+  float dS[NR][CPL], dp[NP];
   const size_t s_base = (size_t)bh * dv * DK;
 #pragma unroll
-  for (int i = 0; i < kBRows; ++i) {
-    const int j = warp + kBW * i;
+  for (int i = 0; i < NR; ++i) {
+    const int j = warp + NW * i;
 #pragma unroll
     for (int c = 0; c < CPL; ++c)
       dS[i][c] = (dS_T && j < dv) ? dS_T[s_base + (size_t)j * DK + lane * CPL + c] : 0.f;
@@ -56,10 +74,86 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
   for (int c = 0; c < NP; ++c)
     dp[c] = dp_T ? dp_T[DIAG ? (size_t)bh * DK + lane * CPL + c : (size_t)bh] : 0.f;
 
-  for (int t = T - 1; t >= 0; --t) {
+  const int nck = (T + kBwdCheckpoint - 1) / kBwdCheckpoint;
+  float* scr = scratch + (size_t)bh * kBwdCheckpoint * dv * DK;
+  for (int blk = nck - 1; blk >= 0; --blk) {
+    const int t0 = blk * kBwdCheckpoint, t1 = min(T, t0 + kBwdCheckpoint);
+    // ---- the block's states, rebuilt from its checkpoint (the forward's
+    // arithmetic, token by token) into the scratch
+    {
+      float S[NR][CPL];
+      const float* ck = Sck + ((size_t)bh * nck + blk) * dv * DK;
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const int j = warp + NW * i;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) S[i][c] = j < dv ? ck[(size_t)j * DK + lane * CPL + c] : 0.f;
+      }
+      for (int t = t0; t < t1; ++t) {
+        float* dst = scr + (size_t)(t - t0) * dv * DK;
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const int j = warp + NW * i;
+          if (j < dv) {
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) dst[(size_t)j * DK + lane * CPL + c] = S[i][c];
+          }
+        }
+        if (t + 1 == t1) break;
+        const size_t tok = ((size_t)b * T + t) * H + h;
+        const size_t sv = ((size_t)bh * T + t);
+        float k[CPL], g[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) k[c] = to_f32(K[tok * DK + lane * CPL + c]);
+        const float a = A[tok], r = R[tok];
+        if constexpr (DIAG) {
+          float pp[CPL], part = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            pp[c] = fmaf(a * a, Psave[sv * DK + lane * CPL + c], Wn[tok * DK + lane * CPL + c]);
+            part = fmaf(pp[c] * k[c], k[c], part);
+          }
+          const float inv_s = 1.f / (warp_sum(part) + r);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) g[c] = pp[c] * k[c] * inv_s;
+        } else {
+          float part = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) part = fmaf(k[c], k[c], part);
+          const float n = warp_sum(part);
+          const float pp = fmaf(a * a, Psave[sv], Wn[tok]);
+          const float beta = pp / fmaf(pp, n, r);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) g[c] = beta * k[c];
+        }
+        float sk[NR];
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          float x = 0.f;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) x = fmaf(S[i][c], k[c], x);
+          sk[i] = x;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int i = 0; i < NR; ++i) sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const int j = warp + NW * i;
+          const float e = (j < dv ? to_f32(V[tok * dv + j]) : 0.f) - a * sk[i];
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) S[i][c] = fmaf(e, g[c], a * S[i][c]);
+        }
+      }
+    }
+
+    // ---- the adjoint over the block, last token first
+    for (int t = t1 - 1; t >= t0; --t) {
     const size_t tok = ((size_t)b * T + t) * H + h;
     const size_t sv = ((size_t)bh * T + t);
-    float k[CPL], q[CPL], S[kBRows][CPL], p[NP], wv[NP];
+    const float* Ssrc = scr + (size_t)(t - t0) * dv * DK;
+    float k[CPL], q[CPL], S[NR][CPL], p[NP], wv[NP];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
       k[c] = to_f32(K[tok * DK + lane * CPL + c]);
@@ -71,17 +165,16 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       p[c] = Psave[DIAG ? sv * DK + lane * CPL + c : sv];
       wv[c] = Wn[DIAG ? tok * DK + lane * CPL + c : tok];
     }
-    float vi[kBRows], doi[kBRows];
+    float vi[NR], doi[NR];
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) {
-      const int j = warp + kBW * i;
+    for (int i = 0; i < NR; ++i) {
+      const int j = warp + NW * i;
       vi[i] = j < dv ? to_f32(V[tok * dv + j]) : 0.f;
       doi[i] = j < dv ? dO[tok * dv + j] : 0.f;
 #pragma unroll
       for (int c = 0; c < CPL; ++c)
-        S[i][c] = j < dv ? Ssave[sv * dv * DK + (size_t)j * DK + lane * CPL + c] : 0.f;
+        S[i][c] = j < dv ? Ssrc[(size_t)j * DK + lane * CPL + c] : 0.f;
     }
-
     // the token's gain, recomputed from the saved variance
     float g[CPL], pm[NP], pn[NP], n = 0.f, den = 0.f, beta = 0.f, s = 0.f;
     if constexpr (DIAG) {
@@ -109,9 +202,9 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
     }
 
     // S k per row (all lanes end with the sums), e = v - a S k
-    float sk[kBRows], e[kBRows];
+    float sk[NR], e[NR];
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) {
+    for (int i = 0; i < NR; ++i) {
       float x = 0.f;
 #pragma unroll
       for (int c = 0; c < CPL; ++c) x = fmaf(S[i][c], k[c], x);
@@ -120,14 +213,14 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int i = 0; i < kBRows; ++i) sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+      for (int i = 0; i < NR; ++i) sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) e[i] = vi[i] - a * sk[i];
+    for (int i = 0; i < NR; ++i) e[i] = vi[i] - a * sk[i];
 
     // dS += do q^T, then de = dS g per row
-    float de[kBRows];
+    float de[NR];
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) {
+    for (int i = 0; i < NR; ++i) {
       float x = 0.f;
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
@@ -139,7 +232,7 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int i = 0; i < kBRows; ++i) de[i] += __shfl_xor_sync(0xffffffffu, de[i], o);
+      for (int i = 0; i < NR; ++i) de[i] += __shfl_xor_sync(0xffffffffu, de[i], o);
 
     // column sums over this warp's rows: S'^T do, dS^T e, S^T de; and <dS, S>
     float cq[CPL], cg[CPL], cs[CPL], dss = 0.f;
@@ -150,7 +243,7 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       cs[c] = 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) {
+    for (int i = 0; i < NR; ++i) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
         const float snew = fmaf(e[i], g[c], a * S[i][c]);
@@ -163,8 +256,8 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
     dss = warp_sum(dss);
     float dek = 0.f;  // <de, S k> over this warp's rows (the same in every lane)
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i) dek = fmaf(de[i], sk[i], dek);
-    float* rd = &red[t & 1][warp][0];
+    for (int i = 0; i < NR; ++i) dek = fmaf(de[i], sk[i], dek);
+    float* rd = red_dyn + ((size_t)(t & 1) * NW + warp) * RED;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
       rd[lane * CPL + c] = cq[c];
@@ -181,14 +274,14 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
       sde[c] = 0.f;
     }
 #pragma unroll
-    for (int w = 0; w < kBW; ++w) {
+    for (int w = 0; w < NW; ++w) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        dq[c] += red[t & 1][w][lane * CPL + c];
-        dg[c] += red[t & 1][w][DK + lane * CPL + c];
-        sde[c] += red[t & 1][w][2 * DK + lane * CPL + c];
+        dq[c] += red_dyn[((size_t)(t & 1) * NW + w) * RED + lane * CPL + c];
+        dg[c] += red_dyn[((size_t)(t & 1) * NW + w) * RED + DK + lane * CPL + c];
+        sde[c] += red_dyn[((size_t)(t & 1) * NW + w) * RED + 2 * DK + lane * CPL + c];
       }
-      da += red[t & 1][w][3 * DK];
+      da += red_dyn[((size_t)(t & 1) * NW + w) * RED + 3 * DK];
     }
 
     // the gain and variance terms
@@ -256,24 +349,25 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
         if constexpr (!DIAG) dW[tok] = dw[0];
       }
     }
-    if (lane < kBRows) {
+    if (lane < NR) {
       // lane i writes row warp + 8 i (every lane holds every de after the butterfly)
       float mine = 0.f;
 #pragma unroll
-      for (int i = 0; i < kBRows; ++i) mine = lane == i ? de[i] : mine;
-      const int j = warp + kBW * lane;
+      for (int i = 0; i < NR; ++i) mine = lane == i ? de[i] : mine;
+      const int j = warp + NW * lane;
       if (j < dv) dV[tok * dv + j] = mine;
     }
     // dS before the token: a (dS - de k^T)
 #pragma unroll
-    for (int i = 0; i < kBRows; ++i)
+    for (int i = 0; i < NR; ++i)
 #pragma unroll
       for (int c = 0; c < CPL; ++c) dS[i][c] = a * fmaf(-de[i], k[c], dS[i][c]);
+    }
   }
 
 #pragma unroll
-  for (int i = 0; i < kBRows; ++i) {
-    const int j = warp + kBW * i;
+  for (int i = 0; i < NR; ++i) {
+    const int j = warp + NW * i;
     if (j < dv) {
 #pragma unroll
       for (int c = 0; c < CPL; ++c) dS0[s_base + (size_t)j * DK + lane * CPL + c] = dS[i][c];
@@ -292,46 +386,60 @@ kdn_bwd_kernel(const InT* __restrict__ Q, const InT* __restrict__ K,
 template <bool DIAG, int CPL, typename InT>
 kdn_status launch_b(const void* q, const void* k, const void* v, const float* a, const float* w,
                     const float* r, const float* dO, const float* dS_T, const float* dp_T,
-                    const float* Ssave, const float* Psave, float* dq, float* dk, float* dv_,
-                    float* da, float* dw, float* dr, float* dS0, float* dp0, int B, int T, int H,
-                    int dv, float kappa, cudaStream_t s) {
-  kdn_bwd_kernel<DIAG, CPL, InT><<<B * H, kBW * 32, 0, s>>>(
+                    const float* Sck, const float* Psave, float* scratch, float* dq, float* dk,
+                    float* dv_, float* da, float* dw, float* dr, float* dS0, float* dp0, int B,
+                    int T, int H, int dv, float kappa, cudaStream_t s) {
+  using X = BwdShape<CPL>;
+  auto kern = kdn_bwd_kernel<DIAG, CPL, InT>;
+  if (X::SMEM > 48u * 1024u &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)X::SMEM) !=
+          cudaSuccess)
+    return KDN_ERR_CUDA;
+  kern<<<B * H, X::NW * 32, X::SMEM, s>>>(
       static_cast<const InT*>(q), static_cast<const InT*>(k), static_cast<const InT*>(v), a, w, r,
-      dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da, dw, dr, dS0, dp0, T, H, dv, kappa);
+      dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk, dv_, da, dw, dr, dS0, dp0, T, H, dv, kappa);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 
 template <bool DIAG, typename InT>
 kdn_status launch_bdk(const void* q, const void* k, const void* v, const float* a,
                       const float* w, const float* r, const float* dO, const float* dS_T,
-                      const float* dp_T, const float* Ssave, const float* Psave, float* dq,
-                      float* dk, float* dv_, float* da, float* dw, float* dr, float* dS0,
-                      float* dp0, int B, int T, int H, int dkk, int dv, float kappa,
+                      const float* dp_T, const float* Sck, const float* Psave, float* scratch,
+                      float* dq, float* dk, float* dv_, float* da, float* dw, float* dr,
+                      float* dS0, float* dp0, int B, int T, int H, int dkk, int dv, float kappa,
                       cudaStream_t s) {
-  if (dkk == 32)
-    return launch_b<DIAG, 1, InT>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_,
-                                  da, dw, dr, dS0, dp0, B, T, H, dv, kappa, s);
-  return launch_b<DIAG, 2, InT>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da,
-                                dw, dr, dS0, dp0, B, T, H, dv, kappa, s);
+  switch (dkk) {
+    case 32:
+      return launch_b<DIAG, 1, InT>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk,
+                                    dv_, da, dw, dr, dS0, dp0, B, T, H, dv, kappa, s);
+    case 64:
+      return launch_b<DIAG, 2, InT>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk,
+                                    dv_, da, dw, dr, dS0, dp0, B, T, H, dv, kappa, s);
+    default:
+      return launch_b<DIAG, 4, InT>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk,
+                                    dv_, da, dw, dr, dS0, dp0, B, T, H, dv, kappa, s);
+  }
 }
 
 }  // namespace
 
-bool backward_supported(int dk, int dv) { return (dk == 32 || dk == 64) && dv >= 1 && dv <= 128; }
+bool backward_supported(int dk, int dv) {
+  return (dk == 32 || dk == 64 || dk == 128) && dv >= 1 && dv <= 128;
+}
 
 kdn_status backward_launch(bool diag, kdn_dtype dt, const void* q, const void* k, const void* v,
                            const float* a, const float* w, const float* r, const float* dO,
-                           const float* dS_T, const float* dp_T, const float* Ssave,
-                           const float* Psave, float* dq, float* dk, float* dv_, float* da,
-                           float* dw, float* dr, float* dS0, float* dp0, int B, int T, int H,
-                           int dkk, int dv, float kappa, cudaStream_t s) {
+                           const float* dS_T, const float* dp_T, const float* Sck,
+                           const float* Psave, float* scratch, float* dq, float* dk, float* dv_,
+                           float* da, float* dw, float* dr, float* dS0, float* dp0, int B, int T,
+                           int H, int dkk, int dv, float kappa, cudaStream_t s) {
   if (diag)
     return dt == KDN_BF16
-               ? launch_bdk<true, __nv_bfloat16>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s)
-               : launch_bdk<true, float>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s);
+               ? launch_bdk<true, __nv_bfloat16>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s)
+               : launch_bdk<true, float>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s);
   return dt == KDN_BF16
-             ? launch_bdk<false, __nv_bfloat16>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s)
-             : launch_bdk<false, float>(q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s);
+             ? launch_bdk<false, __nv_bfloat16>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s)
+             : launch_bdk<false, float>(q, k, v, a, w, r, dO, dS_T, dp_T, Sck, Psave, scratch, dq, dk, dv_, da, dw, dr, dS0, dp0, B, T, H, dkk, dv, kappa, s);
 }
 
 }  // namespace kdn

@@ -10,6 +10,7 @@
 
 #include "kdn_common.cuh"
 #include "../../include/kdn_testing.h"
+#include "bwd_checkpoint.h"
 
 namespace kdn {
 size_t mobius_scan_workspace_size(int64_t N, int64_t T);
@@ -46,10 +47,10 @@ kdn_status exact_kalman_launch(bool diag, kdn_dtype dt, const void* q, const voi
 bool backward_supported(int dk, int dv);
 kdn_status backward_launch(bool diag, kdn_dtype dt, const void* q, const void* k, const void* v,
                            const float* a, const float* w, const float* r, const float* dO,
-                           const float* dS_T, const float* dp_T, const float* Ssave,
-                           const float* Psave, float* dq, float* dk, float* dv_, float* da,
-                           float* dw, float* dr, float* dS0, float* dp0, int B, int T, int H,
-                           int dkk, int dv, float kappa, cudaStream_t s);
+                           const float* dS_T, const float* dp_T, const float* Sck,
+                           const float* Psave, float* scratch, float* dq, float* dk, float* dv_,
+                           float* da, float* dw, float* dr, float* dS0, float* dp0, int B, int T,
+                           int H, int dkk, int dv, float kappa, cudaStream_t s);
 bool kla_supported(int dk, int dv);
 kdn_status kla_launch(kdn_dtype dt, const void* q, const void* k, const void* v, const float* a,
                       const float* w, const float* r, const float* S0, const float* L0, float* o,
@@ -305,18 +306,21 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k, 
 }
 
 namespace {
-// backward workspace: saved states, saved variances, then the forward's
-// outputs (o, S_T, p_T), each region 256-byte aligned
+// backward workspace: the state checkpoints (every 16th token), the
+// variance before every token, the per-CTA scratch of 16 rebuilt states,
+// then the forward's outputs (o, S_T, p_T), each region 256-byte aligned
 struct BwdLayout {
-  size_t states, vars, o, s, p, bytes;
+  size_t states, vars, scratch, o, s, p, bytes;
 };
 inline size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 BwdLayout bwd_layout(bool diag, int B, int T, int H, int dk, int dv) {
   BwdLayout L{};
   const size_t bh = (size_t)B * H, np = diag ? (size_t)dk : 1;
+  const size_t nck = ((size_t)T + kdn::kBwdCheckpoint - 1) / kdn::kBwdCheckpoint;
   L.states = 0;
-  L.vars = al256(bh * T * dv * dk * 4);
-  L.o = L.vars + al256(bh * T * np * 4);
+  L.vars = al256(bh * nck * dv * dk * 4);
+  L.scratch = L.vars + al256(bh * T * np * 4);
+  L.o = L.scratch + al256(bh * kdn::kBwdCheckpoint * dv * dk * 4);
   L.s = L.o + al256((size_t)B * T * H * dv * 4);
   L.p = L.s + al256(bh * dv * dk * 4);
   L.bytes = L.p + al256(bh * np * 4);
@@ -356,18 +360,19 @@ kdn_status kdn_backward(kdn_variant variant, const void* q, const void* k, const
   if (!workspace || workspace_bytes < L.bytes) return KDN_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDN_ERR_INVALID_ARG;
   char* ws = static_cast<char*>(workspace);
-  float* Ssave = reinterpret_cast<float*>(ws + L.states);
+  float* Ssave = reinterpret_cast<float*>(ws + L.states);  // checkpoints
   float* Psave = reinterpret_cast<float*>(ws + L.vars);
   const float kappa = diag ? 1.f : (info_scale > 0.f ? info_scale : 1.f / (float)dk);
-  // the forward again, saving the state before every token
+  // the forward again, saving the variance before every token and the state
+  // before every 16th
   kdn_status st = kdn::recurrent_launch(
       diag, in_dtype, q, k, v, a, w, r, S0, p0, reinterpret_cast<float*>(ws + L.o),
       reinterpret_cast<float*>(ws + L.s), reinterpret_cast<float*>(ws + L.p), B, T, H, dk, dv,
       kappa, as_stream(stream), nullptr, nullptr, Ssave, Psave);
   if (st != KDN_OK) return st;
-  return kdn::backward_launch(diag, in_dtype, q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave, dq,
-                              dk_, dv_, da, dw, dr, dS0, dp0, B, T, H, dk, dv, kappa,
-                              as_stream(stream));
+  return kdn::backward_launch(diag, in_dtype, q, k, v, a, w, r, dO, dS_T, dp_T, Ssave, Psave,
+                              reinterpret_cast<float*>(ws + L.scratch), dq, dk_, dv_, da, dw, dr,
+                              dS0, dp0, B, T, H, dk, dv, kappa, as_stream(stream));
 }
 
 kdn_status kdn_kla_forward(const void* q, const void* k, const void* v, kdn_dtype in_dtype,

@@ -21,6 +21,7 @@
 // decode step; the grid then spans all B*H heads and the kernel streams S
 // once in and once out (HBM-bound).
 #include "kdn_common.cuh"
+#include "bwd_checkpoint.h"
 
 namespace kdn {
 namespace {
@@ -62,8 +63,9 @@ __device__ __forceinline__ void load_state(const float* p, int lane, float (&x)[
 
 // Layout of the per-token tensors: q/k/v at ((b*T + t)*H + h)*d; a/w/r at
 // (b*T + t)*H + h (diag w: ((b*T + t)*H + h)*dk).  The decode step is T = 1.
-// SAVE: the state (S, p) before every token is also written to Ssave /
-// Psave ([B H][T][dv][dk] and [B H][T][1 or dk]) for the backward pass.
+// SAVE: for the backward pass, the variance p before every token goes to
+// Psave ([B H][T][1 or dk]) and the state S before every kBwdCheckpoint-th
+// token (t = 0, 16, 32, ...) to Ssave ([B H][ceil(T / 16)][dv][dk]).
 template <bool DIAG, int CPL, typename InT, bool SAVE>
 __global__ void __launch_bounds__(kWarps * 32)
 recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT* __restrict__ V,
@@ -116,13 +118,16 @@ recurrent_kernel(const InT* __restrict__ Q, const InT* __restrict__ K, const InT
   for (int t = 0; t < Tn; ++t) {
     const size_t tok = (row0 + t) * H + h;
     if constexpr (SAVE) {
-      const size_t sb = ((size_t)bh * T + t) * dv * DK;
+      if (t % kBwdCheckpoint == 0) {
+        const int nck = (T + kBwdCheckpoint - 1) / kBwdCheckpoint;
+        const size_t sb = ((size_t)bh * nck + t / kBwdCheckpoint) * dv * DK;
 #pragma unroll
-      for (int i = 0; i < kMaxRowsPerWarp; ++i) {
-        const int j = warp + kWarps * i;
-        if (j < dv) {
+        for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+          const int j = warp + kWarps * i;
+          if (j < dv) {
 #pragma unroll
-          for (int c = 0; c < CPL; ++c) Ssave[sb + (size_t)j * DK + lane * CPL + c] = S[i][c];
+            for (int c = 0; c < CPL; ++c) Ssave[sb + (size_t)j * DK + lane * CPL + c] = S[i][c];
+          }
         }
       }
       if constexpr (DIAG) {

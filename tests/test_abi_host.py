@@ -161,11 +161,13 @@ def test_backward_rejects_bad_arguments(L):
     assert x(var=5) == kdn.KDN_ERR_INVALID_ARG
     assert x(T=0) == kdn.KDN_ERR_INVALID_ARG
     assert x(dS_T=MIS) == kdn.KDN_ERR_INVALID_ARG
-    assert x(dkk=128) == kdn.KDN_ERR_UNSUPPORTED
+    assert x(dkk=96) == kdn.KDN_ERR_UNSUPPORTED
     assert x(dvv=129) == kdn.KDN_ERR_INVALID_ARG or x(dvv=129) == kdn.KDN_ERR_UNSUPPORTED
     assert x(ws=None) == kdn.KDN_ERR_WORKSPACE
     assert x(wsb=16) == kdn.KDN_ERR_WORKSPACE
-    assert L.kdn_backward_workspace_size(kdn.KDN_DIAG, 2, 10, 3, 32, 16) >= 2 * 3 * 10 * 16 * 32 * 4
+    # per head: one state checkpoint (T = 10 < 16) and 16 rebuilt states
+    assert L.kdn_backward_workspace_size(kdn.KDN_DIAG, 2, 10, 3, 32, 16) >= 2 * 3 * 17 * 16 * 32 * 4
+    assert L.kdn_backward_workspace_size(kdn.KDN_ISO, 1, 8, 1, 128, 128) > 0
 
 
 def test_varlen_rejects_bad_arguments(L):

@@ -45,16 +45,19 @@ def test_decode_and_exact_bytes():
 
 
 def test_backward_bytes():
-    B, T, H, d = 8, 4096, 16, 64
-    inputs = _nbytes(((B, T, H, d), 2), ((B, T, H, d), 2), ((B, T, H, d), 2),
-                     ((B, T, H), 4), ((B, T, H), 4), ((B, T, H), 4))
-    bwd = (2 * inputs                                   # the forward again, then the backward
-           + _nbytes(((B, T, H, d), 4))                 # dO read
-           + _nbytes(((B, T, H, d), 4))                 # the forward's o written
-           + 2 * _nbytes(((B, H, T, d, d), 4), ((B, H, T), 4))  # saved states, out and in
-           + _nbytes(((B, T, H, d), 4), ((B, T, H, d), 4), ((B, T, H, d), 4),  # dq, dk, dv
-                     ((B, T, H), 4), ((B, T, H), 4), ((B, T, H), 4)))         # da, dw, dr
-    assert bench.backward_bytes(B, T, H, d) == bwd
+    B, T, H, d = 8, 4096, 16, 128
+    for variant, dim in (('iso', 1), ('diag', d)):
+        wshape = (B, T, H) if variant == 'iso' else (B, T, H, d)
+        inputs = _nbytes(((B, T, H, d), 2), ((B, T, H, d), 2), ((B, T, H, d), 2),
+                         ((B, T, H), 4), (wshape, 4), ((B, T, H), 4))
+        bwd = (2 * inputs                                   # the forward again, then the backward
+               + _nbytes(((B, T, H, d), 4))                 # dO read
+               + _nbytes(((B, T, H, d), 4))                 # the forward's o written
+               + 2 * _nbytes(((B, H, T // 16, d, d), 4))    # state checkpoints, out and in
+               + 2 * _nbytes(((B, H, T, dim), 4))           # variances, out and in
+               + _nbytes(((B, T, H, d), 4), ((B, T, H, d), 4), ((B, T, H, d), 4),  # dq, dk, dv
+                         ((B, T, H), 4), (wshape, 4), ((B, T, H), 4)))            # da, dw, dr
+        assert bench.backward_bytes(B, T, H, d, variant) == bwd, variant
 
 
 def test_fp32_peak_is_the_unit_count_times_the_clock():

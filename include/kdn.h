@@ -166,8 +166,8 @@ kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w,
  *             start variances) is much larger, so query the size with the
  *             device that will run the call current.
  * Segmented forward: with dk = dv = 128 on the chunked path, when B H is at
- * most a quarter of the SM count and T is a multiple of 4096 (the segment
- * count S, a power of two >= 4 with B H S <= SMs and 1024 S dividing T, is
+ * most a quarter of the SM count and T is a multiple of 2048 (the segment
+ * count S, a power of two >= 4 with B H S <= SMs and 512 S dividing T, is
  * chosen by the library), the sequence is cut into S segments run as extra
  * heads of the engine: the variance at each segment start from the composed
  * Mobius maps, each segment's state transition from a run with V = 0 and
@@ -356,9 +356,11 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k,
  * (variant): the gradients of a loss L with respect to every input, given
  * dL/do, dL/dS_T and dL/dp_T ("Kalman Delta Networks: 不确定性感知的联想记忆",
  * 实验: the layers are trained in language models).  It runs the forward
- * again on the token-recurrent kernel, saving the state before every token
- * in the workspace, then the adjoint recursion from the last token to the
- * first (dS, dp carried backwards).
+ * again on the token-recurrent kernel, saving the variance before every
+ * token and the state before every 16th token in the workspace, then the
+ * adjoint recursion from the last token to the first (dS, dp carried
+ * backwards), block by block of 16 tokens: each block's states are rebuilt
+ * from its checkpoint, with the forward's arithmetic, before its adjoint.
  *
  * q, k, v, a, w, r, S0, p0, info_scale, in_dtype: as the forward call
  * dO       [B, T, H, dv] fp32 device: dL/do
@@ -368,9 +370,11 @@ kdn_status kdn_exact_forward(kdn_variant variant, const void* q, const void* k,
  * dw       [B, T, H] (iso) or [B, T, H, dk] (diag);  dS0 [B, H, dv, dk];
  * dp0      [B, H] (iso) or [B, H, dk] (diag): fp32 device outputs
  * workspace   device scratch of >= kdn_backward_workspace_size(...) bytes,
- *          256-byte aligned: B H T (dv dk + 1 or dk) floats of saved state,
- *          plus the forward's outputs
- * Supported: dk in {32, 64}; 1 <= dv <= 128; every pointer 16-byte aligned.
+ *          256-byte aligned: B H ceil(T / 16) dv dk floats of checkpoints,
+ *          B H T (1 or dk) floats of variances, B H 16 dv dk floats of
+ *          rebuilt states, plus the forward's outputs
+ * Supported: dk in {32, 64, 128}; 1 <= dv <= 128; every pointer 16-byte
+ * aligned.
  * Errors: KDN_ERR_INVALID_ARG, KDN_ERR_UNSUPPORTED, KDN_ERR_WORKSPACE,
  * KDN_ERR_CUDA, all before anything is enqueued except KDN_ERR_CUDA.
  * ---------------------------------------------------------------------- */

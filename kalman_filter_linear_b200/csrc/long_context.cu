@@ -16,7 +16,7 @@
 // The sequence is cut into S segments of L = T / S tokens, viewed as S extra
 // batch entries of the same [B, T, H, d] tensors ([B S, L, H, d] is the same
 // memory).  Then:
-//   1. every lane composes the Mobius maps of blocks of 1024 tokens in
+//   1. every lane composes the Mobius maps of blocks of 512 tokens in
 //      parallel, and one pass per lane applies the block products in order,
 //      recording the variance at each segment start;
 //   2. the engine runs all segments from S_start = 0 (giving E) and, with V
@@ -47,7 +47,7 @@ kdn_status chunk_engine_launch_zero_v(bool diag, const void* q, const void* k, c
 namespace {
 
 constexpr int kD = 128;          // d_k = d_v of the engine
-constexpr int kBlock = 1024;     // tokens per composed Mobius block
+constexpr int kBlock = 512;      // tokens per composed Mobius block
 constexpr int kMinSegments = 4;  // three engine passes over 1/S of the tokens each
 
 struct M2 {
@@ -74,35 +74,51 @@ __device__ __forceinline__ M2 step_map(float a, float w, float r, float c) {
   return {r * a2, r * w, c * a2, fmaf(c, w, r)};
 }
 
-// Diagonal variant: lane (b, h, i), block j of kBlock tokens.  Threads of a
-// warp take consecutive i, so every token's w and k reads are coalesced.
+// Diagonal variant: lanes (b, h, i) for i in a group of 4 dimensions, block
+// j of kBlock tokens.  Threads of a warp take consecutive groups, so every
+// token's w (16 bytes) and k (8 bytes) reads are coalesced; the four chains
+// are independent.
 __global__ void __launch_bounds__(256)
 block_maps_diag_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ A,
                        const float* __restrict__ W, const float* __restrict__ R, int B, int T,
                        int H, int nblk, float4* __restrict__ prod) {
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t lanes = (int64_t)B * H * kD;
-  if (gid >= lanes * nblk) return;
-  const int j = (int)(gid / lanes);
-  const int64_t lane = gid % lanes;
-  const int i = (int)(lane % kD);
-  const int h = (int)((lane / kD) % H);
-  const int b = (int)(lane / ((int64_t)kD * H));
+  const int64_t groups = (int64_t)B * H * (kD / 4);
+  if (gid >= groups * nblk) return;
+  const int j = (int)(gid / groups);
+  const int64_t grp = gid % groups;
+  const int i0 = (int)(grp % (kD / 4)) * 4;
+  const int h = (int)((grp / (kD / 4)) % H);
+  const int b = (int)(grp / ((int64_t)(kD / 4) * H));
   const int t0 = j * kBlock, t1 = min(T, t0 + kBlock);
-  M2 P = {1.f, 0.f, 0.f, 1.f};
-#pragma unroll 4
+  M2 P[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) P[e] = {1.f, 0.f, 0.f, 1.f};
+#pragma unroll 2
   for (int t = t0; t < t1; ++t) {
     const size_t tok = ((size_t)b * T + t) * H + h;
-    const float kv = __bfloat162float(K[tok * kD + i]);
-    P = mul(step_map(__ldg(A + tok), __ldg(W + tok * kD + i), __ldg(R + tok), kv * kv), P);
-    if ((t & 7) == 7) P = renorm(P);
+    const float4 w4 = __ldg(reinterpret_cast<const float4*>(W + tok * kD + i0));
+    const uint2 k2 = __ldg(reinterpret_cast<const uint2*>(K + tok * kD + i0));
+    const float a = __ldg(A + tok), r = __ldg(R + tok);
+    const float kv[4] = {__uint_as_float(k2.x << 16), __uint_as_float(k2.x & 0xffff0000u),
+                         __uint_as_float(k2.y << 16), __uint_as_float(k2.y & 0xffff0000u)};
+    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      P[e] = mul(step_map(a, wv[e], r, kv[e] * kv[e]), P[e]);
+      if ((t & 3) == 3) P[e] = renorm(P[e]);
+    }
   }
-  P = renorm(P);
-  prod[lane * nblk + j] = make_float4(P.a, P.b, P.c, P.d);
+  const int64_t lane0 = ((int64_t)b * H + h) * kD + i0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const M2 Q = renorm(P[e]);
+    prod[(lane0 + e) * nblk + j] = make_float4(Q.a, Q.b, Q.c, Q.d);
+  }
 }
 
 // Isotropic variant: lane (b, h), block j; one warp per (lane, block), lane
-// l composing tokens [t0 + 32 l, t0 + 32 l + 32) (c = kappa ||k||^2), then
+// l composing the l-th 1/32 of the block's tokens (c = kappa ||k||^2), then
 // the 32 partial products combined in token order.
 __global__ void __launch_bounds__(256)
 block_maps_iso_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ A,
@@ -115,7 +131,7 @@ block_maps_iso_kernel(const __nv_bfloat16* __restrict__ K, const float* __restri
   const int j = (int)(wid / lanes);
   const int64_t lane = wid % lanes;
   const int h = (int)(lane % H), b = (int)(lane / H);
-  const int t0 = j * kBlock + 32 * l, t1 = min(T, t0 + 32);
+  const int t0 = j * kBlock + (kBlock / 32) * l, t1 = min(T, t0 + kBlock / 32);
   M2 P = {1.f, 0.f, 0.f, 1.f};
   for (int t = t0; t < t1; ++t) {
     const size_t tok = ((size_t)b * T + t) * H + h;
@@ -132,7 +148,7 @@ block_maps_iso_kernel(const __nv_bfloat16* __restrict__ K, const float* __restri
       }
     }
     P = mul(step_map(__ldg(A + tok), __ldg(W + tok), __ldg(R + tok), kappa * n), P);
-    if ((t & 7) == 7) P = renorm(P);
+    if ((t & 3) == 3) P = renorm(P);
   }
   P = renorm(P);
   // ordered product over the warp: lane l's tokens come after lane l - 1's
@@ -180,14 +196,18 @@ __global__ void identity_kernel(float* __restrict__ S, int64_t n) {
 
 // Segment starts: S_start(0) = S0 (or 0), S_start(s + 1) = S_start(s) F(s) +
 // E(s).  One CTA per (batch entry, head, block of 16 rows of S); rows of S
-// do not mix, so the blocks are independent.  State layouts: [(b S + s), H,
-// kD, kD] for F, E and S_start; S0 [B, H, kD, kD].
+// do not mix, so the blocks are independent.  Each F(s) is staged in shared
+// memory (64 KB) with coalesced loads before the products.  State layouts:
+// [(b S + s), H, kD, kD] for F, E and S_start; S0 [B, H, kD, kD].
 constexpr int kRows = 16;
+constexpr size_t kChainSmem = (size_t)(kD * kD + kRows * kD) * sizeof(float);
 __global__ void __launch_bounds__(256)
 chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
                       const float* __restrict__ E, int B, int H, int nseg,
                       float* __restrict__ S_start) {
-  __shared__ float cur[kRows][kD];
+  extern __shared__ float4 chain_smem[];
+  float* Fsm = reinterpret_cast<float*>(chain_smem);  // [kD][kD]
+  float* cur = Fsm + kD * kD;                         // [kRows][kD]
   const int rb = blockIdx.x % (kD / kRows);
   const int h = (blockIdx.x / (kD / kRows)) % H;
   const int b = blockIdx.x / ((kD / kRows) * H);
@@ -201,21 +221,23 @@ chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float x = src ? src[e] : 0.f;
-      cur[r][c0 + e] = x;
+      cur[r * kD + c0 + e] = x;
       dst[e] = x;
     }
   }
-  __syncthreads();
   for (int s = 0; s + 1 < nseg; ++s) {
-    const float* Fs = F + at(s);
+    const float4* Fs4 = reinterpret_cast<const float4*>(F + at(s));
+    for (int i = tid; i < kD * kD / 4; i += 256) chain_smem[i] = __ldg(Fs4 + i);
+    __syncthreads();  // F(s) staged; cur written
     const float* Es = E + at(s) + (size_t)row * kD + c0;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = Es[e];
+#pragma unroll 4
     for (int j = 0; j < kD; ++j) {
-      const float x = cur[r][j];
-      const float4 f0 = *reinterpret_cast<const float4*>(Fs + (size_t)j * kD + c0);
-      const float4 f1 = *reinterpret_cast<const float4*>(Fs + (size_t)j * kD + c0 + 4);
+      const float x = cur[r * kD + j];
+      const float4 f0 = *reinterpret_cast<const float4*>(Fsm + j * kD + c0);
+      const float4 f1 = *reinterpret_cast<const float4*>(Fsm + j * kD + c0 + 4);
       acc[0] = fmaf(x, f0.x, acc[0]);
       acc[1] = fmaf(x, f0.y, acc[1]);
       acc[2] = fmaf(x, f0.z, acc[2]);
@@ -225,14 +247,13 @@ chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
       acc[6] = fmaf(x, f1.z, acc[6]);
       acc[7] = fmaf(x, f1.w, acc[7]);
     }
-    __syncthreads();  // every thread has read cur
+    __syncthreads();  // every thread has read cur and F(s)
     float* dst = S_start + at(s + 1) + (size_t)row * kD + c0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      cur[r][c0 + e] = acc[e];
+      cur[r * kD + c0 + e] = acc[e];
       dst[e] = acc[e];
     }
-    __syncthreads();
   }
 }
 
@@ -279,8 +300,8 @@ SegLayout seg_layout(bool diag, int B, int T, int H, int nseg) {
 
 // Number of segments for a call of the d_v = 128 engine on the current
 // device: the largest power of two S >= 4 with B H S CTAs fitting on the SMs
-// at once and T a multiple of 1024 S (whole composed blocks per segment),
-// or 1 (no segmentation).
+// at once and T a multiple of 512 S (whole composed blocks per segment), or
+// 1 (no segmentation).
 int segment_count(int B, int T, int H) {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -319,7 +340,7 @@ kdn_status segmented_forward(bool diag, const void* q, const void* k, const void
   // 1. variances at the segment starts
   const int64_t lanes = (int64_t)B * H * dim;
   if (diag) {
-    const int64_t n = lanes * nblk;
+    const int64_t n = lanes / 4 * nblk;
     block_maps_diag_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(k), a, w, r, B, T, H, nblk, prod);
   } else {
@@ -342,8 +363,11 @@ kdn_status segmented_forward(bool diag, const void* q, const void* k, const void
   if (stt != KDN_OK) return stt;
 
   // 3. the true state at every segment start
-  chain_segments_kernel<<<(unsigned)(B * H * (kD / kRows)), 256, 0, st>>>(S0, F, E, B, H, nseg,
-                                                                          S_start);
+  if (cudaFuncSetAttribute(chain_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kChainSmem) != cudaSuccess)
+    return KDN_ERR_CUDA;
+  chain_segments_kernel<<<(unsigned)(B * H * (kD / kRows)), 256, kChainSmem, st>>>(
+      S0, F, E, B, H, nseg, S_start);
   if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
 
   // 4. every segment from its true start: o, and each segment's final state

@@ -1735,27 +1735,10 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         umma_commit(mma3_bar);
         pend_mma3 = c & 1;
       }
-      // ---- while MMA3 runs: gamma (Q S')^T in place (before MMA4 adds to it)
-      // and the state decay by gamma_C (before MMA5 adds to it)
+      // ---- while MMA3 runs: the state decay by gamma_C (before MMA5 adds to
+      // it).  (Q S')^T stays in the query half of D2; MMA4 writes U^T P^T to
+      // the key half, which Z has read, and the output pass combines them.
       {
-        float qs[32];
-        uint32_t qr[32];
-        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qs);
-        tmem_wait_ld();
-        const float4* gm4 = reinterpret_cast<const float4*>(sc_gam + 64 * sl + 32 * ch);
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 g4 = gm4[i4];
-          const float2 p0 = __fmul2_rn(make_float2(g4.x, g4.y),
-                                       make_float2(qs[4 * i4], qs[4 * i4 + 1]));
-          const float2 p1 = __fmul2_rn(make_float2(g4.z, g4.w),
-                                       make_float2(qs[4 * i4 + 2], qs[4 * i4 + 3]));
-          qr[4 * i4] = __float_as_uint(p0.x);
-          qr[4 * i4 + 1] = __float_as_uint(p0.y);
-          qr[4 * i4 + 2] = __float_as_uint(p1.x);
-          qr[4 * i4 + 3] = __float_as_uint(p1.y);
-        }
-        tmem_st32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, qr);
         const float gC = sc_gC[sl];
 #pragma unroll
         for (int h32 = 0; h32 < 2; ++h32) {
@@ -1829,8 +1812,9 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint64_t dp = umma_desc_sw128(sbase + P::OFF_P, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          umma_tf32_ts(tmem + P::COL_D2 + 64, tmem + P::COL_D3 + 8 * ks,
-                       dp + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), ID_4, 1u);
+          umma_tf32_ts(tmem + P::COL_D2, tmem + P::COL_D3 + 8 * ks,
+                       dp + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), ID_4,
+                       ks > 0 ? 1u : 0u);
         umma_commit(mma4_bar);
         pend_mma4 = c & 1;
       }
@@ -1849,10 +1833,35 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
       // (also the isotropic variant for the last, partial chunk of a packed
       // sequence: a tile store there would run into the next sequence)
       const bool direct = DIAG || (PACKED && Tn - t0 < kC);
+      // o^T [v][t] of this warp's tokens = gamma_t (Q S')^T (query half of D2)
+      // + (U^T P^T) (key half)
+      auto out_cols = [&](float (&x)[32]) {
+        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
+        const float4* gm4 = reinterpret_cast<const float4*>(sc_gam + 64 * sl + 32 * ch);
+#pragma unroll
+        for (int h16 = 0; h16 < 2; ++h16) {
+          float y[16];
+          tmem_ld16(tmem + tm_lane + P::COL_D2 + 32 * ch + 16 * h16, y);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const float4 g4 = gm4[4 * h16 + i4];
+            const int i = 16 * h16 + 4 * i4;
+            const float2 o0 = __ffma2_rn(make_float2(g4.x, g4.y), make_float2(x[i], x[i + 1]),
+                                         make_float2(y[4 * i4], y[4 * i4 + 1]));
+            const float2 o1 = __ffma2_rn(make_float2(g4.z, g4.w),
+                                         make_float2(x[i + 2], x[i + 3]),
+                                         make_float2(y[4 * i4 + 2], y[4 * i4 + 3]));
+            x[i] = o0.x;
+            x[i + 1] = o0.y;
+            x[i + 2] = o1.x;
+            x[i + 3] = o1.y;
+          }
+        }
+      };
       if (direct) {
         float x[32];
-        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
-        tmem_wait_ld();
+        out_cols(x);
         const int valid = min(kC, Tn - t0);
         float* dst = O + (((size_t)b * T + tbeg + t0 + 32 * ch) * H + h) * DV + v;
         const size_t ostride = (size_t)H * DV;
@@ -1861,8 +1870,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (32 * ch + i < valid) dst[i * ostride] = x[i];
       } else {
         float x[32];
-        tmem_ld32(tmem + tm_lane + P::COL_D2 + 64 + 32 * ch, x);
-        tmem_wait_ld();
+        out_cols(x);
         float* dst = sOut + (32 * ch) * DV + v;
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * DV] = x[i];

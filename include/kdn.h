@@ -171,11 +171,12 @@ kdn_status kdn_mobius_scan_noalloc(const float* a, const float* w,
  * chosen by the library), the sequence is cut into S segments run as extra
  * heads of the engine: the variance at each segment start from the composed
  * Mobius maps, each segment's state transition from a run with V = 0 and
- * S0 = I and its zero-start state from a run with S0 = 0, the segment
- * starts chained, and a last run from the true starts.  The memory
- * recursion is affine in the state, so the result is the same up to
- * rounding; it takes three engine passes over T / S tokens each instead of
- * one over T.
+ * S0 = I and its zero-start state and outputs from a run with S0 = 0, the
+ * segment starts chained, and the outputs corrected by the segment start
+ * state times the transition run's outputs (a tf32 tensor-core product).
+ * The memory recursion is affine in the state, so the result is the same up
+ * to rounding; it takes two engine passes over T / S tokens each instead of
+ * one over T, and a workspace the size of o.
  * Supported: T >= 1; dk in {32, 64, 128}; 1 <= dv <= 128.  KDN_CHUNK_64
  * additionally needs in_dtype == KDN_BF16, dk == 128 and dv in {64, 128}.
  * All pointers 16-byte aligned.  o must not alias the inputs.

@@ -27,6 +27,9 @@
 //   4. the engine runs all segments from their true S_start, writing o and
 //      each segment's final state, of which the last segment's is S_T.
 // Steps 2 and 4 have S times the heads of the call, at 1/S of its length.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
 
 #include "kdn_common.cuh"
@@ -195,7 +198,8 @@ __global__ void identity_kernel(float* __restrict__ S, int64_t n) {
 }
 
 // Segment starts: S_start(0) = S0 (or 0), S_start(s + 1) = S_start(s) F(s) +
-// E(s).  One CTA per (batch entry, head, block of 16 rows of S); rows of S
+// E(s), and after the last segment the call's final state S_T into S_out
+// ([B, H, kD, kD]).  One CTA per (batch entry, head, block of 16 rows of S); rows of S
 // do not mix, so the blocks are independent.  Each F(s) is staged in shared
 // memory (64 KB) with coalesced loads before the products.  State layouts:
 // [(b S + s), H, kD, kD] for F, E and S_start; S0 [B, H, kD, kD].
@@ -204,7 +208,7 @@ constexpr size_t kChainSmem = (size_t)(kD * kD + kRows * kD) * sizeof(float);
 __global__ void __launch_bounds__(256)
 chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
                       const float* __restrict__ E, int B, int H, int nseg,
-                      float* __restrict__ S_start) {
+                      float* __restrict__ S_start, float* __restrict__ S_out) {
   extern __shared__ float4 chain_smem[];
   float* Fsm = reinterpret_cast<float*>(chain_smem);  // [kD][kD]
   float* cur = Fsm + kD * kD;                         // [kRows][kD]
@@ -225,7 +229,7 @@ chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
       dst[e] = x;
     }
   }
-  for (int s = 0; s + 1 < nseg; ++s) {
+  for (int s = 0; s < nseg; ++s) {
     const float4* Fs4 = reinterpret_cast<const float4*>(F + at(s));
     for (int i = tid; i < kD * kD / 4; i += 256) chain_smem[i] = __ldg(Fs4 + i);
     __syncthreads();  // F(s) staged; cur written
@@ -248,7 +252,9 @@ chain_segments_kernel(const float* __restrict__ S0, const float* __restrict__ F,
       acc[7] = fmaf(x, f1.w, acc[7]);
     }
     __syncthreads();  // every thread has read cur and F(s)
-    float* dst = S_start + at(s + 1) + (size_t)row * kD + c0;
+    // (after the last segment: the final state of the call)
+    float* dst = s + 1 < nseg ? S_start + at(s + 1) + (size_t)row * kD + c0
+                              : S_out + ((((size_t)b * H + h) * kD) + row) * kD + c0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       cur[r * kD + c0 + e] = acc[e];
@@ -262,10 +268,167 @@ __global__ void or_error_words(uint32_t* dst, const uint32_t* a, const uint32_t*
   atomicOr(dst, *a | *b | *c);
 }
 
+// ----------------------------------------------------- output correction
+// o(t) = o_E(t) + S_start o_F(t) for every token of a segment: the pass from
+// S_start = I with V = 0 reads out o_F(t) = F_(0..t) q_t, so the state at
+// token t, S_start F_(0..t) + E_t, gives the output through one matrix
+// product per token.  Per (segment, head) it is a [128 v x 128 k] x [128 k x
+// tokens] product, D[v][t] = sum_k S_start[v][k] o_F[t][k], on the tensor
+// cores in tf32 (both operands fp32 in shared memory, K-major, 128-byte
+// swizzle; the correction's relative error is about 2^-10 of its size, well
+// inside the output bound), with the fp32 accumulator in TMEM.  One CTA of
+// four warps per (segment, head, 8 or 4 tiles of 128 tokens): S_start comes in
+// once, each token tile by TMA, 16 MMAs of K = 8, then each thread (one value
+// row v) adds its TMEM row to o in place, 32 tokens at a time, coalesced
+// over v.
+constexpr int kCorrTiles = 8;  // token tiles of 128 per CTA (4 when 8 does not divide a segment)
+constexpr uint32_t kOperandBytes = 128u * 128u * 4u;  // 64 KB, [4 kb][128 rows][32 k]
+constexpr uint32_t kCorrSmem = 2 * kOperandBytes + 1024 + 64;
+
+__device__ __forceinline__ void umma_tf32_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__global__ void __launch_bounds__(128, 1)
+correct_outputs_kernel(const __grid_constant__ CUtensorMap tm_s,
+                       const __grid_constant__ CUtensorMap tm_of, float* __restrict__ O, int H,
+                       int L, int ntile, uint32_t* __restrict__ err) {
+  extern __shared__ uint8_t corr_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(corr_raw) + 1023u) & ~uintptr_t(1023u));
+  uint8_t* sA = smem;                    // S_start [4 kb][128 v][32 k]
+  uint8_t* sB = smem + kOperandBytes;    // o_F tile [4 kb][128 t][32 k]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kOperandBytes);
+  uint64_t* full_a = bars;
+  uint64_t* full_b = bars + 1;
+  uint64_t* mma_done = bars + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  __shared__ int s_bad;
+
+  const int groups = (L / 128) / ntile;
+  const int g = blockIdx.x % groups;
+  const int h = (blockIdx.x / groups) % H;
+  const int bs = blockIdx.x / (groups * H);  // segment (b, s) of the [B S, L, H, d] view
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  if (tid == 0) {
+    mbar_init(full_a, 1);
+    mbar_init(full_b, 1);
+    mbar_init(mma_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    s_bad = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto load_b = [&](int tile) {
+    mbar_expect_tx(full_b, kOperandBytes);
+    for (int kb = 0; kb < 4; ++kb)
+      tma_load_4d(sB + kb * 16384, &tm_of, full_b, 32 * kb, h, 128 * tile, bs);
+  };
+  const int tile0 = g * ntile;
+  if (tid == 0) {
+    mbar_expect_tx(full_a, kOperandBytes);
+    for (int kb = 0; kb < 4; ++kb)
+      tma_load_4d(sA + kb * 16384, &tm_s, full_a, 32 * kb, 0, h, bs);
+    load_b(tile0);
+  }
+  constexpr uint32_t IDESC = umma_idesc(128, 128, 2, 0, 0);  // tf32, both K-major
+  bool bad = !mbar_wait(full_a, 0);
+  for (int i = 0; i < ntile; ++i) {
+    if (!bad && !mbar_wait(full_b, (uint32_t)(i & 1))) bad = true;
+    if (tid == 0 && !bad) {
+      tc_fence_after();
+      const uint64_t da = umma_desc_sw128(smem_u32(sA), 16, 1024);
+      const uint64_t db = umma_desc_sw128(smem_u32(sB), 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const uint64_t off = (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4);
+        umma_tf32_ss(tmem, da + off, db + off, IDESC, ks > 0 ? 1u : 0u);
+      }
+      umma_commit(mma_done);
+    }
+    if (!bad && !mbar_wait(mma_done, (uint32_t)(i & 1))) bad = true;
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) {
+        atomicOr(err, DEV_TIMEOUT);
+        s_bad = 1;
+      }
+      break;
+    }
+    tc_fence_after();
+    // the tile's operand has been read: copy the next one during the epilogue
+    if (tid == 0 && i + 1 < ntile) load_b(tile0 + i + 1);
+    const int t0 = 128 * (tile0 + i);
+    float* orow = O + (((size_t)bs * L + t0) * H + h) * 128 + tid;  // v = tid
+    const size_t tstride = (size_t)H * 128;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      // the 32 o_E values first (all loads in flight at once), then the
+      // TMEM columns, then the sums
+      float e[32], d[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) e[j] = __ldcs(orow + (size_t)(32 * c + j) * tstride);
+      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * c, d);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) __stcs(orow + (size_t)(32 * c + j) * tstride, e[j] + d[j]);
+    }
+    tc_fence_before();
+    __syncthreads();  // every thread has read D before the next MMA writes it
+  }
+  if (tid == 0 && s_bad) {
+    // bounded waits for what may still be in flight
+    (void)mbar_wait(mma_done, 0);
+    (void)mbar_wait(full_b, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// fp32 4-D map, 128-byte swizzle, box (32, box1, box2, 1)
+bool make_f32_map(CUtensorMap* m, const void* base, const cuuint64_t (&dims)[4], int box1,
+                  int box2) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t strides[3] = {dims[0] * 4, dims[0] * dims[1] * 4, dims[0] * dims[1] * dims[2] * 4};
+  cuuint32_t box[4] = {32, (cuuint32_t)box1, (cuuint32_t)box2, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct SegLayout {
-  size_t err_e, err_f, err_g, prod, p_start, p_scratch, ident, E, F, S_start, zero_v, total;
+  size_t err_e, err_f, err_g, prod, p_start, p_scratch, p_scratch2, ident, E, F, S_start, zero_v,
+      o_f, total;
 };
 
 // Workspace: the call's error word (bytes 0-3, first 256-byte block), one
@@ -287,11 +450,13 @@ SegLayout seg_layout(bool diag, int B, int T, int H, int nseg) {
   L.prod = take((size_t)B * H * dim * (T / kBlock) * 16);
   L.p_start = take(vars);
   L.p_scratch = take(vars);
+  L.p_scratch2 = take(vars);
   L.ident = take(states);
   L.E = take(states);
   L.F = take(states);
   L.S_start = take(states);
   L.zero_v = take((size_t)64 * H * kD * 2);
+  L.o_f = take((size_t)B * T * H * kD * 4);  // output of the S_start = I pass
   L.total = off;
   return L;
 }
@@ -353,33 +518,46 @@ kdn_status segmented_forward(bool diag, const void* q, const void* k, const void
   identity_kernel<<<592, 256, 0, st>>>(ident, (int64_t)Bs * H);
   if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
 
-  // 2. every segment from S_start = 0 (E), and with V read as zero from
-  // S_start = I (F).  Their outputs land in o; pass 4 overwrites them.
+  // 2. every segment from S_start = 0 (E; o_E into o), and with V read as
+  // zero from S_start = I (F; o_F(t) = F_(0..t) q_t into the workspace)
+  float* o_f = reinterpret_cast<float*>(base + L.o_f);
+  float* p_scratch2 = reinterpret_cast<float*>(base + L.p_scratch2);
   kdn_status stt = chunk_engine_launch(diag, q, k, v, a, w, r, nullptr, p_start, o, E, p_scratch,
                                        Bs, Ls, H, kD, kappa, base + L.err_e, st, -1, nullptr);
   if (stt != KDN_OK) return stt;
-  stt = chunk_engine_launch_zero_v(diag, q, k, base + L.zero_v, a, w, r, ident, p_start, o, F,
-                                   p_scratch, Bs, Ls, H, kappa, base + L.err_f, st);
+  stt = chunk_engine_launch_zero_v(diag, q, k, base + L.zero_v, a, w, r, ident, p_start, o_f, F,
+                                   p_scratch2, Bs, Ls, H, kappa, base + L.err_f, st);
   if (stt != KDN_OK) return stt;
 
-  // 3. the true state at every segment start
+  // 3. the true state at every segment start, and the final state
   if (cudaFuncSetAttribute(chain_segments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kChainSmem) != cudaSuccess)
     return KDN_ERR_CUDA;
   chain_segments_kernel<<<(unsigned)(B * H * (kD / kRows)), 256, kChainSmem, st>>>(
-      S0, F, E, B, H, nseg, S_start);
+      S0, F, E, B, H, nseg, S_start, S_out);
   if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
 
-  // 4. every segment from its true start: o, and each segment's final state
-  // and variance (into E and p_scratch), of which the last segment's are the
-  // call's
-  stt = chunk_engine_launch(diag, q, k, v, a, w, r, S_start, p_start, o, E, p_scratch, Bs, Ls, H,
-                            kD, kappa, base + L.err_g, st, -1, nullptr);
-  if (stt != KDN_OK) return stt;
-  const size_t sbytes = (size_t)H * kD * kD * 4, pbytes = (size_t)H * dim * 4;
-  if (cudaMemcpy2DAsync(S_out, sbytes, E + (size_t)(nseg - 1) * H * kD * kD, sbytes * nseg,
-                        sbytes, B, cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
-      cudaMemcpy2DAsync(p_out, pbytes, p_scratch + (size_t)(nseg - 1) * H * dim, pbytes * nseg,
+  // 4. o += S_start o_F on every segment (segment 0 of each batch entry too,
+  // unless it starts from zero)
+  CUtensorMap tm_s, tm_of;
+  const cuuint64_t sdims[4] = {(cuuint64_t)kD, (cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)Bs};
+  const cuuint64_t odims[4] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)Ls, (cuuint64_t)Bs};
+  if (!make_f32_map(&tm_s, S_start, sdims, kD, 1) || !make_f32_map(&tm_of, o_f, odims, 1, 128))
+    return KDN_ERR_CUDA;
+  if (cudaFuncSetAttribute(correct_outputs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kCorrSmem) != cudaSuccess)
+    return KDN_ERR_CUDA;
+  if (cudaMemsetAsync(base + L.err_g, 0, 4, st) != cudaSuccess) return KDN_ERR_CUDA;
+  // (every segment: the first of each batch entry adds S0 o_F, zero without S0)
+  const int ntile = (Ls / 128) % kCorrTiles == 0 ? kCorrTiles : 4;
+  const int groups = (Ls / 128) / ntile;
+  correct_outputs_kernel<<<(unsigned)(Bs * H * groups), 128, kCorrSmem, st>>>(
+      tm_s, tm_of, o, H, Ls, ntile, reinterpret_cast<uint32_t*>(base + L.err_g));
+  if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
+
+  // the call's final variance: the end variance of the last segment
+  const size_t pbytes = (size_t)H * dim * 4;
+  if (cudaMemcpy2DAsync(p_out, pbytes, p_scratch + (size_t)(nseg - 1) * H * dim, pbytes * nseg,
                         pbytes, B, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return KDN_ERR_CUDA;
   or_error_words<<<1, 1, 0, st>>>(static_cast<uint32_t*>(ws),

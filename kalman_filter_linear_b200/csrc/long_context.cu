@@ -97,7 +97,7 @@ block_maps_diag_kernel(const __nv_bfloat16* __restrict__ K, const float* __restr
   M2 P[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) P[e] = {1.f, 0.f, 0.f, 1.f};
-#pragma unroll 2
+#pragma unroll 8
   for (int t = t0; t < t1; ++t) {
     const size_t tok = ((size_t)b * T + t) * H + h;
     const float4 w4 = __ldg(reinterpret_cast<const float4*>(W + tok * kD + i0));

@@ -447,7 +447,7 @@ def main():
     # closing barrier (under the process group's timeout) while rank 0 measures
     secondary = {}
     if not args.no_secondary and rank == 0 and world == 1:
-        secondary = measure_secondary(kdn, synth, dev, stream, hbm_peak)
+        secondary = measure_secondary(kdn, synth, dev, stream, hbm_peak, tf_peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -630,6 +630,14 @@ def exact_flops(B, T, H, dk, dv):
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
+def kla_engine_flops(B, T, H):
+    """Tensor FLOPs the KLA engine executes (bf16 hi/lo terms included): per
+    64-token chunk and head, MMA-A 16 and MMA-O 24 instructions of 128x64x16,
+    MMA-I 12 of 128x64x16, MMA-dS 8 of 128x128x16."""
+    per_chunk = (16 + 24 + 12) * 2 * 128 * 64 * 16 + 8 * 2 * 128 * 128 * 16
+    return B * H * ((T + 63) // 64) * per_chunk
+
+
 def exact_case(kdn, synth, dev, B=None, T=None):
     """The dense filter: (launch fn, tokens, algorithmic bytes, description)."""
     import torch
@@ -646,7 +654,7 @@ def exact_case(kdn, synth, dev, B=None, T=None):
     return f, B * T, exact_bytes(B, T, H, dk, dv), {'B': B, 'T': T, 'H': H, 'dk': dk, 'dv': dv}
 
 
-def measure_secondary(kdn, synth, dev, stream, hbm_peak):
+def measure_secondary(kdn, synth, dev, stream, hbm_peak, tensor_peak):
     import torch
     out = {}
     # diagonal forward, same shape
@@ -718,7 +726,9 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     out['iso_varlen'] = {'tokens_per_s': units / ms * 1e3, 'ms': ms,
                          'achieved_gbs': alg / ms / 1e6, 'frac': alg / ms / 1e6 / hbm_peak,
                          'algorithmic_bytes': alg, **desc}
-    # information-form diagonal filter (KLA) on the Diagonal KDN's inputs
+    # information-form diagonal filter (KLA) on the Diagonal KDN's inputs: the
+    # chunked tensor-core engine (kdn_kla_forward_ws), and the token-recurrent
+    # kernel (kdn_kla_forward) for comparison
     c = synth.WORKLOADS['diag_1p3b']
     B, T, H, d = c['B'], c['T'], c['H'], c['dk']
     x = {k: v.to(dev) for k, v in synth.layer_inputs(B, T, H, d, d, 'diag', c['seed'],
@@ -726,16 +736,28 @@ def measure_secondary(kdn, synth, dev, stream, hbm_peak):
     o = torch.empty((B, T, H, d), dtype=torch.float32, device=dev)
     S = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
     lam = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    wsk = torch.zeros(kdn.kdn_kla_workspace_size(B, T, H, d, d), dtype=torch.uint8, device=dev)
     f = lambda: kdn.kdn_kla_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], o=o,
-                                    S_out=S, lam_out=lam)
-    n = 5
+                                    S_out=S, lam_out=lam, workspace=wsk)
+    n = 10
     ms = time_launches(f, n, 3, stream) / n
     alg = layer_bytes('diag', B, T, H, d, d)
-    fl = B * T * H * 5 * d * d  # S f + v u^T (3 per element), S q (2)
+    tfl = kla_engine_flops(B, T, H)
     out['kla_1p3b'] = {'tokens_per_s': B * T / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
                        'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg,
-                       'alu': {'achieved_tflops': fl / ms / 1e9, 'peak_tflops': FP32_PEAK_TFLOPS,
-                               'frac': fl / ms / 1e9 / FP32_PEAK_TFLOPS, 'flops': fl}}
+                       'tensor': {'executed_flops': tfl, 'achieved_tflops': tfl / ms / 1e9,
+                                  'peak_tflops': tensor_peak,
+                                  'frac': tfl / ms / 1e9 / tensor_peak}}
+    fr = lambda: kdn.kdn_kla_forward(x['q'], x['k'], x['v'], x['a'], x['w'], x['r'], o=o,
+                                     S_out=S, lam_out=lam, recurrent=True)
+    n = 5
+    ms = time_launches(fr, n, 3, stream) / n
+    fl = B * T * H * 5 * d * d  # S f + v u^T (3 per element), S q (2)
+    out['kla_recurrent_1p3b'] = {
+        'tokens_per_s': B * T / ms * 1e3, 'ms': ms, 'achieved_gbs': alg / ms / 1e6,
+        'frac': alg / ms / 1e6 / hbm_peak, 'algorithmic_bytes': alg,
+        'alu': {'achieved_tflops': fl / ms / 1e9, 'peak_tflops': FP32_PEAK_TFLOPS,
+                'frac': fl / ms / 1e9 / FP32_PEAK_TFLOPS, 'flops': fl}}
     del x, o, S, lam
     # backward pass (token-recurrent), B8 T4096 H16 d64, isotropic
     c = synth.WORKLOADS['exact_d64']

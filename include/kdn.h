@@ -423,6 +423,37 @@ kdn_status kdn_kla_forward(const void* q, const void* k, const void* v,
                            int H, int dk, int dv, void* stream);
 
 /* ------------------------------------------------------------------------
+ * kdn_kla_forward_ws -- the same filter and arguments as kdn_kla_forward, plus
+ * a workspace.  For dk = dv = 128 with bf16 q, k, v it runs the chunked
+ * tensor-core engine ("Kalman Linear Attention: ...", 方法论 §2: given the
+ * precisions the mean recursion is affine, so a stretch of tokens is a few
+ * dense products).  Per 64-token chunk, with G the running product of the
+ * forget gates and Q~ = Q . G, U~ = U / G:
+ *   A = (Q~ U~^T) masked causal,  O = S0 Q~^T + A V,
+ *   S_C = (S0 + V^T U~) diag(G_C),
+ * on tcgen05 tensor cores with every fp32 operand split into bf16 hi + lo
+ * and fp32 accumulation; the precision recursion runs in fp32 per key
+ * dimension.  A chunk whose gates would drive G below 2^-100 is cut into
+ * shorter pieces (down to single tokens), so every input is served.  Other
+ * shapes and fp32 inputs run kdn_kla_forward's token-recurrent kernel.
+ * workspace   device memory of kdn_kla_workspace_size bytes (16-byte
+ *             aligned): the call's error word; kdn_read_workspace_status
+ *             reports KDN_ERR_TIMEOUT if a bounded on-device wait gave up
+ * Results match kdn_kla_forward's to the engine's operand precision (the
+ * bf16 hi/lo split keeps 16 significant bits of each fp32 operand).
+ * Errors: as kdn_kla_forward, plus KDN_ERR_WORKSPACE (NULL, misaligned or
+ * too small).
+ * ---------------------------------------------------------------------- */
+size_t kdn_kla_workspace_size(int B, int T, int H, int dk, int dv);
+kdn_status kdn_kla_forward_ws(const void* q, const void* k, const void* v,
+                              kdn_dtype in_dtype, const float* a,
+                              const float* w, const float* r, const float* S0,
+                              const float* lam0, float* o, float* S_out,
+                              float* lam_out, int B, int T, int H, int dk,
+                              int dv, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
  * kdn_read_workspace_status -- synchronise `stream`, then report the device
  * error word a previous call left in `workspace`: KDN_OK, KDN_ERR_TIMEOUT
  * if a bounded on-device wait gave up, or KDN_ERR_INVALID_ARG if packed-

@@ -52,6 +52,11 @@ kdn_status backward_launch(bool diag, kdn_dtype dt, const void* q, const void* k
                            float* da, float* dw, float* dr, float* dS0, float* dp0, int B, int T,
                            int H, int dkk, int dv, float kappa, cudaStream_t s);
 bool kla_supported(int dk, int dv);
+bool kla_engine_supported(kdn_dtype dt, int dk, int dv, int T);
+kdn_status kla_engine_launch(const void* q, const void* k, const void* v, const float* a,
+                             const float* w, const float* r, const float* S0, const float* L0,
+                             float* o, float* S_out, float* L_out, int B, int T, int H, void* ws,
+                             cudaStream_t s);
 kdn_status kla_launch(kdn_dtype dt, const void* q, const void* k, const void* v, const float* a,
                       const float* w, const float* r, const float* S0, const float* L0, float* o,
                       float* S_out, float* L_out, int B, int T, int H, int dk, int dv,
@@ -388,6 +393,35 @@ kdn_status kdn_kla_forward(const void* q, const void* k, const void* v, kdn_dtyp
   if (!kdn::kla_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
   return kdn::kla_launch(in_dtype, q, k, v, a, w, r, S0, lam0, o, S_out, lam_out, B, T, H, dk,
                          dv, as_stream(stream));
+}
+
+size_t kdn_kla_workspace_size(int B, int T, int H, int dk, int dv) {
+  if (!shape_ok(B, T, H, dk, dv) || !kdn::kla_supported(dk, dv)) return 0;
+  return 256;
+}
+
+kdn_status kdn_kla_forward_ws(const void* q, const void* k, const void* v, kdn_dtype in_dtype,
+                              const float* a, const float* w, const float* r, const float* S0,
+                              const float* lam0, float* o, float* S_out, float* lam_out, int B,
+                              int T, int H, int dk, int dv, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !a || !w || !r || !o || !S_out || !lam_out) return KDN_ERR_INVALID_ARG;
+  if (in_dtype != KDN_F32 && in_dtype != KDN_BF16) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, dk, dv)) return KDN_ERR_INVALID_ARG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(a) || !al16(w) || !al16(r) || !al16(o) ||
+      !al16(S_out) || !al16(lam_out) || !al16_or_null(S0) || !al16_or_null(lam0))
+    return KDN_ERR_INVALID_ARG;
+  if (!kdn::kla_supported(dk, dv)) return KDN_ERR_UNSUPPORTED;
+  if (!workspace || !al16(workspace) || workspace_bytes < kdn_kla_workspace_size(B, T, H, dk, dv))
+    return KDN_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  if (!kdn::kla_engine_supported(in_dtype, dk, dv, T)) {
+    if (cudaMemsetAsync(workspace, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
+    return kdn::kla_launch(in_dtype, q, k, v, a, w, r, S0, lam0, o, S_out, lam_out, B, T, H, dk,
+                           dv, s);
+  }
+  return kdn::kla_engine_launch(q, k, v, a, w, r, S0, lam0, o, S_out, lam_out, B, T, H, workspace,
+                                s);
 }
 
 size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,

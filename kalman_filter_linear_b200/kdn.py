@@ -82,6 +82,11 @@ def lib():
         [_f32, _vp, _sz, _vp]
     L.kdn_kla_forward.restype = _i32
     L.kdn_kla_forward.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + [_vp]
+    L.kdn_kla_workspace_size.restype = _sz
+    L.kdn_kla_workspace_size.argtypes = [_i32] * 5
+    L.kdn_kla_forward_ws.restype = _i32
+    L.kdn_kla_forward_ws.argtypes = [_vp, _vp, _vp, _i32] + [_vp] * 8 + [_i32] * 5 + \
+        [_vp, _sz, _vp]
     L.kdn_read_workspace_status.restype = _i32
     L.kdn_read_workspace_status.argtypes = [_vp, _sz, _vp]
     L.kdn_testing_mobius_scan_unpublished_tile.restype = _i32
@@ -460,10 +465,18 @@ def kdn_backward(variant, q, k, v, a, w, r, dO, S0=None, p0=None, dS_T=None, dp_
     return g
 
 
-def kdn_kla_forward(q, k, v, a, w, r, S0=None, lam0=None, o=None, S_out=None, lam_out=None):
+def kdn_kla_workspace_size(B, T, H, dk, dv):
+    return int(lib().kdn_kla_workspace_size(B, T, H, dk, dv))
+
+
+def kdn_kla_forward(q, k, v, a, w, r, S0=None, lam0=None, o=None, S_out=None, lam_out=None,
+                    workspace=None, recurrent=False):
     """The information-form diagonal filter (KLA): q, k [B,T,H,dk], v [B,T,H,dv],
     a, r [B,T,H], w [B,T,H,dk].  Returns (o [B,T,H,dv], S_T [B,H,dv,dk],
-    lam_T [B,H,dk]) -- lam is the precision."""
+    lam_T [B,H,dk]) -- lam is the precision.  By default this is
+    kdn_kla_forward_ws (the chunked tensor-core engine at dk = dv = 128 with
+    bf16 inputs, the token-recurrent kernel otherwise); recurrent=True calls
+    kdn_kla_forward, the token-recurrent kernel for every shape."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = q.dtype
@@ -484,10 +497,20 @@ def kdn_kla_forward(q, k, v, a, w, r, S0=None, lam0=None, o=None, S_out=None, la
         torch.empty((B, H, dv, dk), dtype=f, device=dev)
     lam_out = _req(lam_out, 'lam_out', f, (B, H, dk)) if lam_out is not None else \
         torch.empty((B, H, dk), dtype=f, device=dev)
-    st = lib().kdn_kla_forward(_ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w), _ptr(r),
-                               _ptr(S0), _ptr(lam0), _ptr(o), _ptr(S_out), _ptr(lam_out), B, T, H,
-                               dk, dv, _stream())
-    _check(st, 'kdn_kla_forward')
+    if recurrent:
+        st = lib().kdn_kla_forward(_ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w),
+                                   _ptr(r), _ptr(S0), _ptr(lam0), _ptr(o), _ptr(S_out),
+                                   _ptr(lam_out), B, T, H, dk, dv, _stream())
+        _check(st, 'kdn_kla_forward')
+        return o, S_out, lam_out
+    need = kdn_kla_workspace_size(B, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib().kdn_kla_forward_ws(_ptr(q), _ptr(k), _ptr(v), _in_dtype(q), _ptr(a), _ptr(w),
+                                  _ptr(r), _ptr(S0), _ptr(lam0), _ptr(o), _ptr(S_out),
+                                  _ptr(lam_out), B, T, H, dk, dv, _ptr(workspace),
+                                  workspace.numel(), _stream())
+    _check(st, 'kdn_kla_forward_ws')
     return o, S_out, lam_out
 
 

@@ -60,6 +60,14 @@ def test_backward_bytes():
         assert bench.backward_bytes(B, T, H, d, variant) == bwd, variant
 
 
+def test_kla_engine_flops():
+    # per 64-token chunk and head: 52 MMAs of 128x64x16 and 8 of 128x128x16
+    per = 52 * 2 * 128 * 64 * 16 + 8 * 2 * 128 * 128 * 16
+    assert bench.kla_engine_flops(1, 64, 1) == per
+    assert bench.kla_engine_flops(8, 4096, 16) == 8 * 16 * 64 * per
+    assert bench.kla_engine_flops(1, 65, 2) == 2 * 2 * per
+
+
 def test_fp32_peak_is_the_unit_count_times_the_clock():
     assert abs(bench.FP32_PEAK_TFLOPS - 148 * 128 * 2 * 1.965e9 / 1e12) < 1e-9
 

@@ -20,10 +20,12 @@ KLA_TOL = 1e-4
 
 
 def _run(x, S0=None, lam0=None):
+    """kdn_kla_forward: the token-recurrent kernel (the chunked engine has its
+    own tests in test_gpu_kla_engine.py)."""
     xd = {k: v.cuda() for k, v in x.items()}
     return kdn.kdn_kla_forward(xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'],
                                None if S0 is None else S0.cuda(),
-                               None if lam0 is None else lam0.cuda())
+                               None if lam0 is None else lam0.cuda(), recurrent=True)
 
 
 @pytest.mark.parametrize("dk,dv,dtype", [(128, 128, 'bf16'), (64, 64, 'f32'), (32, 40, 'bf16'),
@@ -57,7 +59,7 @@ def test_kla_defaults_and_in_place():
     S = torch.zeros(B, H, d, d, device='cuda')
     lam = torch.ones(B, H, d, device='cuda')
     o2, _, _ = kdn.kdn_kla_forward(xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'], S, lam,
-                                   S_out=S, lam_out=lam)
+                                   S_out=S, lam_out=lam, recurrent=True)
     assert torch.equal(o1, o2) and torch.equal(S1, S) and torch.equal(l1, lam)
 
 

@@ -30,7 +30,7 @@
 // Range.  U~ = U / G grows as the forget gates multiply down.  A piece keeps
 // every G_t >= 2^-100, so U~ <= 2^100 |u| and Q~ >= 2^-100 |q| stay normal
 // numbers and S + V^T U~ stays far below the fp32 limit.  A chunk is one
-// piece when its gates allow it (the check runs on every 16 tokens); else it
+// piece when its gates allow it (checked once per chunk: G only falls); else it
 // is cut where G would cross the bound, down to single tokens.  A single
 // token with f below the bound is scaled by the bound instead: its own term
 // A_tt = q.u does not depend on the scale, and the inter-piece terms then
@@ -207,6 +207,8 @@ __global__ void __launch_bounds__(kKThreads, 1)
 kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mv,
                   const float* __restrict__ A_in, const float* __restrict__ R_in,
+                  const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ Kg,
+                  const float* __restrict__ Wg,
                   const float* S0, const float* L0, float* __restrict__ O, float* S_out,
                   float* L_out, int T, int H, uint32_t* err) {
   extern __shared__ uint8_t ksm_raw[];
@@ -368,9 +370,9 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       acquire_set(p);
       if (bad) break;
       uint8_t* st = set_ptr(p);
-      int start = 0;           // first row of the open piece
       bool first = true;       // the open piece is the chunk's first
       float G = 1.f;           // prod of f over the open piece
+      const float xc = x, yc = y;  // for the slow path
       for (int j = 0; kKQ * j < n; ++j, ++qi) {
         const int nq = min(kKQ, n - kKQ * j);
         const int stage = qi % kKStages;
@@ -378,7 +380,6 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         const uint8_t* sg = sm + KP::OFF_STG + stage * KP::STG;
         const float* ar = reinterpret_cast<const float*>(sg + KP::STG_AR);
 
-        const float xq = x, yq = y, Gq = G;  // for the slow path
         const __nv_bfloat16* sq = reinterpret_cast<const __nv_bfloat16*>(sg + KP::STG_Q) + i;
         const __nv_bfloat16* sk = reinterpret_cast<const __nv_bfloat16*>(sg + KP::STG_K) + i;
         const float* sw = reinterpret_cast<const float*>(sg + KP::STG_W) + i;
@@ -426,43 +427,46 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
             write_row(st, kKQ * j + tt, __bfloat162float(sq[tt * 128]) * G, u * rcp_fast(G));
           }
         }
-        if (!prep_all(G >= kRangeFloor)) {
-          // cut the quarter's tokens into pieces that keep G >= 2^-100: run the
-          // quarter again from its start, one vote per token
-          x = xq;
-          y = yq;
-          G = Gq;
-          for (int tt = 0; tt < nq; ++tt) {
-            const int t = kKQ * j + tt;
-            float f, u;
-            kla_step(ar[tt], ar[16 + tt], ar[32 + tt], __bfloat162float(sk[tt * 128]),
-                     sw[tt * 128], x, y, f, u);
-            if ((tt & 3) == 3) kla_rescale(x, y);
-            float Gt = G * f;
-            if (!prep_all(Gt >= kRangeFloor)) {
-              if (t > start) {
-                zero_rows(st, t, kKC);
-                close_piece(c, G, first ? PF_FIRST : 0u);
-                first = false;
-                acquire_set(p);
-                if (bad) break;
-                st = set_ptr(p);
-                zero_rows(st, 0, t);
-              }
-              start = t;
-              Gt = fmaxf(f, kRangeFloor);
-            }
-            G = Gt;
-            write_row(st, t, __bfloat162float(sq[tt * 128]) * G, u * rcp_fast(G));
-          }
-          if (bad) break;
-        }
-        // every read of this stage is done (the vote, or the slow path's last
-        // one, follows them): hand it back to the loader
+        // this warp's reads of the stage are done: hand it back to the loader
         __syncwarp();
         if ((i & 31) == 0) mbar_arrive(&bars[B_STG_EMPTY + stage]);
       }
       if (bad) break;
+      // G only falls, so its value at the chunk's end bounds every token's
+      if (!prep_all(G >= kRangeFloor)) {
+        // cut the chunk into pieces that keep G >= 2^-100: run it again from
+        // its start, one vote per token, with its inputs read from global
+        // memory (the stages have gone back to the loader)
+        x = xc;
+        y = yc;
+        G = 1.f;
+        int start = 0;  // first row of the open piece
+        for (int t = 0; t < n; ++t) {
+          const size_t tok = tok_index(kKC * c + t);
+          const float a = A_in[tok], r = R_in[tok];
+          float f, u;
+          kla_step(a * a, a * r, r, __bfloat162float(Kg[tok * 128 + i]), Wg[tok * 128 + i], x,
+                   y, f, u);
+          if ((t & 3) == 3) kla_rescale(x, y);
+          float Gt = G * f;
+          if (!prep_all(Gt >= kRangeFloor)) {
+            if (t > start) {
+              zero_rows(st, t, kKC);
+              close_piece(c, G, first ? PF_FIRST : 0u);
+              first = false;
+              acquire_set(p);
+              if (bad) break;
+              st = set_ptr(p);
+              zero_rows(st, 0, t);
+            }
+            start = t;
+            Gt = fmaxf(f, kRangeFloor);
+          }
+          G = Gt;
+          write_row(st, t, __bfloat162float(Qg[tok * 128 + i]) * G, u * rcp_fast(G));
+        }
+        if (bad) break;
+      }
       if (n < kKC) zero_rows(st, n, kKC);
       close_piece(c, G, (first ? PF_FIRST : 0u) | PF_LAST_OF_CHUNK |
                             (c == nchunks - 1 ? PF_LAST : 0u));
@@ -787,7 +791,9 @@ kdn_status kla_engine_launch(const void* q, const void* k, const void* v, const 
   }
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KDN_ERR_CUDA;
   kla_engine_kernel<<<(unsigned)(B * H), kKThreads, KP::SMEM, s>>>(
-      mq, mk, mw, mv, a, r, S0, L0, o, S_out, L_out, T, H, static_cast<uint32_t*>(ws));
+      mq, mk, mw, mv, a, r, static_cast<const __nv_bfloat16*>(q),
+      static_cast<const __nv_bfloat16*>(k), w, S0, L0, o, S_out, L_out, T, H,
+      static_cast<uint32_t*>(ws));
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 

@@ -267,8 +267,7 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
   using P = Plan<DIAG, NV>;
   constexpr int HC = P::HC, QC = P::QC, NVB = NV / 64;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nvblk = dv / NV;
   const int bh = blockIdx.x / nvblk, vblk = blockIdx.x % nvblk;
@@ -1189,8 +1188,7 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
   using P = WsPlan<DIAG>;
   constexpr int DV = 128;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023u));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // packed sequences may be taken longest first: CTA i runs sequence order[i / H]
   const int bh = PACKED && order ? order[blockIdx.x / H] * H + (int)(blockIdx.x % H)

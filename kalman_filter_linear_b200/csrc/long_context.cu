@@ -299,8 +299,7 @@ correct_outputs_kernel(const __grid_constant__ CUtensorMap tm_s,
                        const __grid_constant__ CUtensorMap tm_of, float* __restrict__ O, int H,
                        int L, int ntile, uint32_t* __restrict__ err) {
   extern __shared__ uint8_t corr_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(corr_raw) + 1023u) & ~uintptr_t(1023u));
+  uint8_t* smem = corr_raw + ((1024u - (smem_u32(corr_raw) & 1023u)) & 1023u);
   uint8_t* sA = smem;                    // S_start [4 kb][128 v][32 k]
   uint8_t* sB = smem + kOperandBytes;    // o_F tile [4 kb][128 t][32 k]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + 2 * kOperandBytes);

@@ -78,22 +78,29 @@ __device__ __forceinline__ M2 step_map(float a, float w, float r, float c) {
 }
 
 // Diagonal variant: lanes (b, h, i) for i in a group of 4 dimensions, block
-// j of kBlock tokens.  Threads of a warp take consecutive groups, so every
-// token's w (16 bytes) and k (8 bytes) reads are coalesced; the four chains
-// are independent.
+// j of kBlock tokens, composed by kSub threads (consecutive lanes) of
+// kBlock / kSub tokens each and joined by an ordered product over those lanes.
+// A warp takes 8 consecutive groups (32 dimensions of one head) times kSub
+// sub-blocks, so each token's w (16 bytes) and k (8 bytes) reads are 128- and
+// 64-byte runs; the four chains of a thread are independent.
+constexpr int kSub = 4;
 __global__ void __launch_bounds__(256)
 block_maps_diag_kernel(const __nv_bfloat16* __restrict__ K, const float* __restrict__ A,
                        const float* __restrict__ W, const float* __restrict__ R, int B, int T,
                        int H, int nblk, float4* __restrict__ prod) {
   const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t groups = (int64_t)B * H * (kD / 4);
-  if (gid >= groups * nblk) return;
-  const int j = (int)(gid / groups);
-  const int64_t grp = gid % groups;
+  // (the thread count is a multiple of 128, so whole warps leave together)
+  if (gid >= groups * nblk * kSub) return;
+  const int sub = (int)(gid % kSub);
+  const int64_t rest = gid / kSub;
+  const int j = (int)(rest / groups);
+  const int64_t grp = rest % groups;
   const int i0 = (int)(grp % (kD / 4)) * 4;
   const int h = (int)((grp / (kD / 4)) % H);
   const int b = (int)(grp / ((int64_t)(kD / 4) * H));
-  const int t0 = j * kBlock, t1 = min(T, t0 + kBlock);
+  const int t0 = min(T, j * kBlock + sub * (kBlock / kSub));
+  const int t1 = min(T, t0 + kBlock / kSub);
   M2 P[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) P[e] = {1.f, 0.f, 0.f, 1.f};
@@ -112,11 +119,27 @@ block_maps_diag_kernel(const __nv_bfloat16* __restrict__ K, const float* __restr
       if ((t & 3) == 3) P[e] = renorm(P[e]);
     }
   }
-  const int64_t lane0 = ((int64_t)b * H + h) * kD + i0;
+  // ordered product over the kSub lanes: lane sub's tokens follow lane sub - 1's
+  const int l = threadIdx.x & 31;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const M2 Q = renorm(P[e]);
-    prod[(lane0 + e) * nblk + j] = make_float4(Q.a, Q.b, Q.c, Q.d);
+    M2 Q = renorm(P[e]);
+#pragma unroll
+    for (int d = 1; d < kSub; d <<= 1) {
+      M2 o;
+      o.a = __shfl_down_sync(0xffffffffu, Q.a, d);
+      o.b = __shfl_down_sync(0xffffffffu, Q.b, d);
+      o.c = __shfl_down_sync(0xffffffffu, Q.c, d);
+      o.d = __shfl_down_sync(0xffffffffu, Q.d, d);
+      if ((l & (2 * d - 1)) == 0) Q = renorm(mul(o, Q));
+    }
+    P[e] = Q;
+  }
+  if (sub == 0) {
+    const int64_t lane0 = ((int64_t)b * H + h) * kD + i0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      prod[(lane0 + e) * nblk + j] = make_float4(P[e].a, P[e].b, P[e].c, P[e].d);
   }
 }
 
@@ -504,7 +527,7 @@ kdn_status segmented_forward(bool diag, const void* q, const void* k, const void
   // 1. variances at the segment starts
   const int64_t lanes = (int64_t)B * H * dim;
   if (diag) {
-    const int64_t n = lanes / 4 * nblk;
+    const int64_t n = lanes / 4 * nblk * kSub;
     block_maps_diag_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(k), a, w, r, B, T, H, nblk, prod);
   } else {

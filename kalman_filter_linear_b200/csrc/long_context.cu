@@ -300,10 +300,10 @@ __global__ void or_error_words(uint32_t* dst, const uint32_t* a, const uint32_t*
 // cores in tf32 (both operands fp32 in shared memory, K-major, 128-byte
 // swizzle; the correction's relative error is about 2^-10 of its size, well
 // inside the output bound), with the fp32 accumulator in TMEM.  One CTA of
-// four warps per (segment, head, 8 or 4 tiles of 128 tokens): S_start comes in
-// once, each token tile by TMA, 16 MMAs of K = 8, then each thread (one value
-// row v) adds its TMEM row to o in place, 32 tokens at a time, coalesced
-// over v.
+// eight warps per (segment, head, 8 or 4 tiles of 128 tokens): S_start comes
+// in once, each token tile by TMA, 16 MMAs of K = 8, then each thread (one
+// value row v, half of the tile's tokens; two warps per TMEM lane quarter)
+// adds its TMEM row to o in place, 32 tokens at a time, coalesced over v.
 constexpr int kCorrTiles = 8;  // token tiles of 128 per CTA (4 when 8 does not divide a segment)
 constexpr uint32_t kOperandBytes = 128u * 128u * 4u;  // 64 KB, [4 kb][128 rows][32 k]
 constexpr uint32_t kCorrSmem = 2 * kOperandBytes + 1024 + 64;
@@ -317,7 +317,7 @@ __device__ __forceinline__ void umma_tf32_ss(uint32_t tmem_d, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
 correct_outputs_kernel(const __grid_constant__ CUtensorMap tm_s,
                        const __grid_constant__ CUtensorMap tm_of, float* __restrict__ O, int H,
                        int L, int ntile, uint32_t* __restrict__ err) {
@@ -393,16 +393,18 @@ correct_outputs_kernel(const __grid_constant__ CUtensorMap tm_s,
     // the tile's operand has been read: copy the next one during the epilogue
     if (tid == 0 && i + 1 < ntile) load_b(tile0 + i + 1);
     const int t0 = 128 * (tile0 + i);
-    float* orow = O + (((size_t)bs * L + t0) * H + h) * 128 + tid;  // v = tid
+    // warp w reads TMEM lanes [32 (w % 4), + 32) (v) and column blocks 2 (w / 4), + 1
+    const int v = 32 * (warp & 3) + (tid & 31);
+    float* orow = O + (((size_t)bs * L + t0) * H + h) * 128 + v;
     const size_t tstride = (size_t)H * 128;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 2 * (warp >> 2); c < 2 * (warp >> 2) + 2; ++c) {
       // the 32 o_E values first (all loads in flight at once), then the
       // TMEM columns, then the sums
       float e[32], d[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) e[j] = __ldcs(orow + (size_t)(32 * c + j) * tstride);
-      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * c, d);
+      tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * c, d);
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 32; ++j) __stcs(orow + (size_t)(32 * c + j) * tstride, e[j] + d[j]);
@@ -573,7 +575,7 @@ kdn_status segmented_forward(bool diag, const void* q, const void* k, const void
   // (every segment: the first of each batch entry adds S0 o_F, zero without S0)
   const int ntile = (Ls / 128) % kCorrTiles == 0 ? kCorrTiles : 4;
   const int groups = (Ls / 128) / ntile;
-  correct_outputs_kernel<<<(unsigned)(Bs * H * groups), 128, kCorrSmem, st>>>(
+  correct_outputs_kernel<<<(unsigned)(Bs * H * groups), 256, kCorrSmem, st>>>(
       tm_s, tm_of, o, H, Ls, ntile, reinterpret_cast<uint32_t*>(base + L.err_g));
   if (cudaGetLastError() != cudaSuccess) return KDN_ERR_CUDA;
 

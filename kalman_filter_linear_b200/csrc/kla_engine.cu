@@ -149,7 +149,9 @@ __device__ __forceinline__ void prep_sync() {
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
   const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  // both remainders in one packed FMA (each rounded as the scalar subtraction)
+  const float2 r = __ffma2_rn(hf, make_float2(-1.f, -1.f), make_float2(x0, x1));
+  const __nv_bfloat162 l = __floats2bfloat162_rn(r.x, r.y);
   hi = *reinterpret_cast<const uint32_t*>(&h);
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
@@ -488,7 +490,9 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
           const float4 gl = *reinterpret_cast<const float4*>(GL + 32 * g + j);
-          x[j] *= gl.x; x[j + 1] *= gl.y; x[j + 2] *= gl.z; x[j + 3] *= gl.w;
+          const float2 p0 = __fmul2_rn(make_float2(x[j], x[j + 1]), make_float2(gl.x, gl.y));
+          const float2 p1 = __fmul2_rn(make_float2(x[j + 2], x[j + 3]), make_float2(gl.z, gl.w));
+          x[j] = p0.x; x[j + 1] = p0.y; x[j + 2] = p1.x; x[j + 3] = p1.y;
         }
         if (flags & PF_LAST) {
           float* dst = S_out + ((size_t)bh * 128 + v) * 128 + 32 * g;

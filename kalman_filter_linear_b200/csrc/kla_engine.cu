@@ -192,19 +192,19 @@ __device__ __forceinline__ void kla_rescale(float& x, float& y) {
 __device__ __forceinline__ void st_bf16(uint8_t* p, __nv_bfloat16 x) {
   asm volatile("st.shared.b16 [%0], %1;" ::"r"(smem_u32(p)), "h"(__bfloat16_as_ushort(x)));
 }
-// One token row of a set: Q~ hi at qa, Q~ lo 64 rows (8 KB) below, U~ hi at
-// ua, U~ lo in the next tile (16 KB on).
-__device__ __forceinline__ void st_row4(uint32_t qa, uint32_t ua, __nv_bfloat16 qh,
-                                        __nv_bfloat16 ql, __nv_bfloat16 uh, __nv_bfloat16 ul) {
+// One token row of a set from packed pairs: hi = (Q~ hi, U~ hi), lo = (Q~ lo,
+// U~ lo), each with Q~ in the low half.
+__device__ __forceinline__ void st_row4p(uint32_t qa, uint32_t ua, uint32_t hi, uint32_t lo) {
   asm volatile(
-      "st.shared.b16 [%0], %2;\n\t"
-      "st.shared.b16 [%0+8192], %3;\n\t"
-      "st.shared.b16 [%1], %4;\n\t"
-      "st.shared.b16 [%1+16384], %5;" ::"r"(qa),
-      "r"(ua), "h"(__bfloat16_as_ushort(qh)), "h"(__bfloat16_as_ushort(ql)),
-      "h"(__bfloat16_as_ushort(uh)), "h"(__bfloat16_as_ushort(ul)));
+      "{\n\t.reg .b16 qh, uh, ql, ul;\n\t"
+      "mov.b32 {qh, uh}, %2;\n\t"
+      "mov.b32 {ql, ul}, %3;\n\t"
+      "st.shared.b16 [%0], qh;\n\t"
+      "st.shared.b16 [%0+8192], ql;\n\t"
+      "st.shared.b16 [%1], uh;\n\t"
+      "st.shared.b16 [%1+16384], ul;\n\t}" ::"r"(qa),
+      "r"(ua), "r"(hi), "r"(lo));
 }
-
 __global__ void __launch_bounds__(kKThreads, 1)
 kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mv,
@@ -331,10 +331,9 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     // is the row's offset t * 128 + swizzled column
     const uint32_t qcol = KP::QS + col_half * 16384u, ucol = KP::UH + col_half * 8192u;
     auto write_row_at = [&](uint8_t* st, uint32_t off, float qt, float ut) {
-      __nv_bfloat16 qh, ql, uh, ul;
-      split_bf16(qt, qh, ql);
-      split_bf16(ut, uh, ul);
-      st_row4(smem_u32(st) + qcol + off, smem_u32(st) + ucol + off, qh, ql, uh, ul);
+      uint32_t hi, lo;
+      split2(qt, ut, hi, lo);
+      st_row4p(smem_u32(st) + qcol + off, smem_u32(st) + ucol + off, hi, lo);
     };
     auto write_row = [&](uint8_t* st, int t, float qt, float ut) {
       write_row_at(st, sw128_offset((uint32_t)t, col), qt, ut);

@@ -36,7 +36,7 @@
 // A_tt = q.u does not depend on the scale, and the inter-piece terms then
 // differ from the exact ones by at most 2^-100 of S_start.
 //
-// Roles (13 warps, one CTA per (b, h)):
+// Roles (14 warps, one CTA per (b, h)):
 //  - warps 0-3, prep: thread i runs key dimension i's variance recursion in
 //    projective form (p = x / y; no division on the token-to-token chain),
 //    forms Q~ and U~ rows (bf16 hi/lo, 128-byte swizzled K-major tiles) into
@@ -205,6 +205,7 @@ __device__ __forceinline__ void st_row4p(uint32_t qa, uint32_t ua, uint32_t hi, 
       "st.shared.b16 [%1+16384], ul;\n\t}" ::"r"(qa),
       "r"(ua), "r"(hi), "r"(lo));
 }
+
 __global__ void __launch_bounds__(kKThreads, 1)
 kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                   const __grid_constant__ CUtensorMap mw, const __grid_constant__ CUtensorMap mv,

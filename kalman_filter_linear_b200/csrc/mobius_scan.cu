@@ -40,6 +40,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kPerThread = 8;
 constexpr int kTile = kThreads * kPerThread;  // 2048 steps
+static_assert(kPerThread % 4 == 0 && kThreads % 32 == 0, "tile shape");
 
 struct Mat2 {
   float a, b, c, d;  // [[a, b], [c, d]]
@@ -240,17 +241,20 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
   }
   if (vec_ok && t0 + kPerThread <= T) {
     float4* l4 = reinterpret_cast<float4*>(lam_out + base + t0);
-    l4[0] = make_float4(out_l[0], out_l[1], out_l[2], out_l[3]);
-    l4[1] = make_float4(out_l[4], out_l[5], out_l[6], out_l[7]);
+#pragma unroll
+    for (int h = 0; h < kPerThread / 4; ++h)
+      l4[h] = make_float4(out_l[4 * h], out_l[4 * h + 1], out_l[4 * h + 2], out_l[4 * h + 3]);
     if (prior_out) {
       float4* p4 = reinterpret_cast<float4*>(prior_out + base + t0);
-      p4[0] = make_float4(out_p[0], out_p[1], out_p[2], out_p[3]);
-      p4[1] = make_float4(out_p[4], out_p[5], out_p[6], out_p[7]);
+#pragma unroll
+      for (int h = 0; h < kPerThread / 4; ++h)
+        p4[h] = make_float4(out_p[4 * h], out_p[4 * h + 1], out_p[4 * h + 2], out_p[4 * h + 3]);
     }
     if (gain_out) {
       float4* g4 = reinterpret_cast<float4*>(gain_out + base + t0);
-      g4[0] = make_float4(out_g[0], out_g[1], out_g[2], out_g[3]);
-      g4[1] = make_float4(out_g[4], out_g[5], out_g[6], out_g[7]);
+#pragma unroll
+      for (int h = 0; h < kPerThread / 4; ++h)
+        g4[h] = make_float4(out_g[4 * h], out_g[4 * h + 1], out_g[4 * h + 2], out_g[4 * h + 3]);
     }
   } else {
 #pragma unroll
@@ -289,7 +293,7 @@ mobius_scan_kernel(const float* __restrict__ A, const float* __restrict__ W,
     const float4* r4 = reinterpret_cast<const float4*>(R + base + t0);
     const float4* n4 = reinterpret_cast<const float4*>(Nsq + base + t0);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kPerThread / 4; ++h) {
       float4 x = __ldg(a4 + h), y = __ldg(w4 + h), z = __ldg(r4 + h), u = __ldg(n4 + h);
       a[4 * h] = x.x; a[4 * h + 1] = x.y; a[4 * h + 2] = x.z; a[4 * h + 3] = x.w;
       w[4 * h] = y.x; w[4 * h + 1] = y.y; w[4 * h + 2] = y.z; w[4 * h + 3] = y.w;
@@ -379,7 +383,7 @@ mobius_scan_persistent(const float* __restrict__ A, const float* __restrict__ W,
     const float* buf = reinterpret_cast<const float*>(s_in);
     float a[kPerThread], w[kPerThread], r[kPerThread], n[kPerThread];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kPerThread / 4; ++h) {
       const float4 x = *reinterpret_cast<const float4*>(buf + 0 * kTile + tid * kPerThread + 4 * h);
       const float4 y = *reinterpret_cast<const float4*>(buf + 1 * kTile + tid * kPerThread + 4 * h);
       const float4 z = *reinterpret_cast<const float4*>(buf + 2 * kTile + tid * kPerThread + 4 * h);

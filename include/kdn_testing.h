@@ -48,6 +48,23 @@ kdn_status kdn_testing_forward_skip_v_copy(kdn_variant variant, const void* q,
                                            size_t workspace_bytes,
                                            void* stream);
 
+/* kdn_kla_forward_ws on the chunked KLA engine (dk = dv = 128, bf16 q/k/v,
+ * S0 = 0, lam0 = 1), except that the copy of chunk `skip_chunk`'s V tile is
+ * never issued.  The issuer's bounded wait for it gives up (after about one
+ * second) and records KDN_ERR_TIMEOUT in the workspace error word; every
+ * role of every CTA then leaves through its bounded waits, waits (bounded)
+ * for its copies and MMAs in flight, frees its TMEM and returns.  The call
+ * returns normally; kdn_read_workspace_status() then reports
+ * KDN_ERR_TIMEOUT.  Outputs are not meaningful.
+ * 1 <= skip_chunk < ceil(T / 64). */
+kdn_status kdn_testing_kla_skip_v_copy(const void* q, const void* k,
+                                       const void* v, const float* a,
+                                       const float* w, const float* r,
+                                       float* o, float* S_out, float* lam_out,
+                                       int B, int T, int H, int skip_chunk,
+                                       void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -56,7 +56,7 @@ bool kla_engine_supported(kdn_dtype dt, int dk, int dv, int T);
 kdn_status kla_engine_launch(const void* q, const void* k, const void* v, const float* a,
                              const float* w, const float* r, const float* S0, const float* L0,
                              float* o, float* S_out, float* L_out, int B, int T, int H, void* ws,
-                             cudaStream_t s);
+                             cudaStream_t s, int debug_skip_v);
 kdn_status kla_launch(kdn_dtype dt, const void* q, const void* k, const void* v, const float* a,
                       const float* w, const float* r, const float* S0, const float* L0, float* o,
                       float* S_out, float* L_out, int B, int T, int H, int dk, int dv,
@@ -421,7 +421,22 @@ kdn_status kdn_kla_forward_ws(const void* q, const void* k, const void* v, kdn_d
                            dv, s);
   }
   return kdn::kla_engine_launch(q, k, v, a, w, r, S0, lam0, o, S_out, lam_out, B, T, H, workspace,
-                                s);
+                                s, -1);
+}
+
+kdn_status kdn_testing_kla_skip_v_copy(const void* q, const void* k, const void* v,
+                                       const float* a, const float* w, const float* r, float* o,
+                                       float* S_out, float* lam_out, int B, int T, int H,
+                                       int skip_chunk, void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  if (!q || !k || !v || !a || !w || !r || !o || !S_out || !lam_out) return KDN_ERR_INVALID_ARG;
+  if (!shape_ok(B, T, H, 128, 128)) return KDN_ERR_INVALID_ARG;
+  if (skip_chunk < 1 || skip_chunk >= (T + 63) / 64) return KDN_ERR_INVALID_ARG;
+  if (!workspace || !al16(workspace) ||
+      workspace_bytes < kdn_kla_workspace_size(B, T, H, 128, 128))
+    return KDN_ERR_WORKSPACE;
+  return kdn::kla_engine_launch(q, k, v, a, w, r, nullptr, nullptr, o, S_out, lam_out, B, T, H,
+                                workspace, as_stream(stream), skip_chunk);
 }
 
 size_t kdn_forward_host_workspace_size(kdn_variant variant, int B, int T, int H, int dk, int dv,

@@ -40,7 +40,9 @@
 //  - warps 0-3, prep: thread i runs key dimension i's variance recursion in
 //    projective form (p = x / y; no division on the token-to-token chain),
 //    forms Q~ and U~ rows (bf16 hi/lo, 128-byte swizzled K-major tiles) into
-//    one of two operand sets, and closes pieces.
+//    one of two operand sets, and closes pieces.  Their barrier and range vote
+//    go through an mbarrier with a bounded wait, so no thread can wait for
+//    one that has left on a timeout.
 //  - warps 4-7, state: one TMEM lane quarter each; after MMA-dS they scale S
 //    by G_L and write its bf16 hi/lo split (or, after the last piece, S_T).
 //  - warps 8-11, A and output: after MMA-A they sum the two halves of D_A
@@ -68,7 +70,6 @@ constexpr int kKStages = 3;             // quarter stages
 constexpr int kKWarps = 14;
 constexpr int kKThreads = kKWarps * 32;
 constexpr float kRangeFloor = 7.8886090522101181e-31f;  // 2^-100
-constexpr int kPrepBar = 1;             // named barrier of the prep warps
 
 struct KP {
   // operand set: Qs [2 K halves][128 rows][128 B] | U~ hi [2][64][128 B] | U~ lo
@@ -85,8 +86,9 @@ struct KP {
   static constexpr uint32_t META = 528;
   static constexpr uint32_t OFF_BAR = OFF_META + 4 * META;
   static constexpr uint32_t NBAR = 26;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;     // tmem base, abort flag
-  static constexpr uint32_t TOTAL = OFF_MISC + 16;
+  // tmem base, abort flag, three rotating vote words of the prep barrier
+  static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
+  static constexpr uint32_t TOTAL = OFF_MISC + 32;
   static constexpr uint32_t SMEM = TOTAL + 1024;               // 1024-byte alignment slack
 };
 static_assert(KP::OFF_STG % 1024 == 0 && KP::OFF_A % 1024 == 0, "tile alignment");
@@ -111,6 +113,7 @@ enum : int {
   B_STG = 18,       // [3] quarter stage landed (tx, and the loader's a/r stores)
   B_STG_EMPTY = 21, // [3] the prep is done with a stage (count 4)
   B_FINAL = 24,     // the issuer's last commit
+  B_PREP = 25,      // the prep warps' barrier (count 128)
 };
 static_assert(B_FINAL < (int)KP::NBAR, "barrier count");
 
@@ -123,25 +126,6 @@ __device__ __forceinline__ void tma_load_4d_prefetch(const void* tmap, int c0, i
                    tmap),
                "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                : "memory");
-}
-
-// True on every thread when `ok` holds on all 128 prep threads.
-__device__ __forceinline__ bool prep_all(bool ok) {
-  uint32_t r;
-  __syncwarp();
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)ok), "n"(kPrepBar)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void prep_sync() {
-  __syncwarp();
-  asm volatile("bar.sync %0, 128;" ::"n"(kPrepBar) : "memory");
 }
 
 // (hi, lo) bf16 pairs of two consecutive fp32 values, the lower index in the
@@ -213,7 +197,7 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
                   const __nv_bfloat16* __restrict__ Qg, const __nv_bfloat16* __restrict__ Kg,
                   const float* __restrict__ Wg,
                   const float* S0, const float* L0, float* __restrict__ O, float* S_out,
-                  float* L_out, int T, int H, uint32_t* err) {
+                  float* L_out, int T, int H, uint32_t* err, int debug_skip_v) {
   extern __shared__ uint8_t ksm_raw[];
   // 1024-byte aligned by pointer arithmetic on the shared array, so that every
   // access through `sm` stays a shared-memory access
@@ -258,7 +242,9 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       mbar_init(&bars[B_STG_EMPTY + i], 4);
     }
     mbar_init(&bars[B_FINAL], 1);
+    mbar_init(&bars[B_PREP], 128);
     misc[1] = 0u;
+    misc[2] = misc[3] = misc[4] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     tma_prefetch_desc(&mq);
     tma_prefetch_desc(&mk);
@@ -349,6 +335,26 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         st_bf16(st + KP::UL + col_half * 8192 + sw128_offset((uint32_t)t, col), z);
       }
     };
+    // Barrier of the 128 prep threads with a vote: true when `ok` held on all
+    // of them.  Use k arrives on the mbarrier's phase k and ORs this warp's
+    // failures into vote word k % 3; word k + 2 is cleared after the wait (no
+    // thread can still read it: use k completes only after every thread has
+    // finished use k - 1).  A wait that gives up sets `bad`.
+    volatile uint32_t* vote = misc + 2;
+    int puse = 0;
+    auto prep_vote = [&](bool ok) -> bool {
+      const int k = puse++;
+      if (!__all_sync(0xffffffffu, ok) && (i & 31) == 0) atomicOr((uint32_t*)&vote[k % 3], 1u);
+      __syncwarp();
+      mbar_arrive(&bars[B_PREP]);
+      if (fail(&bars[B_PREP], (uint32_t)(k & 1))) {
+        bad = true;
+        return false;
+      }
+      const bool all = vote[k % 3] == 0u;
+      if (i == 0) vote[(k + 2) % 3] = 0u;
+      return all;
+    };
     // publish piece p: its G_L and flags, then hand the set to the issuer
     auto close_piece = [&](int c, float GL, uint32_t flags) {
       uint8_t* meta = sm + KP::OFF_META + (uint32_t)(p & 3) * KP::META;
@@ -358,7 +364,8 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         reinterpret_cast<uint32_t*>(meta + 512)[1] = flags;
       }
       fence_async_smem();
-      prep_sync();
+      prep_vote(true);
+      if (bad) return;
       if (i == 0) {
         mbar_arrive(&bars[B_OP_FULL + (p & 1)]);
         mbar_arrive(&bars[B_META + (p & 3)]);
@@ -435,7 +442,9 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
       }
       if (bad) break;
       // G only falls, so its value at the chunk's end bounds every token's
-      if (!prep_all(G >= kRangeFloor)) {
+      const bool in_range = prep_vote(G >= kRangeFloor);
+      if (bad) break;
+      if (!in_range) {
         // cut the chunk into pieces that keep G >= 2^-100: run it again from
         // its start, one vote per token, with its inputs read from global
         // memory (the stages have gone back to the loader)
@@ -451,10 +460,13 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
                    y, f, u);
           if ((t & 3) == 3) kla_rescale(x, y);
           float Gt = G * f;
-          if (!prep_all(Gt >= kRangeFloor)) {
+          const bool t_in_range = prep_vote(Gt >= kRangeFloor);
+          if (bad) break;
+          if (!t_in_range) {
             if (t > start) {
               zero_rows(st, t, kKC);
               close_piece(c, G, first ? PF_FIRST : 0u);
+              if (bad) break;
               first = false;
               acquire_set(p);
               if (bad) break;
@@ -573,7 +585,7 @@ kla_engine_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         if (fail(&bars[B_O_FULL + (c & 1)], (uint32_t)((c >> 1) & 1))) break;
         tc_fence_after();
         // every reader of this chunk's V tile is done: copy the next one
-        if (warp == 8 && lane == 0 && c + 1 < nchunks) {
+        if (warp == 8 && lane == 0 && c + 1 < nchunks && c + 1 != debug_skip_v) {
           mbar_expect_tx(&bars[B_V_FULL], 16384);
           tma_load_4d(sm + KP::OFF_V, &mv, &bars[B_V_FULL], 0, h, kKC * (c + 1), b);
           tma_load_4d(sm + KP::OFF_V + 8192, &mv, &bars[B_V_FULL], 64, h, kKC * (c + 1), b);
@@ -779,7 +791,7 @@ bool kla_engine_supported(kdn_dtype dt, int dk, int dv, int T) {
 kdn_status kla_engine_launch(const void* q, const void* k, const void* v, const float* a,
                              const float* w, const float* r, const float* S0, const float* L0,
                              float* o, float* S_out, float* L_out, int B, int T, int H, void* ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, int debug_skip_v) {
   CUtensorMap mq, mk, mw, mv;
   if (!kla_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, T, H, 128, kKQ, false) ||
       !kla_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, T, H, 128, kKQ, false) ||
@@ -797,7 +809,7 @@ kdn_status kla_engine_launch(const void* q, const void* k, const void* v, const 
   kla_engine_kernel<<<(unsigned)(B * H), kKThreads, KP::SMEM, s>>>(
       mq, mk, mw, mv, a, r, static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), w, S0, L0, o, S_out, L_out, T, H,
-      static_cast<uint32_t*>(ws));
+      static_cast<uint32_t*>(ws), debug_skip_v);
   return cudaGetLastError() == cudaSuccess ? KDN_OK : KDN_ERR_CUDA;
 }
 

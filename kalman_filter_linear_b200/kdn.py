@@ -90,6 +90,8 @@ def lib():
     L.kdn_read_workspace_status.restype = _i32
     L.kdn_read_workspace_status.argtypes = [_vp, _sz, _vp]
     L.kdn_testing_mobius_scan_unpublished_tile.restype = _i32
+    L.kdn_testing_kla_skip_v_copy.restype = _i32
+    L.kdn_testing_kla_skip_v_copy.argtypes = [_vp] * 9 + [_i32] * 4 + [_vp, _sz, _vp]
     L.kdn_testing_forward_skip_v_copy.restype = _i32
     L.kdn_testing_forward_skip_v_copy.argtypes = [_i32] + [_vp] * 9 + [_i32] * 4 + [_vp, _sz, _vp]
     L.kdn_testing_mobius_scan_unpublished_tile.argtypes = [_vp] * 5 + [_f32, _vp, _i64, _i64,
@@ -553,3 +555,25 @@ def kdn_testing_forward_skip_v_copy(variant, q, k, v, a, w, r, skip_chunk, works
                                                workspace.numel(), _stream())
     _check(st, 'kdn_testing_forward_skip_v_copy')
     return o, S, p
+
+
+def kdn_testing_kla_skip_v_copy(q, k, v, a, w, r, skip_chunk, workspace):
+    """Fault-injection hook: the KLA engine (d = 128, bf16) with one V copy
+    left out, so a bounded wait gives up.  Returns (o, S_T, lam_T); the status
+    is in the workspace."""
+    B, T, H, d = q.shape
+    for t, n in ((q, 'q'), (k, 'k'), (v, 'v')):
+        _req(t, n, torch.bfloat16, (B, T, H, d))
+    f = torch.float32
+    _req(a, 'a', f, (B, T, H))
+    _req(r, 'r', f, (B, T, H))
+    _req(w, 'w', f, (B, T, H, d))
+    _req(workspace, 'workspace', torch.uint8)
+    o = torch.empty((B, T, H, d), dtype=f, device=q.device)
+    S = torch.empty((B, H, d, d), dtype=f, device=q.device)
+    lam = torch.empty((B, H, d), dtype=f, device=q.device)
+    st = lib().kdn_testing_kla_skip_v_copy(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(w), _ptr(r),
+                                           _ptr(o), _ptr(S), _ptr(lam), B, T, H, int(skip_chunk),
+                                           _ptr(workspace), workspace.numel(), _stream())
+    _check(st, 'kdn_testing_kla_skip_v_copy')
+    return o, S, lam

@@ -146,3 +146,18 @@ def test_engine_full_width_matches_recurrent_kernel():
         o_r, S_r, lam_r = _oracle(sl)
         assert rel_maxabs(o[b, :, h], o_r[0, :, 0]) <= O_TOL, (b, h)
         assert rel_maxabs(S[b, h], S_r[0, 0]) <= S_TOL, (b, h)
+
+
+def test_engine_bounded_wait_reports_timeout_and_context_survives():
+    """One V copy is left out: the issuer's bounded wait gives up, every role
+    of every CTA leaves through its bounded waits, the workspace reports
+    KDN_ERR_TIMEOUT, and the next call on the same context is correct."""
+    B, T, H = 1, 256, 2
+    x = synth.layer_inputs(B, T, H, D, D, 'diag', seed=350, dtype='bf16')
+    xd = {k: v.cuda() for k, v in x.items()}
+    ws = torch.zeros(kdn.kdn_kla_workspace_size(B, T, H, D, D), dtype=torch.uint8, device='cuda')
+    kdn.kdn_testing_kla_skip_v_copy(xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'], 2, ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_ERR_TIMEOUT
+    got = kdn.kdn_kla_forward(xd['q'], xd['k'], xd['v'], xd['a'], xd['w'], xd['r'], workspace=ws)
+    assert kdn.kdn_read_workspace_status(ws) == kdn.KDN_OK
+    _check(got, _oracle(x))

@@ -960,7 +960,9 @@ chunk_engine_kernel(const __grid_constant__ CUtensorMap tm_q,
 // Warps 8-15 (prep) run the part that depends only on the chunk's inputs, one
 // chunk ahead: the D1 epilogue (A, and P once MMA4 of the previous chunk has
 // released its buffer) on all eight warps, then T = (I + A)^-1 on warps 8-11
-// while warps 12-15 prepare the next chunk:
+// while warps 12-15 prepare the next chunk (isotropic: the solve's last two
+// steps, the 32x32 block below the diagonal, on all eight warps, as the next
+// chunk's scalars take warps 12-15 only part of the solve):
 //   isotropic  ||k||^2, decay prefix and the variance scan; MMA1 of the next
 //              chunk is issued as soon as D1 is read.
 //   diagonal   decay prefix and the per-dimension variance (one thread per
@@ -1079,6 +1081,38 @@ __device__ __forceinline__ void warp_put16(const float (&acc)[3][2][4], float s,
     C(g, 8 * nt + 2 * q, v[0], v[1]);
     C(g + 8, 8 * nt + 2 * q, v[2], v[3]);
   }
+}
+
+// The same product for n-tile nt alone (B's columns [8 nt, 8 nt + 8)), with
+// the same fragments, accumulation order and final sum, so that two warps
+// taking one n-tile each give what one warp taking both gives.
+template <class FA, class FB>
+__device__ __forceinline__ void warp_mm16n(float (&acc)[3][4], FA A, FB B, int nt, int lane) {
+  const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < 2; ++ks) {
+    uint32_t ah[4], al[4];
+    split_tf32(A(g, 8 * ks + q), ah[0], al[0]);
+    split_tf32(A(g + 8, 8 * ks + q), ah[1], al[1]);
+    split_tf32(A(g, 8 * ks + q + 4), ah[2], al[2]);
+    split_tf32(A(g + 8, 8 * ks + q + 4), ah[3], al[3]);
+    uint32_t bh[2], bl[2];
+    split_tf32(B(8 * ks + q, 8 * nt + g), bh[0], bl[0]);
+    split_tf32(B(8 * ks + q + 4, 8 * nt + g), bh[1], bl[1]);
+    mma_tf32_16x8x8(acc[0], ah, bh);
+    mma_tf32_16x8x8(acc[1], ah, bl);
+    mma_tf32_16x8x8(acc[2], al, bh);
+  }
+}
+template <class FC>
+__device__ __forceinline__ void warp_put16n(const float (&acc)[3][4], float s, FC C, int nt,
+                                            int lane) {
+  const int g = lane >> 2, q = lane & 3;
+  float v[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = s * (acc[2][e] + acc[1][e] + acc[0][e]);
+  C(g, 8 * nt + 2 * q, v[0], v[1]);
+  C(g + 8, 8 * nt + 2 * q, v[2], v[3]);
 }
 
 constexpr int kChainBar = 3, kPrepBar = 4, kPhase1Bar = 5, kGroup = 256;
@@ -1991,6 +2025,24 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         else issue_mma1(c + 1);
       }
 
+      // AT and T accessors: A's blocks below the diagonal, T's diagonal blocks,
+      // T's blocks below the diagonal (stored transposed above it)
+      auto Ael = [&](int i, int l, int r, int k) { return AT[(16 * i + r) * kLd + 16 * l + k]; };
+      auto Tdg = [&](int i, int r, int k) { return AT[(16 * i + r) * kLd + 16 * i + k]; };
+      auto Tlo = [&](int i, int bb, int r, int k) { return AT[(16 * bb + k) * kLd + 16 * i + r]; };
+      auto Tset = [&](int i, int bb, int r, int k, float v0, float v1) {
+        AT[(16 * bb + k) * kLd + 16 * i + r] = v0;
+        AT[(16 * bb + k + 1) * kLd + 16 * i + r] = v1;
+      };
+      auto Top = [&](int i, int bb, int r, int k, float v0, float v1) {
+        // T[16 i + r][16 bb + k, +1] as bf16 hi/lo pairs
+        uint32_t hi, lo;
+        split_pack2(v0, v1, hi, lo);
+        const uint32_t row = (uint32_t)(16 * i + r), col = (uint32_t)(16 * bb + k);
+        const uint32_t off = chunk_off(row, col >> 3) + ((col & 7u) << 1);
+        *reinterpret_cast<uint32_t*>(sT + off) = hi;
+        *reinterpret_cast<uint32_t*>(sT + 8192 + off) = lo;
+      };
       if (pw < 4) {
         // ---- T = (I + A)^-1 (warps 8-11) into AT and as the bf16 hi/lo B
         // operand [t][j] of MMA3, once MMA3 of the previous chunk released it.
@@ -2014,22 +2066,6 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int i = 0; i < 16; ++i) AT[(16 * blk + i) * kLd + 16 * blk + cc] = x[i];
         }
         named_bar<kTeamA, 128>();
-        auto Ael = [&](int i, int l, int r, int k) { return AT[(16 * i + r) * kLd + 16 * l + k]; };
-        auto Tdg = [&](int i, int r, int k) { return AT[(16 * i + r) * kLd + 16 * i + k]; };
-        auto Tlo = [&](int i, int bb, int r, int k) { return AT[(16 * bb + k) * kLd + 16 * i + r]; };
-        auto Tset = [&](int i, int bb, int r, int k, float v0, float v1) {
-          AT[(16 * bb + k) * kLd + 16 * i + r] = v0;
-          AT[(16 * bb + k + 1) * kLd + 16 * i + r] = v1;
-        };
-        auto Top = [&](int i, int bb, int r, int k, float v0, float v1) {
-          // T[16 i + r][16 bb + k, +1] as bf16 hi/lo pairs
-          uint32_t hi, lo;
-          split_pack2(v0, v1, hi, lo);
-          const uint32_t row = (uint32_t)(16 * i + r), col = (uint32_t)(16 * bb + k);
-          const uint32_t off = chunk_off(row, col >> 3) + ((col & 7u) << 1);
-          *reinterpret_cast<uint32_t*>(sT + off) = hi;
-          *reinterpret_cast<uint32_t*>(sT + 8192 + off) = lo;
-        };
         // T_{b+1,b} = -T_{b+1,b+1} A_{b+1,b} T_bb inside each 32-block
         // (b = 0, 2) on the 128 threads: 64 per product, 2x2 outputs each
         {
@@ -2081,42 +2117,45 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         named_bar<kTeamA, 128>();
         // the 32x32 block below the diagonal: T^(10) = -T^(1) (A^(10) T^(0)),
-        // first X2 = A^(10) T^(0), one 16x16 block per warp
-        const int i2 = 2 + (pw >> 1), b2 = pw & 1;
-        {
-          float acc[3][2][4] = {};
-          if (b2 == 0) {
-            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 0, r, k); },
-                      [&](int k, int n) { return Tdg(0, k, n); }, lane);
-            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
-                      [&](int k, int n) { return Tlo(1, 0, k, n); }, lane);
-          } else {
-            warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
-                      [&](int k, int n) { return Tdg(1, k, n); }, lane);
+        // first X2 = A^(10) T^(0), one 16x16 block per warp (isotropic: on
+        // all eight prep warps, below)
+        if constexpr (DIAG) {
+          const int i2 = 2 + (pw >> 1), b2 = pw & 1;
+          {
+            float acc[3][2][4] = {};
+            if (b2 == 0) {
+              warp_mm16(acc, [&](int r, int k) { return Ael(i2, 0, r, k); },
+                        [&](int k, int n) { return Tdg(0, k, n); }, lane);
+              warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                        [&](int k, int n) { return Tlo(1, 0, k, n); }, lane);
+            } else {
+              warp_mm16(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                        [&](int k, int n) { return Tdg(1, k, n); }, lane);
+            }
+            float* xs = X + pw * 320;
+            warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
+              *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
           }
-          float* xs = X + pw * 320;
-          warp_put16(acc, 1.f, [&](int r, int k, float v0, float v1) {
-            *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, lane);
-        }
-        named_bar<kTeamA, 128>();
-        {
-          // X2 block (mm, b2) sits in X slot 2 (mm - 2) + b2
-          float acc[3][2][4] = {};
-          if (i2 == 2) {
-            warp_mm16(acc, [&](int r, int k) { return Tdg(2, r, k); },
-                      [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
-          } else {
-            warp_mm16(acc, [&](int r, int k) { return Tlo(3, 2, r, k); },
-                      [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
-            warp_mm16(acc, [&](int r, int k) { return Tdg(3, r, k); },
-                      [&](int k, int n) { return X[(2 + b2) * 320 + k * 20 + n]; }, lane);
+          named_bar<kTeamA, 128>();
+          {
+            // X2 block (mm, b2) sits in X slot 2 (mm - 2) + b2
+            float acc[3][2][4] = {};
+            if (i2 == 2) {
+              warp_mm16(acc, [&](int r, int k) { return Tdg(2, r, k); },
+                        [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
+            } else {
+              warp_mm16(acc, [&](int r, int k) { return Tlo(3, 2, r, k); },
+                        [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, lane);
+              warp_mm16(acc, [&](int r, int k) { return Tdg(3, r, k); },
+                        [&](int k, int n) { return X[(2 + b2) * 320 + k * 20 + n]; }, lane);
+            }
+            warp_put16(acc, -1.f, [&](int r, int k, float v0, float v1) {
+              Top(i2, b2, r, k, v0, v1); }, lane);
           }
-          warp_put16(acc, -1.f, [&](int r, int k, float v0, float v1) {
-            Top(i2, b2, r, k, v0, v1); }, lane);
+          fence_async_smem();
+          named_bar<kTeamA, 128>();
+          if (ptid == 0) mbar_arrive(t_ready);
         }
-        fence_async_smem();
-        named_bar<kTeamA, 128>();
-        if (ptid == 0) mbar_arrive(t_ready);
       } else if (c + 1 < nchunks) {
         // ---- the next chunk's scalars (warps 12-15)
         if (warp == 13) {
@@ -2142,12 +2181,52 @@ chunk_engine_ws_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (warp == 12) decay_and_variance(c + 1);
         }
       }
+      if constexpr (!DIAG) {
+        // ---- isotropic: X2 = A^(10) T^(0), then T^(10) = -T^(1) X2, on all
+        // eight prep warps (the next chunk's scalars take warps 12-15 only a
+        // part of the T solve): warp pw takes n-tile pw >> 2 of the 16x16
+        // block pw & 3; X2 block (mm, b2) sits in X slot 2 (mm - 2) + b2
+        const int blk = pw & 3, nt = pw >> 2;
+        const int i2 = 2 + (blk >> 1), b2 = blk & 1;
+        bar_group(kPrepBar);  // T's diagonal and level-1 blocks are in AT
+        {
+          float acc[3][4] = {};
+          if (b2 == 0) {
+            warp_mm16n(acc, [&](int r, int k) { return Ael(i2, 0, r, k); },
+                       [&](int k, int n) { return Tdg(0, k, n); }, nt, lane);
+            warp_mm16n(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                       [&](int k, int n) { return Tlo(1, 0, k, n); }, nt, lane);
+          } else {
+            warp_mm16n(acc, [&](int r, int k) { return Ael(i2, 1, r, k); },
+                       [&](int k, int n) { return Tdg(1, k, n); }, nt, lane);
+          }
+          float* xs = X + blk * 320;
+          warp_put16n(acc, 1.f, [&](int r, int k, float v0, float v1) {
+            *reinterpret_cast<float2*>(xs + r * 20 + k) = make_float2(v0, v1); }, nt, lane);
+        }
+        bar_group(kPrepBar);
+        {
+          float acc[3][4] = {};
+          if (i2 == 2) {
+            warp_mm16n(acc, [&](int r, int k) { return Tdg(2, r, k); },
+                       [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, nt, lane);
+          } else {
+            warp_mm16n(acc, [&](int r, int k) { return Tlo(3, 2, r, k); },
+                       [&](int k, int n) { return X[b2 * 320 + k * 20 + n]; }, nt, lane);
+            warp_mm16n(acc, [&](int r, int k) { return Tdg(3, r, k); },
+                       [&](int k, int n) { return X[(2 + b2) * 320 + k * 20 + n]; }, nt, lane);
+          }
+          warp_put16n(acc, -1.f, [&](int r, int k, float v0, float v1) {
+            Top(i2, b2, r, k, v0, v1); }, nt, lane);
+        }
+      }
 
       fence_async_smem();
       if (bar_group_or(kPrepBar, bad || *sc_abort != 0.f)) {
         bad = true;
         break;
       }
+      if (!DIAG && ptid == 0) mbar_arrive(t_ready);
       if (ptid == 0) mbar_arrive(p_ready);
     }
     if (mma1_issuer && pend_mma1 >= 0) (void)mbar_wait(mma1_bar, (uint32_t)pend_mma1);

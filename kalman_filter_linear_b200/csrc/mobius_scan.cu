@@ -101,7 +101,52 @@ __device__ __forceinline__ Mat2 as_mat(const float4& f) { return {f.x, f.y, f.z,
 struct TileShared {
   Mat2 warp_incl[kThreads / 32];
   Mat2 tile_prefix;
+  Mat2 pred_incl;    // the predecessor's inclusive prefix, when published
+  uint32_t pred_ok;  // 1: it was published when this tile started
 };
+
+// The decoupled look-back of tile `tile` (index j in lane seq) whose
+// predecessor had not published its inclusive prefix when the tile started
+// (its flag then: f_pre): publish the aggregate, combine the predecessors'
+// aggregates back to the first inclusive prefix, publish this tile's.
+// Returns the tile's exclusive prefix.
+__device__ __forceinline__ Mat2 look_back(const ScanWs& ws, int64_t tile, int64_t j, int64_t seq,
+                                       int64_t N, uint32_t f_pre, Mat2 agg, bool skip_publish) {
+  Mat2 excl = identity();
+  if (!skip_publish) {
+    ws.agg[tile] = as_f4(agg);
+    st_release_u32(ws.flag + tile, 1u);
+  }
+  const uint64_t start = globaltimer_ns();
+  bool timed_out = false;
+  uint32_t f0 = f_pre;
+  for (int64_t p = j - 1; p >= 0 && !timed_out;) {
+    const int64_t pt = p * N + seq;
+    uint32_t f = (p == j - 1) ? f0 : ld_acquire_u32(ws.flag + pt);
+    while (f == 0u) {
+      if (globaltimer_ns() - start > kWaitLimitNs) {
+        timed_out = true;
+        break;
+      }
+      __nanosleep(64);
+      f = ld_acquire_u32(ws.flag + pt);
+    }
+    if (timed_out) break;
+    if (f == 2u) {
+      excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
+      break;
+    }
+    excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
+    f0 = 0u;
+    --p;
+  }
+  if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
+  if (!skip_publish) {
+    ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
+    st_release_u32(ws.flag + tile, 2u);
+  }
+  return excl;
+}
 
 // Steps 1-4 for one tile, given this thread's 8 inputs (a, w, r, n).
 __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const float (&w)[kPerThread],
@@ -150,82 +195,53 @@ __device__ __forceinline__ void scan_tile(const float (&a)[kPerThread], const fl
     if (lane >= d) incl = renorm(mul(incl, prev));
   }
   if (lane == 31) s_warp[warp] = incl;
-  __syncthreads();
-  // ---- block scan of the warp totals and 3. the decoupled look-back, both
-  // in warp 0 (the other warps wait at the next barrier).  The release store
-  // of a flag orders this thread's earlier stores of the prefix data before it.
-  if (warp == 0) {
-    Mat2 x = lane < kThreads / 32 ? s_warp[lane] : identity();
-#pragma unroll
-    for (int d = 1; d < kThreads / 32; d <<= 1) {
-      const Mat2 prev = shfl_up(x, d);
-      if (lane >= d) x = renorm(mul(x, prev));
-    }
-    if (lane < kThreads / 32) s_warp[lane] = x;  // inclusive over warps
-    const Mat2 tot = {__shfl_sync(0xffffffffu, x.a, kThreads / 32 - 1),
-                      __shfl_sync(0xffffffffu, x.b, kThreads / 32 - 1),
-                      __shfl_sync(0xffffffffu, x.c, kThreads / 32 - 1),
-                      __shfl_sync(0xffffffffu, x.d, kThreads / 32 - 1)};
-    if (tid == 0) {
-      const Mat2 agg = tot;
-      Mat2 excl = identity();
-      const bool skip_publish = (tile == debug_skip_tile);  // fault-injection hook
-      if (j == 0) {
-        if (!skip_publish) {
-          ws.incl[tile] = as_f4(agg);
-          st_release_u32(ws.flag + tile, 2u);
-        }
-      } else {
-        // Usually the predecessor has finished: take its inclusive prefix and
-        // publish only this tile's.  Otherwise publish the aggregate first and
-        // look back tile by tile.
-        uint32_t f0 = f_pre;
-        if (f0 != 2u) {
-          if (!skip_publish) {
-            ws.agg[tile] = as_f4(agg);
-            st_release_u32(ws.flag + tile, 1u);
-          }
-          const uint64_t start = globaltimer_ns();
-          bool timed_out = false;
-          for (int64_t p = j - 1; p >= 0 && !timed_out;) {
-            const int64_t pt = p * N + seq;
-            uint32_t f = (p == j - 1) ? f0 : ld_acquire_u32(ws.flag + pt);
-            while (f == 0u) {
-              if (globaltimer_ns() - start > kWaitLimitNs) {
-                timed_out = true;
-                break;
-              }
-              __nanosleep(64);
-              f = ld_acquire_u32(ws.flag + pt);
-            }
-            if (timed_out) break;
-            if (f == 2u) {
-              excl = renorm(mul(excl, as_mat(__ldcg(ws.incl + pt))));
-              break;
-            }
-            excl = renorm(mul(excl, as_mat(__ldcg(ws.agg + pt))));
-            f0 = 0u;
-            --p;
-          }
-          if (timed_out) atomicOr(ws.error, DEV_TIMEOUT);
-        } else {
-          excl = as_mat(incl_pre);
-        }
-        if (!skip_publish) {
-          ws.incl[tile] = as_f4(renorm(mul(agg, excl)));
-          st_release_u32(ws.flag + tile, 2u);
-        }
-      }
-      sh.tile_prefix = excl;
-    }
+  if (tid == 0) {
+    sh.pred_ok = (j == 0 || f_pre == 2u) ? 1u : 0u;
+    sh.pred_incl = j == 0 ? identity() : as_mat(incl_pre);
   }
   __syncthreads();
-
-  // ---- 4. apply the exclusive prefix and run the recursion
+  // ---- block scan of the warp totals, in every warp.  Warp 0 takes the
+  // tile's aggregate from it (its thread 0 publishes), every other warp the
+  // product over the warps before it.
+  Mat2 x = lane < kThreads / 32 ? s_warp[lane] : identity();
+#pragma unroll
+  for (int d = 1; d < kThreads / 32; d <<= 1) {
+    const Mat2 prev = shfl_up(x, d);
+    if (lane >= d) x = renorm(mul(x, prev));
+  }
+  const int src = warp > 0 ? warp - 1 : kThreads / 32 - 1;
+  const Mat2 blk = {__shfl_sync(0xffffffffu, x.a, src), __shfl_sync(0xffffffffu, x.b, src),
+                    __shfl_sync(0xffffffffu, x.c, src), __shfl_sync(0xffffffffu, x.d, src)};
+  const Mat2& agg = blk;  // (warp 0)
+  // this thread's prefix within the tile (warps 1-7: blk is the product over
+  // the warps before)
   Mat2 thread_excl = shfl_up(incl, 1);
   if (lane == 0) thread_excl = identity();
-  if (warp > 0) thread_excl = mul(thread_excl, s_warp[warp - 1]);
-  thread_excl = renorm(mul(renorm(thread_excl), sh.tile_prefix));
+  if (warp > 0) thread_excl = mul(thread_excl, blk);
+  thread_excl = renorm(thread_excl);
+  // ---- 3. the tile's prefix.  Usually the predecessor had published its
+  // inclusive prefix when this tile started (thread 0 read it then): every
+  // thread takes it from shared memory and no second barrier is needed.
+  // Otherwise thread 0 publishes the aggregate and looks back tile by tile
+  // while the others wait at a barrier (the choice is the same in every
+  // thread: all read one shared flag).  The release store of a flag orders
+  // this thread's earlier stores of the prefix data before it.
+  const bool skip_publish = (tile == debug_skip_tile);  // fault-injection hook
+  Mat2 tile_prefix;
+  if (sh.pred_ok) {
+    tile_prefix = sh.pred_incl;
+    if (tid == 0 && !skip_publish) {
+      ws.incl[tile] = as_f4(j == 0 ? agg : renorm(mul(agg, tile_prefix)));
+      st_release_u32(ws.flag + tile, 2u);
+    }
+  } else {
+    if (tid == 0) sh.tile_prefix = look_back(ws, tile, j, seq, N, f_pre, agg, skip_publish);
+    __syncthreads();
+    tile_prefix = sh.tile_prefix;
+  }
+
+  // ---- 4. apply the exclusive prefix and run the recursion
+  thread_excl = renorm(mul(thread_excl, tile_prefix));
   const float lam0 = lambda0 ? __ldg(lambda0 + seq) : 1.f;
   float lam = apply(thread_excl, lam0);
 

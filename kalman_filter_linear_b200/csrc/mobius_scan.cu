@@ -13,12 +13,16 @@
 //   1. 256 threads load 8 consecutive steps each (two 16-byte loads per
 //      array), build their maps and compose them serially in registers;
 //   2. warp-shuffle inclusive scan of the thread products, then a block scan
-//      of the 8 warp totals in shared memory;
+//      of the 8 warp totals (through shared memory, one barrier; every warp
+//      scans them itself);
 //   3. decoupled look-back across the tiles of the lane: a tile publishes its
-//      aggregate, then its inclusive prefix; a successor combines the
-//      published values of its predecessors.  Tiles are handed out by an
-//      atomic counter in tile-index-major order (all lanes' tile 0 first),
-//      so a predecessor has almost always finished already.  Every wait is
+//      inclusive prefix at once when its predecessor's was published as the
+//      tile started (the usual case), else its aggregate first, then the
+//      inclusive prefix once it has combined the predecessors' published
+//      values (thread 0, while the other threads wait at a second barrier).
+//      Tiles are handed out by an atomic counter in tile-index-major order
+//      (all lanes' tile 0 first), so a predecessor has almost always
+//      finished already.  Every wait is
 //      bounded in wall-clock time; a wait that gives up records
 //      DEV_TIMEOUT in the workspace error word and the tile goes on with
 //      what it has.
